@@ -1,0 +1,270 @@
+/*
+ * gdn_oracle.c -- plain, slow, fp64 CPU oracle of the Gated DeltaNet gated delta rule.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the library (gated_deltanet_05_b200/) calls,
+ * links or includes this file; only the tests, __graft_entry__.smoke() and the CPU
+ * baseline leg of bench.py use it. It shares no source with the CUDA path.
+ *
+ * What it computes (joezjh.github.io notes page "Qwen3.8-Flash-Next", section
+ * "Gated DeltaNet 核心机制", the four-line update rule): per head, with the state
+ * S in R^{d_k x d_v} (the pages' orientation, row index = key dimension),
+ *
+ *     S~      = alpha_t * S_{t-1}                 (decay first)
+ *     e_t     = v_t - S~^T k_t                    (error against the decayed state)
+ *     S_t     = S~ + beta_t * k_t e_t^T           (rank-one write of the error)
+ *     y_t     = S_t^T (scale * q_t)               (read AFTER the write)
+ *
+ * token by token, one (sequence, head) chain at a time, in the order of the pages.
+ * The `scale` factor multiplies q; the pages use none, so every workload passes 1.
+ *
+ * The output epilogue (same page, section "GDN 参数化细节", output-gate equation, and
+ * the pwwt.cn translation, section 2.1.1, "sigmoid output gate ... zero-centred
+ * RMSNorm") is o = sigmoid(z) * RMSNorm(y), with RMSNorm taken per (token, head)
+ * over d_v and the zero-centred weight stored as w, multiplying as (1 + w).
+ *
+ * All arithmetic is IEEE fp64 in the order written; build without -ffast-math.
+ * Chains are independent, so they are spread over POSIX threads; each chain's
+ * arithmetic is the same whatever the thread count.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* ------------------------------------------------------------------ prefill */
+
+typedef struct {
+    const double *q, *k, *v, *log_alpha, *beta, *S0;
+    const int64_t *cu_seqlens;
+    int n_seq, H, dk, dv;
+    double scale;
+    double *y, *S_T;
+    /* work distribution */
+    int n_threads, tid;
+} rec_args;
+
+/* One chain: sequence i, head h. S is d_k x d_v, row-major (S[a*dv + b] = S_{a,b}). */
+static void recurrent_chain(const rec_args *A, int i, int h, double *S, double *e, double *qs)
+{
+    const int H = A->H, dk = A->dk, dv = A->dv;
+    const int64_t bos = A->cu_seqlens[i], eos = A->cu_seqlens[i + 1];
+    const size_t state_off = ((size_t)i * H + h) * (size_t)dk * dv;
+
+    if (A->S0)
+        memcpy(S, A->S0 + state_off, sizeof(double) * dk * dv);
+    else
+        memset(S, 0, sizeof(double) * dk * dv);
+
+    for (int64_t t = bos; t < eos; ++t) {
+        const double *kt = A->k + ((size_t)t * H + h) * dk;
+        const double *qt = A->q + ((size_t)t * H + h) * dk;
+        const double *vt = A->v + ((size_t)t * H + h) * dv;
+        const double alpha = exp(A->log_alpha[(size_t)t * H + h]);
+        const double beta = A->beta[(size_t)t * H + h];
+
+        /* S~ = alpha * S */
+        for (int a = 0; a < dk * dv; ++a)
+            S[a] *= alpha;
+        /* e = v - S~^T k : e_b = v_b - sum_a S~_{a,b} k_a */
+        for (int b = 0; b < dv; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < dk; ++a)
+                acc += S[a * dv + b] * kt[a];
+            e[b] = vt[b] - acc;
+        }
+        /* S = S~ + beta k e^T */
+        for (int a = 0; a < dk; ++a)
+            for (int b = 0; b < dv; ++b)
+                S[a * dv + b] += beta * kt[a] * e[b];
+        /* y = S^T (scale q) */
+        for (int a = 0; a < dk; ++a)
+            qs[a] = A->scale * qt[a];
+        double *yt = A->y + ((size_t)t * H + h) * dv;
+        for (int b = 0; b < dv; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < dk; ++a)
+                acc += S[a * dv + b] * qs[a];
+            yt[b] = acc;
+        }
+    }
+    if (A->S_T)
+        memcpy(A->S_T + state_off, S, sizeof(double) * dk * dv);
+}
+
+static void *recurrent_worker(void *p)
+{
+    const rec_args *A = (const rec_args *)p;
+    double *S = (double *)malloc(sizeof(double) * A->dk * A->dv);
+    double *e = (double *)malloc(sizeof(double) * A->dv);
+    double *qs = (double *)malloc(sizeof(double) * A->dk);
+    if (S && e && qs) {
+        const int n_chain = A->n_seq * A->H;
+        for (int c = A->tid; c < n_chain; c += A->n_threads)
+            recurrent_chain(A, c / A->H, c % A->H, S, e, qs);
+    }
+    free(S);
+    free(e);
+    free(qs);
+    return NULL;
+}
+
+static int resolve_threads(int n_threads, int n_work)
+{
+    if (n_threads <= 0) {
+        long n = sysconf(_SC_NPROCESSORS_ONLN);
+        n_threads = n > 0 ? (int)n : 1;
+    }
+    if (n_threads > n_work)
+        n_threads = n_work > 0 ? n_work : 1;
+    return n_threads;
+}
+
+/*
+ * Token recurrence over packed variable-length sequences.
+ *   q, k      [N_tok][H][dk]      (N_tok = cu_seqlens[n_seq])
+ *   v         [N_tok][H][dv]
+ *   log_alpha [N_tok][H]          alpha_t = exp(log_alpha)
+ *   beta      [N_tok][H]
+ *   S0        [n_seq][H][dk][dv]  or NULL for zeros (the pages' orientation)
+ *   y         [N_tok][H][dv]      out
+ *   S_T       [n_seq][H][dk][dv]  out, or NULL
+ * Returns the number of threads used (>= 1), or -1 on a bad argument.
+ */
+int gdn_oracle_recurrent(const double *q, const double *k, const double *v,
+                         const double *log_alpha, const double *beta, const double *S0,
+                         const int64_t *cu_seqlens, int n_seq, int H, int dk, int dv,
+                         double scale, double *y, double *S_T, int n_threads)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !cu_seqlens || !y || n_seq < 0 || H <= 0 ||
+        dk <= 0 || dv <= 0)
+        return -1;
+    const int n_chain = n_seq * H;
+    n_threads = resolve_threads(n_threads, n_chain);
+    rec_args *args = (rec_args *)calloc((size_t)n_threads, sizeof(rec_args));
+    pthread_t *th = (pthread_t *)calloc((size_t)n_threads, sizeof(pthread_t));
+    if (!args || !th) {
+        free(args);
+        free(th);
+        return -1;
+    }
+    for (int i = 0; i < n_threads; ++i) {
+        rec_args a = {q, k, v, log_alpha, beta, S0, cu_seqlens, n_seq, H, dk, dv, scale,
+                      y, S_T, n_threads, i};
+        args[i] = a;
+    }
+    for (int i = 1; i < n_threads; ++i)
+        pthread_create(&th[i], NULL, recurrent_worker, &args[i]);
+    recurrent_worker(&args[0]);
+    for (int i = 1; i < n_threads; ++i)
+        pthread_join(th[i], NULL);
+    free(args);
+    free(th);
+    return n_threads;
+}
+
+/* ------------------------------------------------------------------- decode */
+
+/*
+ * One token for each of n_chain = n_seq*H independent chains (same update as above,
+ * alpha given directly instead of its log).
+ *   q, k [n_chain][dk]; v [n_chain][dv]; alpha, beta [n_chain]
+ *   S    [n_chain][dk][dv]  updated in place (the pages' orientation)
+ *   y    [n_chain][dv]      out
+ */
+typedef struct {
+    const double *q, *k, *v, *alpha, *beta;
+    double *S, *y;
+    int n_chain, dk, dv;
+    double scale;
+    int n_threads, tid;
+} dec_args;
+
+static void *decode_worker(void *p)
+{
+    const dec_args *A = (const dec_args *)p;
+    const int dk = A->dk, dv = A->dv;
+    double *e = (double *)malloc(sizeof(double) * dv);
+    if (!e)
+        return NULL;
+    for (int c = A->tid; c < A->n_chain; c += A->n_threads) {
+        double *S = A->S + (size_t)c * dk * dv;
+        const double *kt = A->k + (size_t)c * dk, *qt = A->q + (size_t)c * dk;
+        const double *vt = A->v + (size_t)c * dv;
+        const double alpha = A->alpha[c], beta = A->beta[c];
+        for (int a = 0; a < dk * dv; ++a)
+            S[a] *= alpha;
+        for (int b = 0; b < dv; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < dk; ++a)
+                acc += S[a * dv + b] * kt[a];
+            e[b] = vt[b] - acc;
+        }
+        for (int a = 0; a < dk; ++a)
+            for (int b = 0; b < dv; ++b)
+                S[a * dv + b] += beta * kt[a] * e[b];
+        double *yt = A->y + (size_t)c * dv;
+        for (int b = 0; b < dv; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < dk; ++a)
+                acc += S[a * dv + b] * (A->scale * qt[a]);
+            yt[b] = acc;
+        }
+    }
+    free(e);
+    return NULL;
+}
+
+int gdn_oracle_decode_step(const double *q, const double *k, const double *v,
+                           const double *alpha, const double *beta, double *S, double *y,
+                           int n_chain, int dk, int dv, double scale, int n_threads)
+{
+    if (!q || !k || !v || !alpha || !beta || !S || !y || n_chain < 0 || dk <= 0 || dv <= 0)
+        return -1;
+    n_threads = resolve_threads(n_threads, n_chain);
+    dec_args *args = (dec_args *)calloc((size_t)n_threads, sizeof(dec_args));
+    pthread_t *th = (pthread_t *)calloc((size_t)n_threads, sizeof(pthread_t));
+    if (!args || !th) {
+        free(args);
+        free(th);
+        return -1;
+    }
+    for (int i = 0; i < n_threads; ++i) {
+        dec_args a = {q, k, v, alpha, beta, S, y, n_chain, dk, dv, scale, n_threads, i};
+        args[i] = a;
+    }
+    for (int i = 1; i < n_threads; ++i)
+        pthread_create(&th[i], NULL, decode_worker, &args[i]);
+    decode_worker(&args[0]);
+    for (int i = 1; i < n_threads; ++i)
+        pthread_join(th[i], NULL);
+    free(args);
+    free(th);
+    return n_threads;
+}
+
+/* ---------------------------------------------------------------- gate-norm */
+
+/*
+ * o[r][j] = sigmoid(z[r][j]) * y[r][j] / sqrt(mean_j y[r][j]^2 + eps) * (1 + w[j])
+ * for r < n_rows (= N_tok * H), j < dv. Row-local, single threaded.
+ */
+int gdn_oracle_gate_norm(const double *y, const double *z, const double *w, int64_t n_rows,
+                         int dv, double eps, double *o)
+{
+    if (!y || !z || !w || !o || n_rows < 0 || dv <= 0)
+        return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const double *yr = y + (size_t)r * dv, *zr = z + (size_t)r * dv;
+        double ss = 0.0;
+        for (int j = 0; j < dv; ++j)
+            ss += yr[j] * yr[j];
+        const double inv_rms = 1.0 / sqrt(ss / dv + eps);
+        for (int j = 0; j < dv; ++j) {
+            const double gate = 1.0 / (1.0 + exp(-zr[j]));
+            o[(size_t)r * dv + j] = gate * (yr[j] * inv_rms) * (1.0 + w[j]);
+        }
+    }
+    return 1;
+}
