@@ -1,0 +1,483 @@
+"""Benchmark of the gated delta rule hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = chunked prefill (gdn_chunk_fwd) + the sigmoid-gate zero-centred RMSNorm
+epilogue (gdn_gate_norm) over one batch of the prefill workload: 4 sequences x 4096
+tokens, H = 16, d_k = d_v = 128, chunk 64, bf16 q/k/v, fp32 state. Inputs are seeded
+synthetic draws (workloads/), resident in HBM before the timed region; q, k, v and z
+(256 MiB) exceed the 126 MB L2, so no flush is needed between steps.
+
+The decode step (256 sequences x 32 heads, d = 128, 537 MB fp32 state in HBM) is timed
+separately and reported under "decode".
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent batch
+(the chains do not interact), so scaling is weak and the data path has no collective;
+timing is the max over ranks of the device-timed region.
+
+--impl reference runs the fp64 CPU oracle on the host cores (rank 0 only) on bounded
+samples of the same workload; it is the slow reference arm, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s + % tensor peak; decode-step state GB/s vs HBM peak"
+UNIT = "tokens/s"
+WORKLOAD = ("prefill bf16: 4 seqs x 4096 tokens, H=16, d_k=d_v=128, chunk 64, fp32 state, "
+            "fp32 y, then sigmoid-gate zero-centred RMSNorm (bf16 z and o)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["gated_deltanet_05_b200/csrc/gdn_chunk_sm100.cuh",
+                  "gated_deltanet_05_b200/csrc/sm100_ptx.cuh"]
+
+
+def flops_per_token_head(chunk: int, d: int) -> float:
+    """Canonical chunked-form FLOPs per (token, head), full C x C tiles: five C x d
+    products at 2Cd (K K^T, Q K^T, T K, T V, P U~), three d x d products at 2d^2
+    (W S, Q S, state update) and the C x C solve at C^2/3."""
+    return 10.0 * chunk * d + 6.0 * d * d + chunk * chunk / 3.0
+
+
+def prefill_bytes_per_token_head(in_elem: int, y_elem: int, d: int) -> float:
+    """Minimal HBM bytes per (token, head): read q, k, v (3 d in_elem), write y (d y_elem),
+    read log_alpha and beta (8 bytes)."""
+    return 3 * in_elem * d + y_elem * d + 8.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the prefill kernel from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "chunk_fwd_bf16_prefill.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled in the background."""
+
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(", ") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 10:
+                continue
+            try:
+                sm.append(float(r[2]))
+                mx = float(r[3])
+            except ValueError:
+                continue
+            for n, val in zip(names, r[6:10]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    elif args.impl == "ours":
+        torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def max_over_ranks(pg, value: float, device):
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device=None):
+    if pg is not None:
+        if device is not None:
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(inp, seq_heads, n_threads=0):
+    """Run the fp64 oracle on the given (sequence, head) chains of a prefill input;
+    returns (token-heads processed, seconds, threads used)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    seqs = sorted({s for s, _ in seq_heads})
+    heads = sorted({h for _, h in seq_heads})
+    cu = inp["cu_seqlens"].tolist()
+    idx = torch.from_numpy(np.concatenate([np.arange(cu[s], cu[s + 1]) for s in seqs]))
+    hs = torch.tensor(heads)
+    sel = {k: inp[k].index_select(0, idx).index_select(1, hs)
+           for k in ("q", "k", "v", "log_alpha", "beta")}
+    lens = [cu[s + 1] - cu[s] for s in seqs]
+    cu_sub = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    t0 = time.perf_counter()
+    _, _, used = oracle.recurrent(sel["q"], sel["k"], sel["v"], sel["log_alpha"], sel["beta"],
+                                  cu_sub, n_threads=n_threads)
+    dt = time.perf_counter() - t0
+    return int(sum(lens)) * len(heads), dt, used
+
+
+def run_reference(args, rank, world, pg):
+    if rank != 0:
+        return
+    import workloads as W
+    w = W.WORKLOADS["prefill"]
+    inp = W.make_prefill_inputs(w, with_gate=False)
+    cores = os.cpu_count() or 1
+    H = w.H
+    n_seq = len(w.lengths)
+    # one step = one bounded sample: `cores` chains (whole sequences), rotating over the batch
+    chains = [(s, h) for h in range(H) for s in range(n_seq)]
+    per_step = max(1, min(cores, len(chains)))
+    done, elapsed, used = 0, 0.0, 1
+    for i in range(args.warmup + args.steps):
+        pick = [chains[(i * per_step + j) % len(chains)] for j in range(per_step)]
+        # a square sample: every listed sequence with every listed head
+        seqs = sorted({s for s, _ in pick})
+        heads = sorted({h for _, h in pick})
+        n_th, dt, used = oracle_sample(inp, [(s, h) for s in seqs for h in heads])
+        if i >= args.warmup:
+            done += n_th
+            elapsed += dt
+    th_per_s = done / elapsed
+    value = th_per_s / H
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 4, "seq_len": 4096, "heads": 16,
+                   "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                         "sample": f"per step: whole 4096-token chains of the prefill workload, "
+                                   f"{per_step} (sequence, head) pairs; {done} token-heads timed"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local, pg):
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    import workloads as W
+
+    device = torch.device("cuda", local)
+    w = W.WORKLOADS["prefill"]
+    H, d, C = w.H, w.d_k, w.chunk
+    inp = W.make_prefill_inputs(w, seed=w.seed + 1000 * rank)
+    n_tok = int(inp["cu_seqlens"][-1])
+    dev = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    cu_host = inp["cu_seqlens"]
+    y = torch.empty((n_tok, H, d), dtype=torch.float32, device=device)
+    o = torch.empty((n_tok, H, d), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                      dev["cu_seqlens"], chunk=C, cu_seqlens_host=cu_host, out=y,
+                      final_state=True)
+        if ev is not None:
+            ev[1].record(stream)
+        gdn.gate_norm(y, dev["z"], dev["w_norm"], out=o)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    status = gdn.device_error(device)
+    if status != "GDN_OK":
+        raise SystemExit(f"device error after warm-up: {status}")
+
+    # timed region: K steps, per-kernel events inside
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local).start()
+    time.sleep(0.2)
+    barrier(pg, device)
+    torch.cuda.synchronize(device)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(pg, device)
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(pg, elapsed_ms, device)
+    chunk_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    gn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_step = n_tok * world
+    value = tokens_per_step / (ms_per_step * 1e-3)
+
+    peaks, peak_kind = load_peaks()
+    token_heads = n_tok * H
+    flops = flops_per_token_head(C, d) * token_heads
+    algo_bytes = prefill_bytes_per_token_head(2, 4, d) * token_heads + len(w.lengths) * H * d * d * 4
+    chunk_s = chunk_ms * 1e-3
+    tflops = flops / chunk_s / 1e12
+    gbs = algo_bytes / chunk_s / 1e9
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = algo_bytes / (peaks["hbm_gbs"] * 1e9)
+    roofline = {
+        "kernel": "gdn::sm100::chunk_fwd_bf16_kernel",
+        "bound": "hbm" if t_hbm >= t_tensor else "tensor",
+        "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+        "traffic": profiled_traffic(),
+        "algorithmic_bytes_per_launch": algo_bytes,
+        "launch_ms": chunk_ms,
+        "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                   "frac": tflops / peaks["bf16_tflops"],
+                   "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                   "flops_per_launch": flops,
+                   "flops_per_token_head": flops_per_token_head(C, d)},
+    }
+    gn_bytes = (4 + 2 + 2) * n_tok * H * d + 4 * d          # y fp32, z and o bf16
+    gate_norm_obj = {"launch_ms": gn_ms, "achieved": gn_bytes / (gn_ms * 1e-3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gn_bytes / (gn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "bytes_per_launch": gn_bytes}
+
+    decode = None if args.no_decode else bench_decode(args, device, peaks, peak_kind, pg)
+    e2e = bench_e2e(args, inp, device, pg, world)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded draws: L2-normalised q,k ~ N(0,1); v ~ N(0,1); "
+                "beta = sigmoid(N(0,1)); log alpha = -exp(A) softplus(N(0,1)), A ~ U(-1,1))",
+        "config": {"workload": WORKLOAD, "global_batch": 4 * world, "seq_len": 4096,
+                   "heads": H, "d_k": d, "d_v": d, "chunk": C, "parallelism": f"dp{world}",
+                   "l2": "no flush: q, k, v, z are 256 MiB per step, above the 126 MB L2"},
+        "roofline": roofline,
+        "gate_norm": gate_norm_obj,
+        "decode": decode,
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(inp, H)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_decode(args, device, peaks, peak_kind, pg):
+    """Decode step: 256 sequences x 32 heads, d = 128, fp32 state resident in HBM."""
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    import workloads as W
+    w = W.WORKLOADS["decode"]
+    n, H, d = w.n_seq_decode, w.H, w.d_k
+    n_inputs = 8                                    # distinct staged steps, cycled
+    staged = []
+    for s in range(n_inputs):
+        x = W.make_decode_inputs(w, s)
+        staged.append({k: v.to(device) for k, v in x.items()})
+    S = torch.zeros((n, H, d, d), dtype=torch.float32, device=device)
+    y = torch.empty((n, H, d), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def one(i):
+        x = staged[i % n_inputs]
+        gdn.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S, out=y)
+
+    for i in range(max(3, args.warmup)):
+        one(i)
+    torch.cuda.synchronize(device)
+    steps = max(args.steps, 50)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(pg, device)
+    a.record(stream)
+    for i in range(steps):
+        one(i)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(pg, a.elapsed_time(b), device) / steps
+    state_bytes = n * H * d * d * 4
+    step_bytes = 2 * state_bytes + n * H * (3 * d * 4 + d * 4 + 8)
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    return {"workload": "decode fp32 state: 256 seqs x H=32, d_k=d_v=128, one token per step",
+            "ms_per_step": ms, "tokens_per_s": n / (ms * 1e-3), "bytes_per_step": step_bytes,
+            "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+            "steps": steps, "l2": "state 537 MB > L2"}
+
+
+def bench_e2e(args, inp, device, pg, world):
+    """Same step through the public API with the inputs in pinned host memory: H2D copy of
+    q, k, v, log_alpha, beta, z every step, D2H read of the output o."""
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    H, C = inp["H"], inp["chunk"]
+    host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "log_alpha", "beta", "z")}
+    w_dev = inp["w_norm"].to(device)
+    cu_host = inp["cu_seqlens"]
+    cu_dev = cu_host.to(device)
+    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
+    o_host = torch.empty(inp["v"].shape, dtype=inp["v"].dtype).pin_memory()
+    stream = torch.cuda.current_stream(device)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def step():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        y, _ = gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], cu_dev,
+                             chunk=C, cu_seqlens_host=cu_host)
+        o = gdn.gate_norm(y, dev["z"], w_dev, out_dtype=torch.bfloat16)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(device)
+    steps = max(1, min(args.steps, 20))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(pg, device)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(pg, a.elapsed_time(b), device) / steps
+    n_tok = inp["q"].shape[0]
+    return {"value": n_tok * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def cpu_baseline(inp, H):
+    """The fp64 oracle on the host cores over a bounded sample of the same workload."""
+    cores = os.cpu_count() or 1
+    n_seq = inp["cu_seqlens"].numel() - 1
+    heads = list(range(min(H, max(1, cores // n_seq + 1))))
+    pairs = [(s, h) for s in range(n_seq) for h in heads]
+    n_th, dt, used = oracle_sample(inp, pairs)
+    return {"value": n_th / dt / H, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{len(pairs)} whole 4096-token (sequence, head) chains of the prefill "
+                      f"workload ({n_th} token-heads, {dt:.1f} s); tokens/s = token-heads/s / H"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local, pg = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world, pg)
+        else:
+            run_ours(args, rank, world, local, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+"""gated_deltanet_05_b200 -- Python binding of libgdn_b200.so, the B200 gated delta rule library.
+
+Argument marshalling only: every computation runs in the library's CUDA kernels
+(see include/gdn.h for the C ABI). PyTorch supplies device memory and the current
+stream. There is no CPU path: if the shared library is missing or fails to load,
+importing works but every call raises RuntimeError.
+
+    y, S_T = chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64)
+    y = decode_step(q, k, v, alpha, beta, S)          # S updated in place
+    o = gate_norm(y, z, w, eps=1e-6)
+
+State tensors use the library's value-major layout [.., d_v, d_k] in fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["chunk_fwd", "decode_step", "gate_norm", "device_error", "lib", "LIB_PATH",
+           "GdnError", "EXPORTED_SYMBOLS", "STATUS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn_b200.so")
+
+STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
+          4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_DEVICE_CHECK"}
+GDN_F32, GDN_BF16 = 0, 1
+
+EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_decode_step",
+                    "gdn_gate_norm", "gdn_status_string", "gdn_device_error", "gdn_version")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+_load_error = None
+
+
+def lib():
+    """The loaded ctypes library (raises RuntimeError if it cannot be loaded)."""
+    global _lib, _load_error
+    if _lib is None:
+        if _load_error is not None:
+            raise RuntimeError(_load_error)
+        try:
+            L = ctypes.CDLL(LIB_PATH)
+        except OSError as e:
+            _load_error = (f"libgdn_b200.so could not be loaded from {LIB_PATH} ({e}); build it "
+                           "with `python -m gated_deltanet_05_b200.build`")
+            raise RuntimeError(_load_error) from None
+        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        L.gdn_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
+        L.gdn_chunk_fwd_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32]
+        L.gdn_chunk_fwd.restype = i32
+        L.gdn_chunk_fwd.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                    f32, vp, i32, vp, vp, ctypes.c_size_t, vp]
+        L.gdn_decode_step.restype = i32
+        L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, vp, vp]
+        L.gdn_gate_norm.restype = i32
+        L.gdn_gate_norm.argtypes = [vp, i32, vp, i32, vp, i64, i32, f32, vp, i32, vp]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_status_string.argtypes = [i32]
+        L.gdn_device_error.restype = i32
+        L.gdn_device_error.argtypes = [vp]
+        L.gdn_version.restype = i32
+        L.gdn_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDN_F32
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise GdnError(fn, code)
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0,
+              cu_seqlens_host=None, out=None, final_state=True, y_dtype=torch.float32):
+    """Chunked prefill over packed sequences. Returns (y, S_T or None).
+
+    q, k [N, H, d_k] and v [N, H, d_v] (fp32 or bf16, same dtype); log_alpha, beta [N, H]
+    fp32; cu_seqlens [n_seq + 1] int32 (device); S0 [n_seq, H, d_v, d_k] fp32 or None.
+    y is returned in y_dtype (float32 by default; bfloat16 gives the round-to-nearest-even
+    of the same fp32 result).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (log_alpha, "log_alpha"), (beta, "beta"),
+                 (cu_seqlens, "cu_seqlens")):
+        _cuda(t, n)
+    _cuda(S0, "S0")
+    code = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("log_alpha and beta must be float32")
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    n_seq = cu_seqlens.numel() - 1
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.to("cpu")
+    cu_h = cu_seqlens_host.to(torch.int32).contiguous()
+    y = out if out is not None else torch.empty((N, H, dv), dtype=y_dtype, device=q.device)
+    _cuda(y, "out")
+    S_T = (torch.empty((n_seq, H, dv, dk), dtype=torch.float32, device=q.device)
+           if final_state else None)
+    L = lib()
+    ws_bytes = L.gdn_chunk_fwd_workspace_bytes(n_seq, N, H, dk, dv, chunk)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device) if ws_bytes else None
+    rc = L.gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), code, _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                         _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), n_seq, H, dk, dv,
+                         int(chunk), float(scale), _ptr(y), _dtype_code(y), _ptr(S_T), _ptr(ws),
+                         ws_bytes, _stream(q.device))
+    _check("gdn_chunk_fwd", rc)
+    return y, S_T
+
+
+def decode_step(q, k, v, alpha, beta, S, scale=1.0, out=None):
+    """One token per chain; S [n_seq, H, d_v, d_k] fp32 is updated in place. Returns y."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (alpha, "alpha"), (beta, "beta"), (S, "S")):
+        _cuda(t, n)
+    code = _dtype_code(q)
+    n_seq, H, dk = q.shape
+    dv = v.shape[2]
+    y = out if out is not None else torch.empty((n_seq, H, dv), dtype=q.dtype, device=q.device)
+    rc = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha), _ptr(beta), _ptr(S),
+                               n_seq, H, dk, dv, float(scale), _ptr(y), _stream(q.device))
+    _check("gdn_decode_step", rc)
+    return y
+
+
+def gate_norm(y, z, w, eps=1e-6, out=None, out_dtype=None):
+    """o = sigmoid(z) * y / sqrt(mean(y^2) + eps) * (1 + w) over the last axis.
+
+    y and z may each be float32 or bfloat16; o is out_dtype (default: y's dtype)."""
+    for t, n in ((y, "y"), (z, "z"), (w, "w")):
+        _cuda(t, n)
+    if z.shape != y.shape:
+        raise ValueError("z must have y's shape")
+    if w.dtype != torch.float32 or w.numel() != y.shape[-1]:
+        raise TypeError("w must be float32 [d_v]")
+    dv = y.shape[-1]
+    n_rows = y.numel() // dv
+    if out is None:
+        out = torch.empty(y.shape, dtype=out_dtype or y.dtype, device=y.device)
+    _cuda(out, "out")
+    o = out
+    rc = lib().gdn_gate_norm(_ptr(y), _dtype_code(y), _ptr(z), _dtype_code(z), _ptr(w), n_rows,
+                             dv, float(eps), _ptr(o), _dtype_code(o), _stream(y.device))
+    _check("gdn_gate_norm", rc)
+    return o
+
+
+def device_error(device=None) -> str:
+    """Synchronises the current stream and returns (and clears) the device error status."""
+    dev = device if device is not None else torch.cuda.current_device()
+    return STATUS.get(lib().gdn_device_error(_stream(dev)), "?")

@@ -1,0 +1,63 @@
+// gdn_common.cuh -- device helpers shared by the library's kernels (one translation unit).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Per-device error word. Kernels OR bits into it; gdn_device_error() reads and clears it.
+__device__ unsigned int g_error_word;
+
+enum : unsigned int {
+    kErrTimeout = 1u,   // a bounded wait gave up
+    kErrCheck = 2u,     // an in-kernel consistency check failed
+};
+
+__device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
+
+// ---- element conversion -----------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x)
+{
+    return __float2bfloat16_rn(x);
+}
+
+// Load 4 consecutive elements as fp32 (16-byte load for fp32, 8-byte for bf16).
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p)
+{
+    uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+__device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v)
+{
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 raw;
+    raw.x = *reinterpret_cast<uint32_t *>(&a);
+    raw.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = raw;
+}
+
+// Sum over groups of G consecutive lanes (G a power of two <= 32); every lane of the
+// group receives the total.
+template <int G> __device__ __forceinline__ float group_sum(float x)
+{
+#pragma unroll
+    for (int off = G / 2; off > 0; off >>= 1)
+        x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+}  // namespace gdn

@@ -1,0 +1,283 @@
+// gdn_lib.cu -- the C ABI of libgdn_b200.so (declared in include/gdn.h): argument
+// validation, kernel selection and launch. The only translation unit of the library;
+// the kernels live in the headers it includes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "gdn.h"
+#include "gdn_chunk_f32.cuh"
+#include "gdn_chunk_sm100.cuh"
+#include "gdn_common.cuh"
+#include "gdn_decode.cuh"
+#include "gdn_gate_norm.cuh"
+
+namespace {
+
+using gdn::chunk_f32_layout;
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+gdn_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// ---- driver entry point for tensor-map encoding (no link-time libcuda dependency)
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode;
+}
+
+// 3-D map over a [n_tok][H][128] bf16 tensor, box {64, 1, 64}, 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *base, int64_t n_tok, int H)
+{
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)n_tok};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int g_smem_optin = -1;
+
+int smem_optin()
+{
+    if (g_smem_optin < 0) {
+        int dev = 0, v = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        g_smem_optin = v;
+    }
+    return g_smem_optin;
+}
+
+template <typename T, typename TY>
+gdn_status launch_chunk_f32(const void *q, const void *k, const void *v, const float *la,
+                            const float *beta, const float *S0, const int32_t *cu, int n_seq,
+                            int H, int dk, int dv, int C, float scale, void *y, float *S_T,
+                            cudaStream_t st)
+{
+    const int dvt = dv < 32 ? dv : 32;
+    const size_t smem = (size_t)chunk_f32_layout(C, dk, dvt).total * sizeof(float);
+    if ((int)smem > smem_optin()) return GDN_ERR_UNSUPPORTED;
+    auto kern = gdn::chunk_fwd_f32_kernel<T, TY>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const unsigned grid = (unsigned)((int64_t)n_seq * H * (dv / dvt));
+    kern<<<grid, gdn::kChunkF32Threads, smem, st>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), la, beta, S0,
+        cu, H, dk, dv, C, dvt, scale, static_cast<TY *>(y), S_T);
+    return launch_status();
+}
+
+template <typename TY>
+gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const float *la,
+                              const float *beta, const float *S0, const int32_t *cu, int n_seq,
+                              int64_t n_tok, int H, float scale, void *y, float *S_T,
+                              cudaStream_t st)
+{
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, n_tok, H) || !make_map(&mk, k, n_tok, H) || !make_map(&mv, v, n_tok, H))
+        return GDN_ERR_CUDA;
+    const int smem = (int)gdn::sm100::SMEM_BYTES;
+    if (smem > smem_optin()) return GDN_ERR_UNSUPPORTED;
+    auto kern = gdn::sm100::chunk_fwd_bf16_kernel<TY>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const unsigned grid = (unsigned)((int64_t)n_seq * H);
+    kern<<<grid, gdn::sm100::kThreads, smem, st>>>(mq, mk, mv, la, beta, S0, cu, n_seq, H, scale,
+                                                   static_cast<TY *>(y), S_T);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status s)
+{
+    switch (s) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    case GDN_ERR_DEVICE_CHECK: return "GDN_ERR_DEVICE_CHECK";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+int gdn_version(void) { return 100; }
+
+size_t gdn_chunk_fwd_workspace_bytes(int n_seq, int64_t total_tokens, int H, int d_k, int d_v,
+                                     int chunk)
+{
+    (void)n_seq; (void)total_tokens; (void)H; (void)d_k; (void)d_v; (void)chunk;
+    return 0;
+}
+
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                         int n_seq, int H, int d_k, int d_v, int chunk, float scale, void *y,
+                         gdn_dtype y_dtype, float *S_T, void *workspace, size_t workspace_bytes,
+                         void *stream)
+{
+    (void)workspace; (void)workspace_bytes;
+    if (n_seq < 0 || H <= 0 || !cu_seqlens_host || (n_seq > 0 && !cu_seqlens_dev))
+        return GDN_ERR_INVALID_ARG;
+    if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (y_dtype != GDN_F32 && y_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!pow2_in(d_k, 16, 128) || !pow2_in(d_v, 16, 128) || !pow2_in(chunk, 16, 64))
+        return GDN_ERR_UNSUPPORTED;
+    if (cu_seqlens_host[0] != 0) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < n_seq; ++i)
+        if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return GDN_ERR_INVALID_ARG;
+    if (n_seq == 0) return GDN_OK;
+    const int64_t n_tok = cu_seqlens_host[n_seq];
+    if (n_tok > 0 && (!q || !k || !v || !log_alpha || !beta || !y)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(y, 16) ||
+        !aligned(S0, 16) || !aligned(S_T, 16) || !aligned(log_alpha, 4) || !aligned(beta, 4) ||
+        !aligned(cu_seqlens_dev, 4))
+        return GDN_ERR_INVALID_ARG;
+    if ((int64_t)n_seq * H * (d_v / (d_v < 32 ? d_v : 32)) > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    const bool y32 = y_dtype == GDN_F32;
+    if (in_dtype == GDN_BF16 && d_k == 128 && d_v == 128 && chunk == 64)
+        return y32 ? launch_chunk_sm100<float>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev, n_seq,
+                                               n_tok, H, scale, y, S_T, st)
+                   : launch_chunk_sm100<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev,
+                                                       n_seq, n_tok, H, scale, y, S_T, st);
+#define GDN_F32_PATH(T, TY)                                                                        \
+    launch_chunk_f32<T, TY>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev, n_seq, H, d_k, d_v, chunk, \
+                            scale, y, S_T, st)
+    if (in_dtype == GDN_BF16)
+        return y32 ? GDN_F32_PATH(__nv_bfloat16, float) : GDN_F32_PATH(__nv_bfloat16, __nv_bfloat16);
+    return y32 ? GDN_F32_PATH(float, float) : GDN_F32_PATH(float, __nv_bfloat16);
+#undef GDN_F32_PATH
+}
+
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                           const float *alpha, const float *beta, float *S, int n_seq, int H,
+                           int d_k, int d_v, float scale, void *y, void *stream)
+{
+    if (n_seq < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+    if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!pow2_in(d_k, 16, 128) || !pow2_in(d_v, 16, 128)) return GDN_ERR_UNSUPPORTED;
+    const int64_t n_chain = (int64_t)n_seq * H;
+    if (n_chain == 0) return GDN_OK;
+    if (n_chain > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !S || !y) return GDN_ERR_INVALID_ARG;
+    const size_t vec = in_dtype == GDN_F32 ? 16 : 8;
+    if (!aligned(q, vec) || !aligned(k, vec) || !aligned(S, 16) || !aligned(alpha, 4) ||
+        !aligned(beta, 4) || !aligned(v, 4) || !aligned(y, 4))
+        return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    const unsigned grid = (unsigned)n_chain;
+#define GDN_DECODE_CASE(DK)                                                                        \
+    case DK:                                                                                       \
+        if (in_dtype == GDN_F32)                                                                   \
+            gdn::decode_step_kernel<DK, float><<<grid, gdn::kDecodeThreads, 0, st>>>(              \
+                (const float *)q, (const float *)k, (const float *)v, alpha, beta, S, d_v, scale,  \
+                (float *)y);                                                                       \
+        else                                                                                       \
+            gdn::decode_step_kernel<DK, __nv_bfloat16><<<grid, gdn::kDecodeThreads, 0, st>>>(      \
+                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,      \
+                alpha, beta, S, d_v, scale, (__nv_bfloat16 *)y);                                   \
+        break;
+    switch (d_k) {
+        GDN_DECODE_CASE(16)
+        GDN_DECODE_CASE(32)
+        GDN_DECODE_CASE(64)
+        GDN_DECODE_CASE(128)
+    default: return GDN_ERR_UNSUPPORTED;
+    }
+#undef GDN_DECODE_CASE
+    return launch_status();
+}
+
+gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dtype z_dtype,
+                         const float *w, int64_t n_rows, int d_v, float eps, void *o,
+                         gdn_dtype o_dtype, void *stream)
+{
+    if (n_rows < 0) return GDN_ERR_INVALID_ARG;
+    for (gdn_dtype dt : {y_dtype, z_dtype, o_dtype})
+        if (dt != GDN_F32 && dt != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!pow2_in(d_v, 16, 256)) return GDN_ERR_UNSUPPORTED;
+    if (n_rows == 0) return GDN_OK;
+    if (!y || !z || !w || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned(y, 16) || !aligned(z, 16) || !aligned(o, 16) || !aligned(w, 4))
+        return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    int dev = 0, n_sm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    // rows per CTA pass = 8 warps x rows-per-warp x 2 (unroll); at most 8 CTAs per SM
+    const int64_t rows_per_cta = (int64_t)(gdn::kGateNormThreads / 32) * (32 / (d_v / 8)) * 2;
+    int64_t blocks = (n_rows + rows_per_cta - 1) / rows_per_cta;
+    const int64_t cap = (int64_t)n_sm * 8;
+    if (blocks > cap) blocks = cap;
+    const int combo = (y_dtype == GDN_BF16) * 4 + (z_dtype == GDN_BF16) * 2 + (o_dtype == GDN_BF16);
+    using f32 = float;
+    using b16 = __nv_bfloat16;
+#define GDN_GN(TY, TZ, TO, DV)                                                                     \
+    gdn::gate_norm_kernel<TY, TZ, TO, DV><<<(unsigned)blocks, gdn::kGateNormThreads, 0, st>>>(     \
+        (const TY *)y, (const TZ *)z, w, n_rows, eps, (TO *)o)
+#define GDN_GN_DV(TY, TZ, TO)                                                                      \
+    switch (d_v) {                                                                                 \
+    case 16: GDN_GN(TY, TZ, TO, 16); break;                                                        \
+    case 32: GDN_GN(TY, TZ, TO, 32); break;                                                        \
+    case 64: GDN_GN(TY, TZ, TO, 64); break;                                                        \
+    case 128: GDN_GN(TY, TZ, TO, 128); break;                                                      \
+    default: GDN_GN(TY, TZ, TO, 256); break;                                                       \
+    }
+    switch (combo) {
+    case 0: GDN_GN_DV(f32, f32, f32) break;
+    case 1: GDN_GN_DV(f32, f32, b16) break;
+    case 2: GDN_GN_DV(f32, b16, f32) break;
+    case 3: GDN_GN_DV(f32, b16, b16) break;
+    case 4: GDN_GN_DV(b16, f32, f32) break;
+    case 5: GDN_GN_DV(b16, f32, b16) break;
+    case 6: GDN_GN_DV(b16, b16, f32) break;
+    default: GDN_GN_DV(b16, b16, b16) break;
+    }
+#undef GDN_GN_DV
+#undef GDN_GN
+    return launch_status();
+}
+
+gdn_status gdn_device_error(void *stream)
+{
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return GDN_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, gdn::g_error_word, sizeof(word)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(gdn::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (word & gdn::kErrTimeout) return GDN_ERR_TIMEOUT;
+    if (word & gdn::kErrCheck) return GDN_ERR_DEVICE_CHECK;
+    return GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,159 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated delta rule library, libgdn_b200.so.
+ *
+ * The library computes the Gated DeltaNet token mixer's gated delta rule and its
+ * output epilogue, as defined on the joezjh.github.io notes page "Qwen3.8-Flash-Next"
+ * (section "Gated DeltaNet 核心机制", the four-line update rule and its equivalent
+ * form; section "GDN 参数化细节", the output-gate equation) and on the pwwt.cn
+ * translation of the report (section 2.1.1, "sigmoid output gate", "zero-centred
+ * RMSNorm"). Per head, with state S in R^{d_k x d_v}:
+ *
+ *     S~ = alpha_t S_{t-1};  e_t = v_t - S~^T k_t;  S_t = S~ + beta_t k_t e_t^T;
+ *     y_t = S_t^T (scale * q_t)            (equivalently S_t = alpha_t (I - beta_t k_t k_t^T)
+ *                                            S_{t-1} + beta_t k_t v_t^T)
+ *     o_t = sigmoid(z_t) * y_t / sqrt(mean(y_t^2) + eps) * (1 + w)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor argument is a DEVICE pointer owned by the caller (cudaMalloc'd or a
+ *    torch tensor's data pointer), contiguous, in the layout stated. Pointers to q, k,
+ *    v, y, z, o, S0, S_T and S must be 16-byte aligned; log_alpha/alpha/beta and
+ *    cu_seqlens_dev 4-byte aligned.
+ *  - STATE LAYOUT is value-major: [.., d_v, d_k], i.e. the transpose S^T stored
+ *    row-major with the key dimension contiguous. (Row j holds column j of the pages'
+ *    S.) All states in and out are fp32.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *    legacy default stream) and never synchronise, except gdn_device_error().
+ *  - The library allocates no device memory in any call.
+ *  - Outputs must not alias inputs, except S in gdn_decode_step, which is updated in
+ *    place.
+ *  - Argument errors are reported before any launch: GDN_ERR_INVALID_ARG (null or
+ *    misaligned pointer, negative size, inconsistent cu_seqlens) or
+ *    GDN_ERR_UNSUPPORTED (a size outside the supported set). A failed launch returns
+ *    GDN_ERR_CUDA. Conditions a kernel detects while running (a bounded wait that
+ *    gave up, an internal check) set a device-side error word that gdn_device_error()
+ *    reads. No exception or abort crosses this boundary.
+ *  - Not thread-safe with respect to gdn_device_error(): the error word is per device.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_seqlens      */
+    GDN_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes/dtypes          */
+    GDN_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed                   */
+    GDN_ERR_TIMEOUT = 4,       /* (device error word) a bounded wait inside a kernel     */
+    GDN_ERR_DEVICE_CHECK = 5   /* (device error word) an in-kernel consistency check     */
+} gdn_status;
+
+typedef enum {
+    GDN_F32 = 0,               /* IEEE binary32                                          */
+    GDN_BF16 = 1               /* bfloat16; results rounded to nearest even              */
+} gdn_dtype;
+
+/*
+ * gdn_chunk_fwd -- chunked prefill of the gated delta rule over packed sequences.
+ *
+ * Defines: the four-line update rule above, applied token by token within each
+ * sequence (joezjh.github.io notes, "Gated DeltaNet 核心机制"); the library computes it
+ * in the chunkwise-parallel form (exact up to rounding), chunk tokens at a time.
+ * Sequences are independent; the state starts at S0 (or 0) at each sequence start.
+ *
+ *   q, k        [N_tok, H, d_k]  in in_dtype (N_tok = cu_seqlens[n_seq]); the
+ *                                parameterisation expects L2-normalised q, k
+ *   v           [N_tok, H, d_v]  in in_dtype
+ *   log_alpha   [N_tok, H] fp32  log of the decay gate, <= 0 (alpha in (0, 1])
+ *   beta        [N_tok, H] fp32  write strength, in [0, 1]
+ *   S0          [n_seq, H, d_v, d_k] fp32, or NULL for a zero initial state
+ *   cu_seqlens_dev  [n_seq + 1] int32, device copy read by the kernels
+ *   cu_seqlens_host [n_seq + 1] int32, HOST copy with identical contents, used to
+ *                   validate and size the launch without a device->host copy;
+ *                   element 0 must be 0 and the sequence non-decreasing
+ *   n_seq >= 0, H >= 1
+ *   d_k, d_v    each in {16, 32, 64, 128}
+ *   chunk       in {16, 32, 64}; chunk boundaries restart at every sequence start
+ *   scale       multiplies q (the pages use none: pass 1.0)
+ *   y           [N_tok, H, d_v]  out, in y_dtype (GDN_F32 or GDN_BF16, independent of
+ *               in_dtype; a bf16 y is the round-to-nearest-even of the fp32 result)
+ *   S_T         [n_seq, H, d_v, d_k] fp32 out (final state per sequence), or NULL
+ *   workspace   device scratch of workspace_bytes >= gdn_chunk_fwd_workspace_bytes(..)
+ *               (may be NULL when that is 0)
+ *
+ * Paths: bf16 inputs with d_k = d_v = 128 and chunk = 64 run the sm_100a tensor-core
+ * kernel (tcgen05 MMA with TMEM accumulators, TMA loads, fp32 state carry; bf16 inputs
+ * feed the K K^T / Q K^T product, all other products use fp16 operands -- the inputs
+ * convert exactly -- which requires |q|, |k|, |v| and the state entries below 65504);
+ * every other supported case runs the CUDA-core fp32 chunk kernel.
+ */
+size_t gdn_chunk_fwd_workspace_bytes(int n_seq, int64_t total_tokens, int H, int d_k, int d_v,
+                                     int chunk);
+
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                         int n_seq, int H, int d_k, int d_v, int chunk, float scale,
+                         void *y, gdn_dtype y_dtype, float *S_T, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_decode_step -- one token for each of n_seq * H independent chains, in place.
+ *
+ * Defines: the same four-line update (joezjh.github.io notes, "Gated DeltaNet 核心机制")
+ * for a single token, with alpha given directly. It is computed in one pass over S:
+ * with u = S^T k and r = S^T q taken on the old state, e = v - alpha u,
+ * y = scale (alpha r + beta (k.q) e) (which equals S_new^T (scale q)), and
+ * S <- alpha S + beta k e^T.
+ *
+ *   q, k   [n_seq, H, d_k] in in_dtype;  v [n_seq, H, d_v] in in_dtype
+ *   alpha  [n_seq, H] fp32 in (0, 1];  beta [n_seq, H] fp32 in [0, 1]
+ *   S      [n_seq, H, d_v, d_k] fp32, read and overwritten with the new state
+ *   y      [n_seq, H, d_v] out, in in_dtype
+ *   d_k, d_v each in {16, 32, 64, 128}
+ */
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                           const float *alpha, const float *beta, float *S, int n_seq, int H,
+                           int d_k, int d_v, float scale, void *y, void *stream);
+
+/*
+ * gdn_gate_norm -- the output epilogue o = sigmoid(z) * RMSNorm(y) * (1 + w).
+ *
+ * Defines: the output-gate equation of the joezjh.github.io notes ("GDN 参数化细节")
+ * without its W_z / W_o projections (z is the already projected gate logit), with the
+ * zero-centred RMSNorm of the pwwt.cn translation (section 2.1.1): the stored weight
+ * w multiplies as (1 + w); the input is not mean-subtracted. One row = one (token,
+ * head); the mean is over its d_v elements.
+ *
+ *   y      [n_rows, d_v] in y_dtype;  z [n_rows, d_v] in z_dtype;  w [d_v] fp32
+ *   o      [n_rows, d_v] out in o_dtype (each dtype GDN_F32 or GDN_BF16)
+ *   n_rows >= 0; d_v in {16, 32, 64, 128, 256}; eps > 0 recommended (1e-6)
+ */
+gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dtype z_dtype,
+                         const float *w, int64_t n_rows, int d_v, float eps, void *o,
+                         gdn_dtype o_dtype, void *stream);
+
+/* A static, human-readable name for a status code. */
+const char *gdn_status_string(gdn_status status);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error word.
+ * Returns GDN_OK, GDN_ERR_TIMEOUT or GDN_ERR_DEVICE_CHECK for conditions kernels
+ * recorded, or GDN_ERR_CUDA if the synchronisation itself failed.
+ */
+gdn_status gdn_device_error(void *stream);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

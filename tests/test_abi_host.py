@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol gdn.h declares,
+and rejects bad arguments before any launch (these calls never touch a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import gated_deltanet_05_b200 as gdn
+from gated_deltanet_05_b200 import build as gdn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gdn_build.build()
+    return gdn.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    assert set(names) == set(gdn.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", gdn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gdn_[a-z_]+)\b", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_status_strings_and_version(L):
+    for code, name in gdn.STATUS.items():
+        assert L.gdn_status_string(code).decode() == name
+    assert L.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+    assert L.gdn_version() == 100
+    assert L.gdn_chunk_fwd_workspace_bytes(4, 16384, 16, 128, 128, 64) == 0
+
+
+def _cu(vals):
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return arr
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced on these paths
+
+
+def _chunk(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, la=FAKE, b=FAKE, S0=None, cud=FAKE, cuh=_cu([0, 64]),
+             n_seq=1, H=2, dk=128, dv=128, C=64, scale=1.0, y=FAKE, ydt=0, ST=None, ws=None,
+             wsb=0, st=None)
+    a.update(kw)
+    return L.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["dt"], a["la"], a["b"], a["S0"], a["cud"],
+                           ctypes.cast(a["cuh"], ctypes.c_void_p) if a["cuh"] is not None else None,
+                           a["n_seq"], a["H"], a["dk"], a["dv"], a["C"], a["scale"], a["y"],
+                           a["ydt"], a["ST"], a["ws"], a["wsb"], a["st"])
+
+
+def test_chunk_fwd_rejects_bad_arguments(L):
+    assert _chunk(L, cuh=None) == 1                         # no host cu_seqlens
+    assert _chunk(L, n_seq=-1) == 1
+    assert _chunk(L, H=0) == 1
+    assert _chunk(L, dt=7) == 1                             # unknown dtype
+    assert _chunk(L, ydt=3) == 1
+    assert _chunk(L, dk=96) == 2                            # unsupported sizes
+    assert _chunk(L, dv=256) == 2
+    assert _chunk(L, C=128) == 2
+    assert _chunk(L, C=8) == 2
+    assert _chunk(L, cuh=_cu([1, 64])) == 1                 # must start at 0
+    assert _chunk(L, cuh=_cu([0, 64, 32]), n_seq=2) == 1    # must not decrease
+    assert _chunk(L, q=None) == 1                           # null input
+    assert _chunk(L, y=ctypes.c_void_p(0x10008)) == 1       # misaligned output
+    assert _chunk(L, la=ctypes.c_void_p(0x10002)) == 1      # misaligned gate
+    assert _chunk(L, n_seq=0, cuh=_cu([0])) == 0            # nothing to do
+
+
+def test_decode_and_gate_norm_reject_bad_arguments(L):
+    dec = lambda **kw: L.gdn_decode_step(kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 0), FAKE,
+                                         FAKE, kw.get("S", FAKE), kw.get("n", 4), kw.get("H", 2),
+                                         kw.get("dk", 128), kw.get("dv", 128), 1.0, FAKE, None)
+    assert dec(n=-1) == 1
+    assert dec(H=0) == 1
+    assert dec(dk=48) == 2
+    assert dec(dv=512) == 2
+    assert dec(q=None) == 1
+    assert dec(S=ctypes.c_void_p(0x10004)) == 1
+    assert dec(n=0) == 0
+    gn = lambda **kw: L.gdn_gate_norm(kw.get("y", FAKE), kw.get("dt", 1), FAKE, 1, FAKE,
+                                      kw.get("rows", 10), kw.get("dv", 128), 1e-6,
+                                      kw.get("o", FAKE), kw.get("odt", 1), None)
+    assert gn(rows=-1) == 1
+    assert gn(dv=96) == 2
+    assert gn(dv=512) == 2
+    assert gn(dt=5) == 1
+    assert gn(odt=2) == 1
+    assert gn(y=None) == 1
+    assert gn(o=ctypes.c_void_p(0x10008)) == 1
+    assert gn(rows=0) == 0
+
+
+def test_binding_has_no_cpu_fallback(monkeypatch):
+    """Calls on CPU tensors raise instead of computing anything."""
+    import torch
+    q = torch.zeros(4, 1, 16)
+    with pytest.raises(ValueError):
+        gdn.decode_step(q, q, q, torch.ones(4, 1), torch.ones(4, 1), torch.zeros(4, 1, 16, 16))
+    with pytest.raises(ValueError):
+        gdn.gate_norm(q, q, torch.zeros(16))
+
+
+def test_package_does_not_import_oracle():
+    pkg_dir = os.path.dirname(gdn.__file__)
+    for root, _, files in os.walk(pkg_dir):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "gdn_oracle" not in text, f
