@@ -10,15 +10,16 @@
 //   S <- gamma_C S + (diag(exp(g_C - g)) K)^T U~
 // Every product is taken "value-major" so that the MMA M dimension is d_v = 128 (or
 // d_k = 128) and all accumulators fill the 128 TMEM lanes:
-//   G   = [K; Q] K^T                      M=128 (64 K rows, 64 Q rows), N=64, K=128
-//   W^T = K^T (T diag(beta gamma))^T      M=128 (d_k), N=64, K=64       A MN-major
-//   U^T = V^T (T diag(beta))^T            M=128 (d_v), N=64, K=64       A MN-major
-//   U~^T = U^T - S^T W^T                  M=128 (d_v), N=64, K=128      B MN-major (-W^T)
-//   Y^T  = S^T (diag(gamma) Q)^T + U~^T P^T   M=128, N=64, K=128 + 64
+//   G    = [K; Q] K^T                      M=128 (64 K rows, 64 Q rows), N=64, K=128
+//   W^T  = K^T (T diag(beta gamma))^T      M=128 (d_k), N=64, K=64       A MN-major
+//   U^T  = V^T (T diag(beta))^T            M=128 (d_v), N=64, K=64       A MN-major
+//   U~^T = U^T - S^T W^T                   M=128 (d_v), N=64, K=128      B MN-major (-W^T)
+//   Y^T  = S^T (diag(gamma) Q)^T + U~^T P^T    M=128, N=64, K=128 + 64
 //   S^T <- gamma_C S^T + (U~^T diag(exp(g_C - g))) K   M=128, N=128, K=64, B MN-major
 // The state S^T (value-major, the library's state layout) lives in TMEM in fp32 for the
 // whole sequence; each chunk it is also written as an fp16 copy to shared memory as the
-// MMA operand. Every exponent is <= 0.
+// MMA operand. Every exponent is <= 0 (exponentials are taken base 2 on log2-scaled
+// decays, with the SM's approximate exp2 instruction).
 //
 // Operand precision: G = [K; Q] K^T runs on the bf16 inputs as loaded. Every other
 // product runs on fp16 operands (kind::f16, fp32 accumulate): after G, the K, Q, V tiles
@@ -29,14 +30,20 @@
 // (8-bit) operands do not. y is written in fp32 or bf16.
 //
 // One CTA owns one (sequence, head) chain. Warp roles (384 threads):
-//   warp 0     TMA producer: K, Q, V tiles of each chunk (2-stage ring, 128B swizzle)
-//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2-3  idle
-//   warps 4-7  "solve" warpgroup: gates, L and P from G, the triangular solve (fp32,
-//              blocked forward substitution in shared memory), T/P/Q/K/V fp16 operands,
-//              and the -W^T operand from its TMEM accumulator
-//   warps 8-11 "state" warpgroup: U~ -> fp16 operands, y = Y^T out, S carry
-//              (scale by gamma_C, fp16 copy), S0 in and S_T out
+//   warp 0      TMA producer: K, Q, V tiles of each chunk (2-stage ring, 128B swizzle)
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2-3   converters: the stage's K, V -> fp16 and Q -> fp16(gamma scale q), in place
+//   warps 4-7   "solve" warpgroup: L and P from G, T = (I + L)^-1 in fp32 (16x16 diagonal
+//               blocks by forward substitution, then two levels of block merges), the
+//               fp16 T/P operands and -W^T from its TMEM accumulator
+//   warps 8-11  "state" warpgroup: U~ -> fp16 operands, the fp16 state copy, y out,
+//               the state carry (scale by gamma_C), S0 in and S_T out
+// The state warpgroup publishes the fp16 copy of S_{c+1} and the rescaled fp32 state
+// before it writes y_c, which keeps the y stores off the chunk-to-chunk critical path;
+// the Y^T accumulator is double-buffered for that reason, and y leaves through a
+// shared-memory staging tile and one asynchronous bulk copy per token row. The MMA issuer polls its
+// barriers and issues whichever product is ready (chain products first), so the next
+// chunk's K K^T / Q K^T and solve overlap the current chunk's state chain.
 // All mbarrier waits are bounded (~1 s); on a timeout the kernel records it in the
 // device error word, every role leaves its loop, in-flight TMA and MMA work is drained
 // (again with bounded waits) and TMEM is released before the CTA exits.
@@ -53,6 +60,7 @@ constexpr int kC = 64;       // chunk length
 constexpr int kD = 128;      // d_k = d_v
 constexpr int kThreads = 384;
 constexpr long long kWaitLimit = 2000000000LL;   // SM cycles (~1 s at 1.9 GHz)
+constexpr float kLog2e = 1.4426950408889634f;
 
 // shared-memory layout (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_QK = 0;          // 2 stages x 32 KB: [K d0..63 | Q d0..63 | K d64.. | Q d64..]
@@ -63,43 +71,50 @@ constexpr uint32_t OFF_SB = 98304;      // 32 KB fp16 S^T [128 v][128 k], K-majo
 constexpr uint32_t OFF_UB = 131072;     // 16 KB fp16 U~^T [128 v][64 s]
 constexpr uint32_t OFF_UD = 147456;     // 16 KB fp16 U~^T diag(exp(g_C - g))
 constexpr uint32_t OFF_WB = 163840;     // 16 KB fp16 -W^T [128 k][64 t], MN-major
-constexpr uint32_t OFF_P = 180224;      // 8 KB fp16 P [64 t][64 s]
+constexpr uint32_t OFF_YST = OFF_UB;    // y staging [64 t][128 v] (32 KB over U~b and U~d, free in E3)
+constexpr uint32_t OFF_SPARE = 180224;  // 8 KB unused
 constexpr uint32_t OFF_TBG = 188416;    // 8 KB fp16 T diag(beta gamma) [64 t][64 s]
 constexpr uint32_t OFF_TB = 196608;     // 8 KB fp16 T diag(beta)
-constexpr uint32_t OFF_LS = 204800;     // fp32 [64][65]: L, then T in place
-constexpr int LS_LD = 65;
-constexpr uint32_t OFF_RT = OFF_LS + 64 * LS_LD * 4;     // fp32 [16][48] block-row temp
-constexpr uint32_t OFF_GATES = OFF_RT + 16 * 48 * 4;     // {g, gamma, beta}[64] fp32 of the solve's chunk
-constexpr uint32_t OFF_BAR = OFF_GATES + 3 * 64 * 4;     // mbarriers
-constexpr int N_BAR = 16;
+constexpr uint32_t OFF_LS = 204800;     // fp32 [64][68]: L, then T in place
+constexpr int LS_LD = 68;
+constexpr uint32_t OFF_RT = OFF_LS + 64 * LS_LD * 4;     // fp32 merge temp, [32][36] at most
+constexpr int RT_LD = 36;
+constexpr uint32_t OFF_GATES = OFF_RT + 32 * RT_LD * 4;  // {g2, gamma, beta}[64] fp32 of the solve's chunk
+constexpr uint32_t OFF_DEC = OFF_GATES + 3 * 64 * 4;     // state warpgroup: exp(g_C - g)[64] per warp
+constexpr uint32_t OFF_BAR = OFF_DEC + 4 * 64 * 4;       // mbarriers
+constexpr int N_BAR = 18;
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BAR * 8;       // tmem base, abort flag, chain's sequence
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;        // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// TMEM columns (fp32, 128 lanes)
+// TMEM columns (fp32, 128 lanes); the Y^T accumulator is double-buffered
 constexpr uint32_t TM_S = 0, TM_G = 128, TM_W = 192, TM_U = 256, TM_Y = 320, TM_COLS = 512;
 
 // barrier indices
 enum {
-    B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_GFULL, B_GEMPTY, B_TBG, B_WFULL, B_TB, B_WB,
-    B_P, B_XFULL, B_UD, B_SFULL, B_SB, B_DRAIN
+    B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_GFULL, B_GEMPTY, B_CONV, B_TBG, B_WFULL, B_TB,
+    B_WB, B_P, B_XFULL, B_UD, B_SFULL, B_SB, B_SACC, B_DRAIN
 };
+static_assert(B_DRAIN + 1 == N_BAR, "barrier count");
+
+// named barriers (0 is __syncthreads)
+enum { NB_SOLVE = 1, NB_STATE = 2, NB_SOLVE_LO = 3, NB_CONV = 4 };
 
 struct ChainInfo {
     int seq, h;
     int64_t bos, len;
 };
 
-// Inclusive scan of one chunk's log decays (zero past the sequence end), two tokens per
-// lane: g_lo for tokens 0..31, g_hi for 32..63. Every warp that calls it gets
+// Inclusive scan of one chunk's log2-scaled decays (zero past the sequence end), two
+// tokens per lane: g_lo for tokens 0..31, g_hi for 32..63. Every warp that calls it gets
 // bit-identical values.
-__device__ __forceinline__ void chunk_log_decay_scan(const float *__restrict__ log_alpha, int64_t tok0,
-                                                     int H, int h, int n_valid, int lane,
-                                                     float &g_lo, float &g_hi)
+__device__ __forceinline__ void chunk_log2_decay_scan(const float *__restrict__ log_alpha, int64_t tok0,
+                                                      int H, int h, int n_valid, int lane,
+                                                      float &g_lo, float &g_hi)
 {
-    float x0 = lane < n_valid ? log_alpha[(size_t)(tok0 + lane) * H + h] : 0.f;
-    float x1 = lane + 32 < n_valid ? log_alpha[(size_t)(tok0 + lane + 32) * H + h] : 0.f;
+    float x0 = lane < n_valid ? log_alpha[(size_t)(tok0 + lane) * H + h] * kLog2e : 0.f;
+    float x1 = lane + 32 < n_valid ? log_alpha[(size_t)(tok0 + lane + 32) * H + h] * kLog2e : 0.f;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const float o0 = __shfl_up_sync(0xffffffffu, x0, off);
@@ -115,6 +130,25 @@ __device__ __forceinline__ void chunk_log_decay_scan(const float *__restrict__ l
 
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+__device__ __forceinline__ void sts128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+__device__ __forceinline__ float4 ldsf4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ void stsf4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+
+// fp16 pairs of 8 consecutive floats
+__device__ __forceinline__ uint4 pack8_f16(const float *x)
+{
+    return make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]), pack_f16x2(x[4], x[5]),
+                      pack_f16x2(x[6], x[7]));
+}
+
+// One bf16 16-byte chunk -> fp16, each value multiplied by f.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v, float f)
+{
+    return make_uint4(pack_f16x2(bf_lo(v.x) * f, bf_hi(v.x) * f), pack_f16x2(bf_lo(v.y) * f, bf_hi(v.y) * f),
+                      pack_f16x2(bf_lo(v.z) * f, bf_hi(v.z) * f), pack_f16x2(bf_lo(v.w) * f, bf_hi(v.w) * f));
+}
 
 template <typename TY>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -132,6 +166,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    int *seq_slot = reinterpret_cast<int *>(smem + OFF_MISC + 8);
     float *Ls = reinterpret_cast<float *>(smem + OFF_LS);
     float *Rt = reinterpret_cast<float *>(smem + OFF_RT);
 
@@ -141,7 +176,6 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // ---- which chain: sequences in order of decreasing length (ties by index), so the
     // longest chains start first; identity order beyond kThreads sequences
     const int rank = blockIdx.x / H;
-    int *seq_slot = reinterpret_cast<int *>(smem + OFF_MISC + 8);
     if (n_seq > kThreads) {
         if (tid == 0) *seq_slot = rank;
     } else if (tid < n_seq) {
@@ -156,22 +190,14 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     // ---- setup
     if (tid == 0) {
-        mbar_init(&bar[B_FULL0], 1);
-        mbar_init(&bar[B_FULL1], 1);
-        mbar_init(&bar[B_EMPTY0], 1);
-        mbar_init(&bar[B_EMPTY1], 1);
-        mbar_init(&bar[B_GFULL], 1);
-        mbar_init(&bar[B_GEMPTY], 128);
-        mbar_init(&bar[B_TBG], 128);
-        mbar_init(&bar[B_WFULL], 1);
-        mbar_init(&bar[B_TB], 128);
-        mbar_init(&bar[B_WB], 128);
-        mbar_init(&bar[B_P], 128);
-        mbar_init(&bar[B_XFULL], 1);
-        mbar_init(&bar[B_UD], 128);
-        mbar_init(&bar[B_SFULL], 1);
-        mbar_init(&bar[B_SB], 128);
-        mbar_init(&bar[B_DRAIN], 1);
+        for (int b = 0; b < N_BAR; ++b) {
+            uint32_t count = 1;
+            if (b == B_GEMPTY || b == B_TBG || b == B_TB || b == B_WB || b == B_P || b == B_UD ||
+                b == B_SB || b == B_SACC)
+                count = 128;
+            if (b == B_CONV) count = 64;
+            mbar_init(&bar[b], count);
+        }
         *abort_flag = 0;
         fence_mbarrier_init();
         fence_proxy_async_smem();
@@ -191,6 +217,10 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     ci.len = (int64_t)cu_seqlens[ci.seq + 1] - ci.bos;
     const int n_chunks = (int)((ci.len + kC - 1) / kC);
     const size_t state_off = ((size_t)ci.seq * H + ci.h) * (size_t)kD * kD;
+    auto chunk_valid = [&](int c) -> int {
+        const int64_t rem = ci.len - (int64_t)c * kC;
+        return (int)(rem < kC ? rem : kC);
+    };
 
     if (warp == 0) {
         // ================================================================ TMA producer
@@ -228,286 +258,402 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint32_t id_xw = idesc_f32acc(kFmtF16, 128, 64, 0, 1);
             const uint32_t id_yq = idesc_f32acc(kFmtF16, 128, 64, 0, 0);
             const uint32_t id_s = idesc_f32acc(kFmtF16, 128, 128, 0, 1);
-            bool ok = true;
-            auto issue_G = [&](int c) -> bool {
-                const int st = c & 1;
-                if (!mbar_wait_bounded(&bar[B_FULL0 + st], (c >> 1) & 1, abort_flag, kWaitLimit)) return false;
-                if (c > 0 && !mbar_wait_bounded(&bar[B_GEMPTY], (c - 1) & 1, abort_flag, kWaitLimit)) return false;
-                tc_fence_after();
-                const uint32_t qk = sbase + OFF_QK + st * QK_STAGE;
+            auto done = [&](int b, int parity) { return mbar_test(&bar[b], parity & 1); };
+            auto do_G = [&](int c) {
+                const uint32_t qk = sbase + OFF_QK + (c & 1) * QK_STAGE;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = qk + (kk >> 2) * 16384 + (kk & 3) * 32;
                     mma_f16kind_ss(tmem + TM_G, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id_g, kk > 0);
                 }
                 mma_commit(&bar[B_GFULL]);
-                return true;
             };
-            auto issue_W = [&](int c) -> bool {
-                if (!mbar_wait_bounded(&bar[B_TBG], c & 1, abort_flag, kWaitLimit)) return false;
-                tc_fence_after();
+            auto do_W = [&](int c) {
                 const uint32_t kt = sbase + OFF_QK + (c & 1) * QK_STAGE;   // K^T: MN-major, LBO 16 KB
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16kind_ss(tmem + TM_W, sdesc_sw128(kt + kk * 2048, 16384, 1024),
-                                sdesc_sw128(sbase + OFF_TBG + kk * 32, 16, 1024), id_wu, kk > 0);
+                                   sdesc_sw128(sbase + OFF_TBG + kk * 32, 16, 1024), id_wu, kk > 0);
                 mma_commit(&bar[B_WFULL]);
-                return true;
             };
-            auto issue_U = [&](int c) -> bool {
-                if (!mbar_wait_bounded(&bar[B_TB], c & 1, abort_flag, kWaitLimit)) return false;
-                tc_fence_after();
+            auto do_U = [&](int c) {
                 const uint32_t vt = sbase + OFF_V + (c & 1) * V_STAGE;     // V^T: MN-major, LBO 8 KB
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16kind_ss(tmem + TM_U, sdesc_sw128(vt + kk * 2048, 8192, 1024),
-                                sdesc_sw128(sbase + OFF_TB + kk * 32, 16, 1024), id_wu, kk > 0);
-                return true;
+                                   sdesc_sw128(sbase + OFF_TB + kk * 32, 16, 1024), id_wu, kk > 0);
             };
-            auto issue_X = [&](int c) -> bool {
-                if (!mbar_wait_bounded(&bar[B_WB], c & 1, abort_flag, kWaitLimit)) return false;
-                if (!mbar_wait_bounded(&bar[B_SB], c & 1, abort_flag, kWaitLimit)) return false;
-                tc_fence_after();
+            auto do_X = [&](int c) {
                 const uint32_t qk = sbase + OFF_QK + (c & 1) * QK_STAGE;
+                const uint32_t ty = tmem + TM_Y + (c & 1) * 64;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = sbase + OFF_SB + (kk >> 2) * 16384 + (kk & 3) * 32;
                     // U~^T += S^T (-W^T): B = -W^T stored [k][t], MN-major
                     mma_f16kind_ss(tmem + TM_U, sdesc_sw128(a, 16, 1024),
-                                sdesc_sw128(sbase + OFF_WB + kk * 2048, 8192, 1024), id_xw, 1);
-                    // Y^T = S^T (gamma Q)^T: B = Q rows (K-major), Q at +8 KB / +24 KB
-                    mma_f16kind_ss(tmem + TM_Y, sdesc_sw128(a, 16, 1024),
-                                sdesc_sw128(qk + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                id_yq, kk > 0);
+                                   sdesc_sw128(sbase + OFF_WB + kk * 2048, 8192, 1024), id_xw, 1);
+                    // Y^T = S^T (gamma scale Q)^T: B = Q rows (K-major), Q at +8 KB / +24 KB
+                    mma_f16kind_ss(ty, sdesc_sw128(a, 16, 1024),
+                                   sdesc_sw128(qk + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                   id_yq, kk > 0);
                 }
                 mma_commit(&bar[B_XFULL]);
-                return true;
             };
-            auto issue_S = [&](int c) -> bool {
-                if (!mbar_wait_bounded(&bar[B_UD], c & 1, abort_flag, kWaitLimit)) return false;
-                if (!mbar_wait_bounded(&bar[B_P], c & 1, abort_flag, kWaitLimit)) return false;
-                tc_fence_after();
+            auto do_S = [&](int c) {
                 const uint32_t kb = sbase + OFF_QK + (c & 1) * QK_STAGE;   // K as [s][k]: MN-major B
+                const uint32_t ty = tmem + TM_Y + (c & 1) * 64;
+                const uint32_t pp = sbase + OFF_V + (c & 1) * V_STAGE;     // P of chunk c
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    mma_f16kind_ss(tmem + TM_Y, sdesc_sw128(sbase + OFF_UB + kk * 32, 16, 1024),
-                                sdesc_sw128(sbase + OFF_P + kk * 32, 16, 1024), id_yq, 1);
+                    mma_f16kind_ss(ty, sdesc_sw128(sbase + OFF_UB + kk * 32, 16, 1024),
+                                   sdesc_sw128(pp + kk * 32, 16, 1024), id_yq, 1);
                     mma_f16kind_ss(tmem + TM_S, sdesc_sw128(sbase + OFF_UD + kk * 32, 16, 1024),
-                                sdesc_sw128(kb + kk * 2048, 16384, 1024), id_s, 1);
+                                   sdesc_sw128(kb + kk * 2048, 16384, 1024), id_s, 1);
                 }
                 mma_commit(&bar[B_SFULL]);
                 mma_commit(&bar[B_EMPTY0 + (c & 1)]);
-                return true;
             };
-            ok = issue_G(0) && issue_W(0) && issue_U(0) && issue_X(0);
-            for (int c = 0; ok && c < n_chunks; ++c) {
-                if (c + 1 < n_chunks) ok = issue_G(c + 1);
-                ok = ok && issue_S(c);
-                if (ok && c + 1 < n_chunks) ok = issue_W(c + 1) && issue_U(c + 1) && issue_X(c + 1);
+            // Issue whatever is ready, chain products first. Per operation the chunks go in
+            // order; the preconditions also keep every TMEM accumulator single-writer:
+            //   G(c): stage loaded, G(c-1) read by the solve group (TMEM G is single), and
+            //         W(c-1) issued (so the converters, which start on G(c), never run two
+            //         phases ahead of the CONV barrier polled for W)
+            //   W(c): T diag(beta gamma) and the converted tiles of c
+            //   U(c): T diag(beta) of c, and S(c-1) issued (it waited for U~(c-1) to be read)
+            //   X(c): U(c) issued, -W^T(c) and the fp16 state copy of c written
+            //   S(c): X(c) issued, U~ operands, P and the rescaled state of c ready
+            int nG = 0, nW = 0, nU = 0, nX = 0, nS = 0;
+            long long idle_since = clock64();
+            while (nS < n_chunks) {
+                bool progressed = false;
+                if (nS < nX && done(B_UD, nS) && done(B_P, nS) && done(B_SACC, nS)) {
+                    tc_fence_after();
+                    do_S(nS++);
+                    progressed = true;
+                } else if (nX < nU && done(B_WB, nX) && done(B_SB, nX)) {
+                    tc_fence_after();
+                    do_X(nX++);
+                    progressed = true;
+                } else if (nU < nW && nU <= nS && done(B_TB, nU)) {
+                    tc_fence_after();
+                    do_U(nU++);
+                    progressed = true;
+                } else if (nW < nG && done(B_TBG, nW) && done(B_CONV, nW)) {
+                    tc_fence_after();
+                    do_W(nW++);
+                    progressed = true;
+                } else if (nG < n_chunks && nG <= nW && done(B_FULL0 + (nG & 1), nG >> 1) &&
+                           (nG == 0 || done(B_GEMPTY, nG - 1))) {
+                    tc_fence_after();
+                    do_G(nG++);
+                    progressed = true;
+                }
+                if (progressed) {
+                    idle_since = clock64();
+                    continue;
+                }
+                if (*abort_flag) break;
+                if (clock64() - idle_since > kWaitLimit) {
+                    *abort_flag = 1;
+                    raise_error(kErrTimeout);
+                    break;
+                }
+                __nanosleep(32);              // leave the issue slots to the warps doing the work
             }
             // drain the tensor pipe before TMEM is released
             mma_commit(&bar[B_DRAIN]);
             mbar_wait_drain(&bar[B_DRAIN], 0, kWaitLimit);
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp < 4) {
+        // ================================================================ converters
+        const int u = tid - 64;               // token row 0..63 of every tile
+        for (int c = 0; c < n_chunks; ++c) {
+            float g_lo, g_hi;
+            chunk_log2_decay_scan(log_alpha, ci.bos + (int64_t)c * kC, H, ci.h, chunk_valid(c), lane, g_lo, g_hi);
+            const float fq = fast_exp2(warp == 2 ? g_lo : g_hi) * scale;     // gamma_u * scale
+            bool ok = true;
+            if (u == 0) ok = mbar_wait_bounded(&bar[B_GFULL], c & 1, abort_flag, kWaitLimit);
+            if (!named_bar_and(NB_CONV, 64, ok)) break;
+            uint8_t *qk = smem + OFF_QK + (c & 1) * QK_STAGE;
+            uint8_t *vv = smem + OFF_V + (c & 1) * V_STAGE;
+            uint8_t *rows[6] = {qk + u * 128, qk + 16384 + u * 128, qk + 8192 + u * 128,
+                                qk + 24576 + u * 128, vv + u * 128, vv + 8192 + u * 128};
+#pragma unroll
+            for (int which = 0; which < 6; ++which) {
+                const float f = (which == 2 || which == 3) ? fq : 1.f;
+                // a whole 128-byte row is rewritten, so the swizzle does not matter; the
+                // rotated order keeps the eight threads of a row group on distinct banks.
+                // All eight loads are issued before the first store.
+                uint4 v[8];
+#pragma unroll
+                for (int it = 0; it < 8; ++it) v[it] = lds128(rows[which] + (((it + u) & 7) << 4));
+#pragma unroll
+                for (int it = 0; it < 8; ++it)
+                    sts128(rows[which] + (((it + u) & 7) << 4), bf16x8_to_f16x8(v[it], f));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar[B_CONV]);
+        }
+    } else if (warp < 8) {
         // ================================================================ solve warpgroup
         const int r = tid - 128;              // TMEM lane / row
         const int t = r & 63;
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u << 16;
+        float *g2s = reinterpret_cast<float *>(smem + OFF_GATES);
+        float *gam = g2s + 64, *bet = g2s + 128;
         for (int c = 0; c < n_chunks; ++c) {
-            float *gs = reinterpret_cast<float *>(smem + OFF_GATES);
-            float *gam = gs + 64, *bet = gs + 128;
             const int64_t tok0 = ci.bos + (int64_t)c * kC;
-            const int n_valid = (int)(ci.len - (int64_t)c * kC < kC ? ci.len - (int64_t)c * kC : kC);
+            const int n_valid = chunk_valid(c);
             if (warp == 4) {
-                // gates of this chunk
                 float g_lo, g_hi;
-                chunk_log_decay_scan(log_alpha, tok0, H, ci.h, n_valid, lane, g_lo, g_hi);
-                gs[lane] = g_lo;
-                gs[lane + 32] = g_hi;
-                gam[lane] = expf(g_lo);
-                gam[lane + 32] = expf(g_hi);
+                chunk_log2_decay_scan(log_alpha, tok0, H, ci.h, n_valid, lane, g_lo, g_hi);
+                g2s[lane] = g_lo;
+                g2s[lane + 32] = g_hi;
+                gam[lane] = fast_exp2(g_lo);
+                gam[lane + 32] = fast_exp2(g_hi);
                 bet[lane] = lane < n_valid ? beta[(size_t)(tok0 + lane) * H + ci.h] : 0.f;
                 bet[lane + 32] = lane + 32 < n_valid ? beta[(size_t)(tok0 + lane + 32) * H + ci.h] : 0.f;
             }
-            // (a) G = [K K^T ; Q K^T] rows
+            // (a) G rows: K K^T (lanes 0..63), Q K^T (lanes 64..127)
             bool ok = true;
             if (r == 0) ok = mbar_wait_bounded(&bar[B_GFULL], c & 1, abort_flag, kWaitLimit);
-            if (!named_bar_and(1, 128, ok)) break;
+            if (!named_bar_and(NB_SOLVE, 128, ok)) break;
             tc_fence_after();
-            uint32_t gv[64];
-            {
-                uint32_t (&g0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&gv[0]);
-                uint32_t (&g1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&gv[32]);
-                tmem_ld_x32(tmem + lane_base + TM_G, g0);
-                tmem_ld_x32(tmem + lane_base + TM_G + 32, g1);
-                tmem_wait_ld();
-            }
+            uint32_t ga[32], gb[32];
+            tmem_ld_x32(tmem + lane_base + TM_G, ga);
+            tmem_ld_x32(tmem + lane_base + TM_G + 32, gb);
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bar[B_GEMPTY]);
-            const float gt = gs[t];
+            const float g2t = g2s[t];
             uint32_t pk[32];                  // P row (threads 64..127), fp16 pairs
             if (r < 64) {
                 const float bt = bet[t];
 #pragma unroll
-                for (int s = 0; s < 64; ++s)
-                    Ls[t * LS_LD + s] = (s < t) ? bt * __uint_as_float(gv[s]) * expf(gt - gs[s]) : 0.f;
-            } else {
-#pragma unroll
-                for (int s = 0; s < 64; s += 2) {
-                    const float p0 = (s <= t) ? scale * __uint_as_float(gv[s]) * expf(gt - gs[s]) : 0.f;
-                    const float p1 = (s + 1 <= t) ? scale * __uint_as_float(gv[s + 1]) * expf(gt - gs[s + 1]) : 0.f;
-                    pk[s >> 1] = pack_f16x2(p0, p1);
-                }
-            }
-            named_bar_sync(1, 128);
-            // (b) T = (I + L)^-1: 16x16 diagonal blocks, one column per thread in registers
-            if (r < 64) {
-                const int j = r, b0 = (j >> 4) << 4, jb = j & 15;
-                float x[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float acc = (i == jb) ? 1.f : 0.f;
-#pragma unroll
-                    for (int s = 0; s < i; ++s)
-                        if (s >= jb) acc = fmaf(-Ls[(b0 + i) * LS_LD + b0 + s], x[s], acc);
-                    x[i] = (i < jb) ? 0.f : acc;
-                }
-                named_bar_sync(3, 64);        // the 64 column threads have read their L blocks
-#pragma unroll
-                for (int i = 0; i < 16; ++i) Ls[(b0 + i) * LS_LD + j] = x[i];
-            }
-            named_bar_sync(1, 128);
-            // off-diagonal block rows: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj
-            for (int ib = 1; ib < 4; ++ib) {
-                const int w = 16 * ib, n_out = 16 * w;
-                for (int o = r; o < n_out; o += 128) {
-                    const int i = o / w, jj = o % w;
-                    float acc = 0.f;
-                    for (int s = (jj >> 4) << 4; s < w; ++s)
-                        acc = fmaf(Ls[(w + i) * LS_LD + s], Ls[s * LS_LD + jj], acc);
-                    Rt[i * 48 + jj] = acc;
-                }
-                named_bar_sync(1, 128);
-                for (int o = r; o < n_out; o += 128) {
-                    const int i = o / w, jj = o % w;
-                    float acc = 0.f;
-                    for (int m = 0; m <= i; ++m)
-                        acc = fmaf(-Ls[(w + i) * LS_LD + w + m], Rt[m * 48 + jj], acc);
-                    Ls[(w + i) * LS_LD + jj] = acc;
-                }
-                named_bar_sync(1, 128);
-            }
-            // (c) T diag(beta gamma) (rows by threads 0..63) and the input tiles in place
-            const uint32_t qk_off = OFF_QK + (c & 1) * QK_STAGE;
-            if (r < 64) {
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint4 v4;
-                    uint32_t *vv = reinterpret_cast<uint32_t *>(&v4);
+                for (int s4 = 0; s4 < 64; s4 += 4) {
+                    const float4 g4 = ldsf4(g2s + s4);
+                    const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int s = ch * 8 + 2 * e;
-                        vv[e] = pack_f16x2(Ls[t * LS_LD + s] * bet[s] * gam[s],
-                                            Ls[t * LS_LD + s + 1] * bet[s + 1] * gam[s + 1]);
+                        const int s = s4 + e;
+                        uint32_t &gr = s < 32 ? ga[s] : gb[s - 32];
+                        gr = __float_as_uint((s < t) ? bt * __uint_as_float(gr) * fast_exp2(g2t - gg[e]) : 0.f);
                     }
-                    *reinterpret_cast<uint4 *>(smem + OFF_TBG + sw128_off(t, ch)) = v4;
+                }
+#pragma unroll
+                for (int s4 = 0; s4 < 64; s4 += 4) {
+                    const uint32_t *src = s4 < 32 ? ga + s4 : gb + (s4 - 32);
+                    stsf4(Ls + t * LS_LD + s4, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
+                                                           __uint_as_float(src[2]), __uint_as_float(src[3])));
+                }
+            } else {
+#pragma unroll
+                for (int s4 = 0; s4 < 64; s4 += 4) {
+                    const float4 g4 = ldsf4(g2s + s4);
+                    const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
+                    float pv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int s = s4 + e;
+                        const float gv = __uint_as_float(s < 32 ? ga[s] : gb[s - 32]);
+                        pv[e] = (s <= t) ? scale * gv * fast_exp2(g2t - gg[e]) : 0.f;
+                    }
+                    pk[s4 >> 1] = pack_f16x2(pv[0], pv[1]);
+                    pk[(s4 >> 1) + 1] = pack_f16x2(pv[2], pv[3]);
                 }
             }
+            named_bar_sync(NB_SOLVE, 128);
+            // (b) T = (I + L)^-1
+            // 16x16 diagonal blocks: one column per thread, right-looking substitution
+            if (r < 64) {
+                const int j = r, b0 = (j >> 4) << 4, jb = j & 15;
+                float acc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = (i == jb) ? 1.f : 0.f;
+#pragma unroll
+                for (int s = 0; s < 16; ++s) {
+                    const float xs = acc[s];
+#pragma unroll
+                    for (int i = s + 1; i < 16; ++i) acc[i] = fmaf(-Ls[(b0 + i) * LS_LD + b0 + s], xs, acc[i]);
+                }
+                named_bar_sync(NB_SOLVE_LO, 64);   // every column thread has read its L block
+#pragma unroll
+                for (int i = 0; i < 16; ++i) Ls[(b0 + i) * LS_LD + j] = acc[i];
+            }
+            named_bar_sync(NB_SOLVE, 128);
+            // level 1: blocks (1,0) and (3,2): X = -T_aa (L_ab T_bb), 16x16 each
             {
-                // the stage's K, V tiles -> fp16 in place (exact); Q -> fp16(gamma_t * scale * q_t).
-                // Thread r owns token row t of the d-half (r >> 6) of each tile; a whole
-                // 128-byte row is rewritten, so the swizzle does not matter.
-                const float sc = gam[t] * scale;
-                uint8_t *rows[3] = {smem + qk_off + (r >> 6) * 16384 + t * 128,
-                                    smem + qk_off + 8192 + (r >> 6) * 16384 + t * 128,
-                                    smem + OFF_V + (c & 1) * V_STAGE + (r >> 6) * 8192 + t * 128};
+                const int pair = r >> 6, rr = r & 63;
+                const int a0 = 16 + 32 * pair, b0 = 32 * pair;   // (a, b) = (1, 0) or (3, 2)
+                const int i = rr >> 2, q4 = (rr & 3) * 4;
+                float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int which = 0; which < 3; ++which) {
-                    const float f = which == 1 ? sc : 1.f;
+                for (int k4 = 0; k4 < 16; k4 += 4) {
+                    const float4 l4 = ldsf4(Ls + (a0 + i) * LS_LD + b0 + k4);
+                    const float lk[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint4 v4 = *reinterpret_cast<uint4 *>(rows[which] + ch * 16);
-                        uint32_t *vv = reinterpret_cast<uint32_t *>(&v4);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) vv[e] = pack_f16x2(bf_lo(vv[e]) * f, bf_hi(vv[e]) * f);
-                        *reinterpret_cast<uint4 *>(rows[which] + ch * 16) = v4;
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 tr = ldsf4(Ls + (b0 + k4 + e) * LS_LD + b0 + q4);
+                        m[0] = fmaf(lk[e], tr.x, m[0]);
+                        m[1] = fmaf(lk[e], tr.y, m[1]);
+                        m[2] = fmaf(lk[e], tr.z, m[2]);
+                        m[3] = fmaf(lk[e], tr.w, m[3]);
                     }
                 }
+                stsf4(Rt + pair * 16 * 16 + i * 16 + q4, make_float4(m[0], m[1], m[2], m[3]));
+                named_bar_sync(NB_SOLVE, 128);
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int k4 = 0; k4 < 16; k4 += 4) {
+                    const float4 t4 = ldsf4(Ls + (a0 + i) * LS_LD + a0 + k4);
+                    const float tk[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 mr = ldsf4(Rt + pair * 16 * 16 + (k4 + e) * 16 + q4);
+                        x[0] = fmaf(-tk[e], mr.x, x[0]);
+                        x[1] = fmaf(-tk[e], mr.y, x[1]);
+                        x[2] = fmaf(-tk[e], mr.z, x[2]);
+                        x[3] = fmaf(-tk[e], mr.w, x[3]);
+                    }
+                }
+                stsf4(Ls + (a0 + i) * LS_LD + b0 + q4, make_float4(x[0], x[1], x[2], x[3]));
+            }
+            named_bar_sync(NB_SOLVE, 128);
+            // level 2: rows 32..63 x cols 0..31: X = -T_B (L_BA T_A), 32x32 each.
+            // Warp w owns 8 columns (8w..8w+7), lane = row.
+            {
+                const int w = warp - 4, i = lane, c0 = 8 * w;
+                const int k_lo = w >= 2 ? 16 : 0;        // T_A is zero in rows 0..15 of cols 16..31
+                float m[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m[e] = 0.f;
+#pragma unroll
+                for (int k4 = 0; k4 < 32; k4 += 4) {
+                    if (k4 < k_lo) continue;
+                    const float4 l4 = ldsf4(Ls + (32 + i) * LS_LD + k4);
+                    const float lk[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 ta = ldsf4(Ls + (k4 + e) * LS_LD + c0);
+                        const float4 tb = ldsf4(Ls + (k4 + e) * LS_LD + c0 + 4);
+                        m[0] = fmaf(lk[e], ta.x, m[0]);
+                        m[1] = fmaf(lk[e], ta.y, m[1]);
+                        m[2] = fmaf(lk[e], ta.z, m[2]);
+                        m[3] = fmaf(lk[e], ta.w, m[3]);
+                        m[4] = fmaf(lk[e], tb.x, m[4]);
+                        m[5] = fmaf(lk[e], tb.y, m[5]);
+                        m[6] = fmaf(lk[e], tb.z, m[6]);
+                        m[7] = fmaf(lk[e], tb.w, m[7]);
+                    }
+                }
+                stsf4(Rt + i * RT_LD + c0, make_float4(m[0], m[1], m[2], m[3]));
+                stsf4(Rt + i * RT_LD + c0 + 4, make_float4(m[4], m[5], m[6], m[7]));
+                named_bar_sync(NB_SOLVE, 128);
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = 0.f;
+#pragma unroll
+                for (int k4 = 0; k4 < 32; k4 += 4) {
+                    const float4 t4 = ldsf4(Ls + (32 + i) * LS_LD + 32 + k4);
+                    const float tk[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 ma = ldsf4(Rt + (k4 + e) * RT_LD + c0);
+                        const float4 mb = ldsf4(Rt + (k4 + e) * RT_LD + c0 + 4);
+                        x[0] = fmaf(-tk[e], ma.x, x[0]);
+                        x[1] = fmaf(-tk[e], ma.y, x[1]);
+                        x[2] = fmaf(-tk[e], ma.z, x[2]);
+                        x[3] = fmaf(-tk[e], ma.w, x[3]);
+                        x[4] = fmaf(-tk[e], mb.x, x[4]);
+                        x[5] = fmaf(-tk[e], mb.y, x[5]);
+                        x[6] = fmaf(-tk[e], mb.z, x[6]);
+                        x[7] = fmaf(-tk[e], mb.w, x[7]);
+                    }
+                }
+                stsf4(Ls + (32 + i) * LS_LD + c0, make_float4(x[0], x[1], x[2], x[3]));
+                stsf4(Ls + (32 + i) * LS_LD + c0 + 4, make_float4(x[4], x[5], x[6], x[7]));
+            }
+            named_bar_sync(NB_SOLVE, 128);
+            // (c) T diag(beta gamma), rows by threads 0..63. The row is computed into registers
+            // first, then stored, so no load waits behind a store.
+            float trow[64];
+            {
+#pragma unroll
+                for (int s4 = 0; s4 < 64; s4 += 4) {
+                    const float4 t4 = ldsf4(Ls + t * LS_LD + s4);
+                    const float4 b4 = ldsf4(bet + s4);
+                    const float4 c4 = r < 64 ? ldsf4(gam + s4) : make_float4(1.f, 1.f, 1.f, 1.f);
+                    trow[s4] = t4.x * b4.x * c4.x;
+                    trow[s4 + 1] = t4.y * b4.y * c4.y;
+                    trow[s4 + 2] = t4.z * b4.z * c4.z;
+                    trow[s4 + 3] = t4.w * b4.w * c4.w;
+                }
+            }
+            if (r < 64) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) sts128(smem + OFF_TBG + sw128_off(t, ch), pack8_f16(trow + ch * 8));
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar[B_TBG]);
-            // (d) T diag(beta) once the previous chunk's U^T product is done (x_full(c-1))
+            // (d) T diag(beta) (rows by threads 64..127) once the previous chunk's U^T product
+            // is done (x_full(c-1))
             ok = true;
             if (c > 0 && r == 0) ok = mbar_wait_bounded(&bar[B_XFULL], (c - 1) & 1, abort_flag, kWaitLimit);
-            if (!named_bar_and(1, 128, ok)) break;
+            if (!named_bar_and(NB_SOLVE, 128, ok)) break;
             if (r >= 64) {
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint4 v4;
-                    uint32_t *vv = reinterpret_cast<uint32_t *>(&v4);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = ch * 8 + 2 * e;
-                        vv[e] = pack_f16x2(Ls[t * LS_LD + s] * bet[s], Ls[t * LS_LD + s + 1] * bet[s + 1]);
-                    }
-                    *reinterpret_cast<uint4 *>(smem + OFF_TB + sw128_off(t, ch)) = v4;
-                }
+                for (int ch = 0; ch < 8; ++ch) sts128(smem + OFF_TB + sw128_off(t, ch), pack8_f16(trow + ch * 8));
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar[B_TB]);
-            // (e) P once the previous chunk's state products are done (s_full(c-1))
-            ok = true;
-            if (c > 0 && r == 0) ok = mbar_wait_bounded(&bar[B_SFULL], (c - 1) & 1, abort_flag, kWaitLimit);
-            if (!named_bar_and(1, 128, ok)) break;
-            if (r >= 64) {
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4 *>(smem + OFF_P + sw128_off(t, ch)) =
-                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&bar[B_P]);
             // (f) -W^T from its accumulator into the MN-major operand [k][t]
             ok = true;
             if (r == 0) ok = mbar_wait_bounded(&bar[B_WFULL], c & 1, abort_flag, kWaitLimit);
-            if (!named_bar_and(1, 128, ok)) break;
+            if (!named_bar_and(NB_SOLVE, 128, ok)) break;
             tc_fence_after();
-            {
-                uint32_t (&w0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&gv[0]);
-                uint32_t (&w1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&gv[32]);
-                tmem_ld_x32(tmem + lane_base + TM_W, w0);
-                tmem_ld_x32(tmem + lane_base + TM_W + 32, w1);
-                tmem_wait_ld();
-            }
+            tmem_ld_x32(tmem + lane_base + TM_W, ga);
+            tmem_ld_x32(tmem + lane_base + TM_W + 32, gb);
+            tmem_wait_ld();
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                uint4 v4;
-                uint32_t *vv = reinterpret_cast<uint32_t *>(&v4);
+                float v8[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    vv[e] = pack_f16x2(-__uint_as_float(gv[ch * 8 + 2 * e]), -__uint_as_float(gv[ch * 8 + 2 * e + 1]));
-                *reinterpret_cast<uint4 *>(smem + OFF_WB + sw128_off(r, ch)) = v4;
+                for (int e = 0; e < 8; ++e) {
+                    const int s = ch * 8 + e;
+                    v8[e] = -__uint_as_float(s < 32 ? ga[s] : gb[s - 32]);
+                }
+                sts128(smem + OFF_WB + sw128_off(r, ch), pack8_f16(v8));
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[B_WB]);
+            // (e) P into the V stage of this chunk, free once U^T(c) is done (x_full(c));
+            // S(c) reads it, and the stage is reloaded only after S(c) completes
+            ok = true;
+            if (r == 0) ok = mbar_wait_bounded(&bar[B_XFULL], c & 1, abort_flag, kWaitLimit);
+            if (!named_bar_and(NB_SOLVE, 128, ok)) break;
+            if (r >= 64) {
+                uint8_t *pdst = smem + OFF_V + (c & 1) * V_STAGE;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    sts128(pdst + sw128_off(t, ch), make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar[B_P]);
         }
-    } else if (warp >= 8) {
+    } else {
         // ================================================================ state warpgroup
         const int r = tid - 256;              // TMEM lane = value index v
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u << 16;
-        // every warp scans the log decays itself (bit-identical to the solve warpgroup's)
+        float *decw = reinterpret_cast<float *>(smem + OFF_DEC) + (warp - 8) * 64;
         auto scan = [&](int c, float &g_lo, float &g_hi) {
-            const int64_t tok0 = ci.bos + (int64_t)c * kC;
-            const int n_valid = (int)(ci.len - (int64_t)c * kC < kC ? ci.len - (int64_t)c * kC : kC);
-            chunk_log_decay_scan(log_alpha, tok0, H, ci.h, n_valid, lane, g_lo, g_hi);
+            chunk_log2_decay_scan(log_alpha, ci.bos + (int64_t)c * kC, H, ci.h, chunk_valid(c), lane, g_lo, g_hi);
         };
         float g_lo = 0.f, g_hi = 0.f;
         if (n_chunks > 0) scan(0, g_lo, g_hi);
         // S0 -> TMEM (scaled by gamma_C of chunk 0) and its fp16 copy
         {
-            const float gC = expf(__shfl_sync(0xffffffffu, g_hi, 31));
+            const float gC = fast_exp2(__shfl_sync(0xffffffffu, g_hi, 31));
             const float *src = S0 ? S0 + state_off + (size_t)r * kD : nullptr;
             if (n_chunks == 0) {
                 if (S_T) {
@@ -529,13 +675,11 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     uint8_t *sb_half = smem + OFF_SB + (q4 >> 1) * 16384;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int e0 = ch * 8;
-                        *reinterpret_cast<uint4 *>(sb_half + sw128_off(r, (q4 & 1) * 4 + ch)) = make_uint4(
-                            pack_f16x2(__uint_as_float(sv[e0]), __uint_as_float(sv[e0 + 1])),
-                            pack_f16x2(__uint_as_float(sv[e0 + 2]), __uint_as_float(sv[e0 + 3])),
-                            pack_f16x2(__uint_as_float(sv[e0 + 4]), __uint_as_float(sv[e0 + 5])),
-                            pack_f16x2(__uint_as_float(sv[e0 + 6]), __uint_as_float(sv[e0 + 7])));
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float v8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(sv[cc * 8 + e]);
+                        sts128(sb_half + sw128_off(r, (q4 & 1) * 4 + cc), pack8_f16(v8));
                     }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gC);
@@ -545,106 +689,134 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bar[B_SB]);
+                mbar_arrive(&bar[B_SACC]);
             }
         }
         for (int c = 0; c < n_chunks; ++c) {
             const int64_t tok0 = ci.bos + (int64_t)c * kC;
-            const int n_valid = (int)(ci.len - (int64_t)c * kC < kC ? ci.len - (int64_t)c * kC : kC);
+            const int n_valid = chunk_valid(c);
             const bool last = (c + 1 == n_chunks);
-            // exp(g_C - g_s) of this chunk, two per lane
-            const float gC = __shfl_sync(0xffffffffu, g_hi, 31);
-            const float dec_lo = expf(gC - g_lo), dec_hi = expf(gC - g_hi);
-            // the next chunk's scan (its gamma_C scales the carried state below)
+            // exp(g_C - g_s) of this chunk into the warp's own slot (read back as broadcasts)
+            const float g2C = __shfl_sync(0xffffffffu, g_hi, 31);
+            __syncwarp();                     // the previous chunk's reads of decw are done
+            decw[lane] = fast_exp2(g2C - g_lo);
+            decw[lane + 32] = fast_exp2(g2C - g_hi);
+            __syncwarp();
+            // the next chunk's scan: its gamma_C rescales the carried state below
             float n_lo = 0.f, n_hi = 0.f;
             if (!last) scan(c + 1, n_lo, n_hi);
-            const float gC_next = last ? 1.f : expf(__shfl_sync(0xffffffffu, n_hi, 31));
-            // E2: U~^T -> fp16 operands (plain and decayed)
+            const float gC_next = last ? 1.f : fast_exp2(__shfl_sync(0xffffffffu, n_hi, 31));
+            // E2: U~^T -> fp16 operands (plain and decayed). The previous chunk's y copies
+            // read the same buffers: every issuer waits for them before the barrier.
+            bulk_wait_read();
             bool ok = true;
             if (r == 0) ok = mbar_wait_bounded(&bar[B_XFULL], c & 1, abort_flag, kWaitLimit);
-            if (!named_bar_and(2, 128, ok)) break;
+            if (!named_bar_and(NB_STATE, 128, ok)) break;
             tc_fence_after();
             {
-                uint32_t u[64];
-                uint32_t (&u0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&u[0]);
-                uint32_t (&u1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&u[32]);
-                tmem_ld_x32(tmem + lane_base + TM_U, u0);
-                tmem_ld_x32(tmem + lane_base + TM_U + 32, u1);
+                uint32_t ua[32], ub[32];
+                tmem_ld_x32(tmem + lane_base + TM_U, ua);
+                tmem_ld_x32(tmem + lane_base + TM_U + 32, ub);
                 tmem_wait_ld();
+                float dd[64];
+#pragma unroll
+                for (int s4 = 0; s4 < 64; s4 += 4) {
+                    const float4 d4 = ldsf4(decw + s4);
+                    dd[s4] = d4.x;
+                    dd[s4 + 1] = d4.y;
+                    dd[s4 + 2] = d4.z;
+                    dd[s4 + 3] = d4.w;
+                }
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    uint4 a4, d4;
-                    uint32_t *aa = reinterpret_cast<uint32_t *>(&a4), *dd = reinterpret_cast<uint32_t *>(&d4);
+                    float pl[8], dc[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = ch * 8 + 2 * e;
-                        const float u0f = __uint_as_float(u[s]), u1f = __uint_as_float(u[s + 1]);
-                        const float d0 = __shfl_sync(0xffffffffu, s < 32 ? dec_lo : dec_hi, s & 31);
-                        const float d1 = __shfl_sync(0xffffffffu, s + 1 < 32 ? dec_lo : dec_hi, (s + 1) & 31);
-                        aa[e] = pack_f16x2(u0f, u1f);
-                        dd[e] = pack_f16x2(u0f * d0, u1f * d1);
+                    for (int e = 0; e < 8; ++e) {
+                        const int s = ch * 8 + e;
+                        pl[e] = __uint_as_float(s < 32 ? ua[s] : ub[s - 32]);
+                        dc[e] = pl[e] * dd[s];
                     }
-                    *reinterpret_cast<uint4 *>(smem + OFF_UB + sw128_off(r, ch)) = a4;
-                    *reinterpret_cast<uint4 *>(smem + OFF_UD + sw128_off(r, ch)) = d4;
+                    sts128(smem + OFF_UB + sw128_off(r, ch), pack8_f16(pl));
+                    sts128(smem + OFF_UD + sw128_off(r, ch), pack8_f16(dc));
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[B_UD]);
-            // E3: y out, S carry
+            // E3: the fp16 copy of S_{c+1} and the fp32 state rescaled by the next gamma_C
+            // (both gate the next chunk), then y
             ok = true;
             if (r == 0) ok = mbar_wait_bounded(&bar[B_SFULL], c & 1, abort_flag, kWaitLimit);
-            if (!named_bar_and(2, 128, ok)) break;
+            if (!named_bar_and(NB_STATE, 128, ok)) break;
             tc_fence_after();
-            {
-                uint32_t yv[64];
-                uint32_t (&y0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&yv[0]);
-                uint32_t (&y1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&yv[32]);
-                tmem_ld_x32(tmem + lane_base + TM_Y, y0);
-                tmem_ld_x32(tmem + lane_base + TM_Y + 32, y1);
-                tmem_wait_ld();
-                TY *yp = y + ((size_t)tok0 * H + ci.h) * kD + r;
-#pragma unroll 8
-                for (int tt = 0; tt < 64; ++tt)
-                    if (tt < n_valid) yp[(size_t)tt * H * kD] = from_f32<TY>(__uint_as_float(yv[tt]));
-            }
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t sv[32];
-                tmem_ld_x32(tmem + lane_base + TM_S + q4 * 32, sv);
+            for (int h2 = 0; h2 < 2; ++h2) {
+                // two 32-column loads in flight, then the fp16 copy (or S_T) and the rescale
+                uint32_t sa[32], sb[32];
+                tmem_ld_x32(tmem + lane_base + TM_S + h2 * 64, sa);
+                tmem_ld_x32(tmem + lane_base + TM_S + h2 * 64 + 32, sb);
                 tmem_wait_ld();
                 if (last) {
                     if (S_T) {
-                        float *dst = S_T + state_off + (size_t)r * kD + q4 * 32;
+                        float *dst = S_T + state_off + (size_t)r * kD + h2 * 64;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            store4(dst + i, make_float4(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1]),
-                                                        __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])));
+                        for (int i = 0; i < 64; i += 4) {
+                            const uint32_t *sv = i < 32 ? sa + i : sb + (i - 32);
+                            store4(dst + i, make_float4(__uint_as_float(sv[0]), __uint_as_float(sv[1]),
+                                                        __uint_as_float(sv[2]), __uint_as_float(sv[3])));
+                        }
                     }
                 } else {
-                    uint8_t *sb_half = smem + OFF_SB + (q4 >> 1) * 16384;
+                    uint8_t *sb_half = smem + OFF_SB + h2 * 16384;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int e0 = ch * 8;
-                        *reinterpret_cast<uint4 *>(sb_half + sw128_off(r, (q4 & 1) * 4 + ch)) = make_uint4(
-                            pack_f16x2(__uint_as_float(sv[e0]), __uint_as_float(sv[e0 + 1])),
-                            pack_f16x2(__uint_as_float(sv[e0 + 2]), __uint_as_float(sv[e0 + 3])),
-                            pack_f16x2(__uint_as_float(sv[e0 + 4]), __uint_as_float(sv[e0 + 5])),
-                            pack_f16x2(__uint_as_float(sv[e0 + 6]), __uint_as_float(sv[e0 + 7])));
+                    for (int cc = 0; cc < 8; ++cc) {
+                        float v8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int i = cc * 8 + e;
+                            v8[e] = __uint_as_float(i < 32 ? sa[i] : sb[i - 32]);
+                        }
+                        sts128(sb_half + sw128_off(r, cc), pack8_f16(v8));
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gC_next);
-                    tmem_st_x32(tmem + lane_base + TM_S + q4 * 32, sv);
+                    for (int i = 0; i < 32; ++i) {
+                        sa[i] = __float_as_uint(__uint_as_float(sa[i]) * gC_next);
+                        sb[i] = __float_as_uint(__uint_as_float(sb[i]) * gC_next);
+                    }
+                    tmem_st_x32(tmem + lane_base + TM_S + h2 * 64, sa);
+                    tmem_st_x32(tmem + lane_base + TM_S + h2 * 64 + 32, sb);
                 }
             }
             if (!last) {
-                tmem_wait_st();
                 fence_proxy_async_smem();
+                tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bar[B_SB]);
+                mbar_arrive(&bar[B_SACC]);
+            }
+            {
+                // y: Y^T column v of every token into the staging tile [t][v] (the U~ operand
+                // buffers, idle until the next chunk's E2), then one bulk copy per token row
+                uint32_t ya[32], yb[32];
+                tmem_ld_x32(tmem + lane_base + TM_Y + (c & 1) * 64, ya);
+                tmem_ld_x32(tmem + lane_base + TM_Y + (c & 1) * 64 + 32, yb);
+                tmem_wait_ld();
+                TY *ys = reinterpret_cast<TY *>(smem + OFF_YST);
+#pragma unroll
+                for (int tt = 0; tt < 64; ++tt)
+                    ys[tt * kD + r] = from_f32<TY>(__uint_as_float(tt < 32 ? ya[tt] : yb[tt - 32]));
+                fence_proxy_async_smem();
+                named_bar_sync(NB_STATE, 128);
+                const int tt = (warp - 8) * 16 + lane;
+                if (lane < 16 && tt < n_valid) {
+                    bulk_store_s2g(y + ((size_t)(tok0 + tt) * H + ci.h) * kD, ys + tt * kD, kD * sizeof(TY));
+                    bulk_commit();
+                }
             }
             g_lo = n_lo;
             g_hi = n_hi;
         }
+        bulk_wait_all();                      // y copies complete before the CTA exits
     }
 
     // ---- teardown: every role has left its loop and drained its own async work
