@@ -457,6 +457,49 @@ def cpu_baseline(inp, H):
                       f"workload ({n_th} token-heads, {dt:.1f} s); tokens/s = token-heads/s / H"}
 
 
+def run_case(args):
+    """A few launches of one kernel on a named shape, nothing else (for ncu captures):
+    --case prefill:S,T,H   (bf16, d=128, chunk 64, fp32 y)
+    --case decode:N        (N sequences x 32 heads, d=128, fp32 state)
+    --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)"""
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    import workloads as W
+    kind, _, shape = args.case.partition(":")
+    dims = [int(x) for x in shape.split(",")] if shape else []
+    torch.cuda.set_device(0)
+    if kind == "prefill":
+        n_seq, T, H = dims
+        w = W.Workload("case", "bf16", (T,) * n_seq, H, 128, 128, 64, seed=1)
+        inp = W.make_prefill_inputs(w, with_gate=False)
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        for _ in range(args.reps):
+            gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
+                          cu_seqlens_host=inp["cu_seqlens"])
+    elif kind == "decode":
+        (n,) = dims
+        x = {k: v.cuda() for k, v in W.make_decode_inputs(W.WORKLOADS["decode"], 0, n_seq=n).items()}
+        S = torch.zeros(n, 32, 128, 128, device="cuda")
+        for _ in range(args.reps):
+            gdn.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S)
+    elif kind == "gate_norm":
+        (rows,) = dims
+        g = torch.Generator().manual_seed(0)
+        y = torch.randn(rows, 128, generator=g).cuda()
+        z = torch.randn(rows, 128, generator=g).to(torch.bfloat16).cuda()
+        wn = (torch.randn(128, generator=g) * 0.02).cuda()
+        for _ in range(args.reps):
+            gdn.gate_norm(y, z, wn, out_dtype=torch.bfloat16)
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    torch.cuda.synchronize()
+    status = gdn.device_error()
+    print(f"case {args.case} x{args.reps}: {status}")
+    if status != "GDN_OK":
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -465,7 +508,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, help="profiling case, e.g. prefill:4,4096,16")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local, pg = dist_setup(args)

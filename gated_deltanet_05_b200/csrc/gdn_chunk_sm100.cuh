@@ -33,9 +33,9 @@
 //   warp 0      TMA producer: K, Q, V tiles of each chunk (2-stage ring, 128B swizzle)
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 2-3   converters: the stage's K, V -> fp16 and Q -> fp16(gamma scale q), in place
-//   warps 4-7   "solve" warpgroup: L and P from G, T = (I + L)^-1 in fp32 (16x16 diagonal
-//               blocks by forward substitution, then two levels of block merges), the
-//               fp16 T/P operands and -W^T from its TMEM accumulator
+//   warps 4-7   "solve" warpgroup: L and P from G, T = (I + L)^-1 (16x16 diagonal blocks
+//               by fp32 forward substitution, then two levels of block merges on tf32
+//               mma.sync tiles), the fp16 T/P operands and -W^T from its TMEM accumulator
 //   warps 8-11  "state" warpgroup: U~ -> fp16 operands, the fp16 state copy, y out,
 //               the state carry (scale by gamma_C), S0 in and S_T out
 // The state warpgroup publishes the fp16 copy of S_{c+1} and the rescaled fp32 state
@@ -77,12 +77,13 @@ constexpr uint32_t OFF_TBG = 188416;    // 8 KB fp16 T diag(beta gamma) [64 t][6
 constexpr uint32_t OFF_TB = 196608;     // 8 KB fp16 T diag(beta)
 constexpr uint32_t OFF_LS = 204800;     // fp32 [64][68]: L, then T in place
 constexpr int LS_LD = 68;
-constexpr uint32_t OFF_RT = OFF_LS + 64 * LS_LD * 4;     // fp32 merge temp, [32][36] at most
-constexpr int RT_LD = 36;
-constexpr uint32_t OFF_GATES = OFF_RT + 32 * RT_LD * 4;  // {g2, gamma, beta}[64] fp32 of the solve's chunk
-constexpr uint32_t OFF_DEC = OFF_GATES + 3 * 64 * 4;     // state warpgroup: exp(g_C - g)[64] per warp
+constexpr uint32_t OFF_RT = OFF_LS + 64 * LS_LD * 4;     // fp32 merge temp: [32][8] per solve warp
+constexpr int RT_LD = 36;                                // (region sized [32][36])
+constexpr float kSpanMax = 240.f;       // log2 span of a chunk's decays for the factored Gamma
+constexpr uint32_t OFF_GATES = OFF_RT + 32 * RT_LD * 4;  // {g2, gamma, beta, 2^(m - g2)}[64] fp32 of the solve's chunk
+constexpr uint32_t OFF_DEC = OFF_GATES + 4 * 64 * 4;     // state warpgroup: exp(g_C - g)[64] per warp
 constexpr uint32_t OFF_BAR = OFF_DEC + 4 * 64 * 4;       // mbarriers
-constexpr int N_BAR = 18;
+constexpr int N_BAR = 19;
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BAR * 8;       // tmem base, abort flag, chain's sequence
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;        // + alignment slack
@@ -94,7 +95,7 @@ constexpr uint32_t TM_S = 0, TM_G = 128, TM_W = 192, TM_U = 256, TM_Y = 320, TM_
 // barrier indices
 enum {
     B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_GFULL, B_GEMPTY, B_CONV, B_TBG, B_WFULL, B_TB,
-    B_WB, B_P, B_XFULL, B_UD, B_SFULL, B_SB, B_SACC, B_DRAIN
+    B_WB, B_P, B_XFULL, B_UD, B_SFULL, B_SB, B_SACC, B_UFULL, B_DRAIN
 };
 static_assert(B_DRAIN + 1 == N_BAR, "barrier count");
 
@@ -259,60 +260,68 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint32_t id_yq = idesc_f32acc(kFmtF16, 128, 64, 0, 0);
             const uint32_t id_s = idesc_f32acc(kFmtF16, 128, 128, 0, 1);
             auto done = [&](int b, int parity) { return mbar_test(&bar[b], parity & 1); };
+            // Base descriptors, computed once; a k-step adds a constant to the start address
+            // field (addresses < 256 KB keep it inside its 14 bits).
+            const uint64_t dqk0 = sdesc_sw128(sbase + OFF_QK, 16, 1024);
+            const uint64_t dkt0 = sdesc_sw128(sbase + OFF_QK, 16384, 1024);     // K^T / K as MN-major
+            const uint64_t dvt0 = sdesc_sw128(sbase + OFF_V, 8192, 1024);       // V^T MN-major
+            const uint64_t dtbg = sdesc_sw128(sbase + OFF_TBG, 16, 1024);
+            const uint64_t dtb = sdesc_sw128(sbase + OFF_TB, 16, 1024);
+            const uint64_t dsb = sdesc_sw128(sbase + OFF_SB, 16, 1024);
+            const uint64_t dwb = sdesc_sw128(sbase + OFF_WB, 8192, 1024);
+            const uint64_t dub = sdesc_sw128(sbase + OFF_UB, 16, 1024);
+            const uint64_t dud = sdesc_sw128(sbase + OFF_UD, 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(sbase + OFF_V, 16, 1024);          // P in the V stage
+#define GDN_DOFF(bytes) ((uint64_t)((bytes) >> 4))
             auto do_G = [&](int c) {
-                const uint32_t qk = sbase + OFF_QK + (c & 1) * QK_STAGE;
+                const uint64_t base = dqk0 + GDN_DOFF((c & 1) * QK_STAGE);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a = qk + (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_f16kind_ss(tmem + TM_G, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id_g, kk > 0);
+                    const uint64_t d = base + GDN_DOFF((kk >> 2) * 16384 + (kk & 3) * 32);
+                    mma_f16kind_ss(tmem + TM_G, d, d, id_g, kk > 0);
                 }
                 mma_commit(&bar[B_GFULL]);
             };
             auto do_W = [&](int c) {
-                const uint32_t kt = sbase + OFF_QK + (c & 1) * QK_STAGE;   // K^T: MN-major, LBO 16 KB
+                const uint64_t kt = dkt0 + GDN_DOFF((c & 1) * QK_STAGE);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16kind_ss(tmem + TM_W, sdesc_sw128(kt + kk * 2048, 16384, 1024),
-                                   sdesc_sw128(sbase + OFF_TBG + kk * 32, 16, 1024), id_wu, kk > 0);
+                    mma_f16kind_ss(tmem + TM_W, kt + GDN_DOFF(kk * 2048), dtbg + GDN_DOFF(kk * 32), id_wu, kk > 0);
                 mma_commit(&bar[B_WFULL]);
             };
             auto do_U = [&](int c) {
-                const uint32_t vt = sbase + OFF_V + (c & 1) * V_STAGE;     // V^T: MN-major, LBO 8 KB
+                const uint64_t vt = dvt0 + GDN_DOFF((c & 1) * V_STAGE);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16kind_ss(tmem + TM_U, sdesc_sw128(vt + kk * 2048, 8192, 1024),
-                                   sdesc_sw128(sbase + OFF_TB + kk * 32, 16, 1024), id_wu, kk > 0);
+                    mma_f16kind_ss(tmem + TM_U, vt + GDN_DOFF(kk * 2048), dtb + GDN_DOFF(kk * 32), id_wu, kk > 0);
+                mma_commit(&bar[B_UFULL]);
             };
             auto do_X = [&](int c) {
-                const uint32_t qk = sbase + OFF_QK + (c & 1) * QK_STAGE;
+                const uint64_t q0 = dqk0 + GDN_DOFF((c & 1) * QK_STAGE + 8192);
                 const uint32_t ty = tmem + TM_Y + (c & 1) * 64;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a = sbase + OFF_SB + (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint64_t a = dsb + GDN_DOFF((kk >> 2) * 16384 + (kk & 3) * 32);
                     // U~^T += S^T (-W^T): B = -W^T stored [k][t], MN-major
-                    mma_f16kind_ss(tmem + TM_U, sdesc_sw128(a, 16, 1024),
-                                   sdesc_sw128(sbase + OFF_WB + kk * 2048, 8192, 1024), id_xw, 1);
+                    mma_f16kind_ss(tmem + TM_U, a, dwb + GDN_DOFF(kk * 2048), id_xw, 1);
                     // Y^T = S^T (gamma scale Q)^T: B = Q rows (K-major), Q at +8 KB / +24 KB
-                    mma_f16kind_ss(ty, sdesc_sw128(a, 16, 1024),
-                                   sdesc_sw128(qk + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                   id_yq, kk > 0);
+                    mma_f16kind_ss(ty, a, q0 + GDN_DOFF((kk >> 2) * 16384 + (kk & 3) * 32), id_yq, kk > 0);
                 }
                 mma_commit(&bar[B_XFULL]);
             };
             auto do_S = [&](int c) {
-                const uint32_t kb = sbase + OFF_QK + (c & 1) * QK_STAGE;   // K as [s][k]: MN-major B
+                const uint64_t kb = dkt0 + GDN_DOFF((c & 1) * QK_STAGE);      // K as [s][k]: MN-major B
+                const uint64_t pp = dv0 + GDN_DOFF((c & 1) * V_STAGE);        // P of chunk c
                 const uint32_t ty = tmem + TM_Y + (c & 1) * 64;
-                const uint32_t pp = sbase + OFF_V + (c & 1) * V_STAGE;     // P of chunk c
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    mma_f16kind_ss(ty, sdesc_sw128(sbase + OFF_UB + kk * 32, 16, 1024),
-                                   sdesc_sw128(pp + kk * 32, 16, 1024), id_yq, 1);
-                    mma_f16kind_ss(tmem + TM_S, sdesc_sw128(sbase + OFF_UD + kk * 32, 16, 1024),
-                                   sdesc_sw128(kb + kk * 2048, 16384, 1024), id_s, 1);
+                    mma_f16kind_ss(ty, dub + GDN_DOFF(kk * 32), pp + GDN_DOFF(kk * 32), id_yq, 1);
+                    mma_f16kind_ss(tmem + TM_S, dud + GDN_DOFF(kk * 32), kb + GDN_DOFF(kk * 2048), id_s, 1);
                 }
                 mma_commit(&bar[B_SFULL]);
                 mma_commit(&bar[B_EMPTY0 + (c & 1)]);
             };
+#undef GDN_DOFF
             // Issue whatever is ready, chain products first. Per operation the chunks go in
             // order; the preconditions also keep every TMEM accumulator single-writer:
             //   G(c): stage loaded, G(c-1) read by the solve group (TMEM G is single), and
@@ -322,30 +331,45 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             //   U(c): T diag(beta) of c, and S(c-1) issued (it waited for U~(c-1) to be read)
             //   X(c): U(c) issued, -W^T(c) and the fp16 state copy of c written
             //   S(c): X(c) issued, U~ operands, P and the rescaled state of c ready
+            // A barrier phase seen complete is remembered until its operation is issued, so
+            // each pass re-tests only what is still pending.
             int nG = 0, nW = 0, nU = 0, nX = 0, nS = 0;
+            uint32_t seen = 0;                // bit per (operation, barrier) seen complete
+            enum : uint32_t { kS_UD = 1, kS_P = 2, kS_SACC = 4, kX_WB = 8, kX_SB = 16, kU_TB = 32,
+                              kW_TBG = 64, kW_CONV = 128, kG_FULL = 256, kG_EMPTY = 512 };
+            auto ready = [&](uint32_t bit, int b, int parity) {
+                if (seen & bit) return true;
+                if (done(b, parity)) { seen |= bit; return true; }
+                return false;
+            };
             long long idle_since = clock64();
             while (nS < n_chunks) {
                 bool progressed = false;
-                if (nS < nX && done(B_UD, nS) && done(B_P, nS) && done(B_SACC, nS)) {
+                if (nS < nX && ready(kS_UD, B_UD, nS) && ready(kS_P, B_P, nS) && ready(kS_SACC, B_SACC, nS)) {
                     tc_fence_after();
                     do_S(nS++);
+                    seen &= ~(kS_UD | kS_P | kS_SACC);
                     progressed = true;
-                } else if (nX < nU && done(B_WB, nX) && done(B_SB, nX)) {
+                } else if (nX < nU && ready(kX_WB, B_WB, nX) && ready(kX_SB, B_SB, nX)) {
                     tc_fence_after();
                     do_X(nX++);
+                    seen &= ~(kX_WB | kX_SB);
                     progressed = true;
-                } else if (nU < nW && nU <= nS && done(B_TB, nU)) {
-                    tc_fence_after();
-                    do_U(nU++);
-                    progressed = true;
-                } else if (nW < nG && done(B_TBG, nW) && done(B_CONV, nW)) {
+                } else if (nW < nG && ready(kW_TBG, B_TBG, nW) && ready(kW_CONV, B_CONV, nW)) {
                     tc_fence_after();
                     do_W(nW++);
+                    seen &= ~(kW_TBG | kW_CONV);
                     progressed = true;
-                } else if (nG < n_chunks && nG <= nW && done(B_FULL0 + (nG & 1), nG >> 1) &&
-                           (nG == 0 || done(B_GEMPTY, nG - 1))) {
+                } else if (nU < nW && nU <= nS && ready(kU_TB, B_TB, nU)) {
+                    tc_fence_after();
+                    do_U(nU++);
+                    seen &= ~kU_TB;
+                    progressed = true;
+                } else if (nG < n_chunks && nG <= nW && ready(kG_FULL, B_FULL0 + (nG & 1), nG >> 1) &&
+                           (nG == 0 || ready(kG_EMPTY, B_GEMPTY, nG - 1))) {
                     tc_fence_after();
                     do_G(nG++);
+                    seen &= ~(kG_FULL | kG_EMPTY);
                     progressed = true;
                 }
                 if (progressed) {
@@ -358,7 +382,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     raise_error(kErrTimeout);
                     break;
                 }
-                __nanosleep(32);              // leave the issue slots to the warps doing the work
+                __nanosleep(20);              // leave the issue slots to the warps doing the work
             }
             // drain the tensor pipe before TMEM is released
             mma_commit(&bar[B_DRAIN]);
@@ -378,18 +402,24 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             uint8_t *vv = smem + OFF_V + (c & 1) * V_STAGE;
             uint8_t *rows[6] = {qk + u * 128, qk + 16384 + u * 128, qk + 8192 + u * 128,
                                 qk + 24576 + u * 128, vv + u * 128, vv + 8192 + u * 128};
+            // A whole 128-byte row is rewritten, so the swizzle does not matter; the rotated
+            // order keeps the eight threads of a row group on distinct banks. Three rows of
+            // loads are issued before their first store.
 #pragma unroll
-            for (int which = 0; which < 6; ++which) {
-                const float f = (which == 2 || which == 3) ? fq : 1.f;
-                // a whole 128-byte row is rewritten, so the swizzle does not matter; the
-                // rotated order keeps the eight threads of a row group on distinct banks.
-                // All eight loads are issued before the first store.
-                uint4 v[8];
+            for (int grp = 0; grp < 6; grp += 3) {
+                uint4 v[3][8];
 #pragma unroll
-                for (int it = 0; it < 8; ++it) v[it] = lds128(rows[which] + (((it + u) & 7) << 4));
+                for (int w3 = 0; w3 < 3; ++w3)
 #pragma unroll
-                for (int it = 0; it < 8; ++it)
-                    sts128(rows[which] + (((it + u) & 7) << 4), bf16x8_to_f16x8(v[it], f));
+                    for (int it = 0; it < 8; ++it) v[w3][it] = lds128(rows[grp + w3] + (((it + u) & 7) << 4));
+#pragma unroll
+                for (int w3 = 0; w3 < 3; ++w3) {
+                    const int which = grp + w3;
+                    const float f = (which == 2 || which == 3) ? fq : 1.f;
+#pragma unroll
+                    for (int it = 0; it < 8; ++it)
+                        sts128(rows[which] + (((it + u) & 7) << 4), bf16x8_to_f16x8(v[w3][it], f));
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar[B_CONV]);
@@ -400,19 +430,23 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int t = r & 63;
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u << 16;
         float *g2s = reinterpret_cast<float *>(smem + OFF_GATES);
-        float *gam = g2s + 64, *bet = g2s + 128;
+        float *gam = g2s + 64, *bet = g2s + 128, *bfac = g2s + 192;
         for (int c = 0; c < n_chunks; ++c) {
             const int64_t tok0 = ci.bos + (int64_t)c * kC;
             const int n_valid = chunk_valid(c);
             if (warp == 4) {
                 float g_lo, g_hi;
                 chunk_log2_decay_scan(log_alpha, tok0, H, ci.h, n_valid, lane, g_lo, g_hi);
+                // Gamma_ts = 2^(g_t - g_s) = 2^(g_t - m) 2^(m - g_s) around the mid decay m
+                const float mid = 0.5f * (__shfl_sync(0xffffffffu, g_lo, 0) + __shfl_sync(0xffffffffu, g_hi, 31));
                 g2s[lane] = g_lo;
                 g2s[lane + 32] = g_hi;
                 gam[lane] = fast_exp2(g_lo);
                 gam[lane + 32] = fast_exp2(g_hi);
                 bet[lane] = lane < n_valid ? beta[(size_t)(tok0 + lane) * H + ci.h] : 0.f;
                 bet[lane + 32] = lane + 32 < n_valid ? beta[(size_t)(tok0 + lane + 32) * H + ci.h] : 0.f;
+                bfac[lane] = fast_exp2(mid - g_lo);
+                bfac[lane + 32] = fast_exp2(mid - g_hi);
             }
             // (a) G rows: K K^T (lanes 0..63), Q K^T (lanes 64..127)
             bool ok = true;
@@ -426,40 +460,52 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_before();
             mbar_arrive(&bar[B_GEMPTY]);
             const float g2t = g2s[t];
+            // one uniform choice per chunk: factored Gamma (both factors in the fp32 normal
+            // range when the chunk's decay span is at most kSpanMax) or one exp2 per entry
+            const float g2first = g2s[0], g2last = g2s[63];
+            const bool factored = (g2first - g2last) <= kSpanMax;
+            const float at = fast_exp2(g2t - 0.5f * (g2first + g2last));
             uint32_t pk[32];                  // P row (threads 64..127), fp16 pairs
-            if (r < 64) {
-                const float bt = bet[t];
+            // the row's weight for column s: w_s = c * Gamma_ts, c = beta_t (L) or scale (P)
+            const float cw = r < 64 ? bet[t] : scale;
+            float wrow[64];
+            if (factored) {
+                const float cat = cw * at;
 #pragma unroll
                 for (int s4 = 0; s4 < 64; s4 += 4) {
-                    const float4 g4 = ldsf4(g2s + s4);
-                    const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = s4 + e;
-                        uint32_t &gr = s < 32 ? ga[s] : gb[s - 32];
-                        gr = __float_as_uint((s < t) ? bt * __uint_as_float(gr) * fast_exp2(g2t - gg[e]) : 0.f);
-                    }
-                }
-#pragma unroll
-                for (int s4 = 0; s4 < 64; s4 += 4) {
-                    const uint32_t *src = s4 < 32 ? ga + s4 : gb + (s4 - 32);
-                    stsf4(Ls + t * LS_LD + s4, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
-                                                           __uint_as_float(src[2]), __uint_as_float(src[3])));
+                    const float4 b4 = ldsf4(bfac + s4);
+                    wrow[s4] = cat * b4.x;
+                    wrow[s4 + 1] = cat * b4.y;
+                    wrow[s4 + 2] = cat * b4.z;
+                    wrow[s4 + 3] = cat * b4.w;
                 }
             } else {
 #pragma unroll
                 for (int s4 = 0; s4 < 64; s4 += 4) {
                     const float4 g4 = ldsf4(g2s + s4);
-                    const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
-                    float pv[4];
+                    wrow[s4] = cw * fast_exp2(fminf(g2t - g4.x, 0.f));
+                    wrow[s4 + 1] = cw * fast_exp2(fminf(g2t - g4.y, 0.f));
+                    wrow[s4 + 2] = cw * fast_exp2(fminf(g2t - g4.z, 0.f));
+                    wrow[s4 + 3] = cw * fast_exp2(fminf(g2t - g4.w, 0.f));
+                }
+            }
+            if (r < 64) {
+#pragma unroll
+                for (int s4 = 0; s4 < 64; s4 += 4) {
+                    float lv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int s = s4 + e;
-                        const float gv = __uint_as_float(s < 32 ? ga[s] : gb[s - 32]);
-                        pv[e] = (s <= t) ? scale * gv * fast_exp2(g2t - gg[e]) : 0.f;
+                        lv[e] = (s < t) ? wrow[s] * __uint_as_float(s < 32 ? ga[s] : gb[s - 32]) : 0.f;
                     }
-                    pk[s4 >> 1] = pack_f16x2(pv[0], pv[1]);
-                    pk[(s4 >> 1) + 1] = pack_f16x2(pv[2], pv[3]);
+                    stsf4(Ls + t * LS_LD + s4, make_float4(lv[0], lv[1], lv[2], lv[3]));
+                }
+            } else {
+#pragma unroll
+                for (int s2 = 0; s2 < 64; s2 += 2) {
+                    const float p0 = (s2 <= t) ? wrow[s2] * __uint_as_float(s2 < 32 ? ga[s2] : gb[s2 - 32]) : 0.f;
+                    const float p1 = (s2 + 1 <= t) ? wrow[s2 + 1] * __uint_as_float(s2 + 1 < 32 ? ga[s2 + 1] : gb[s2 - 31]) : 0.f;
+                    pk[s2 >> 1] = pack_f16x2(p0, p1);
                 }
             }
             named_bar_sync(NB_SOLVE, 128);
@@ -481,97 +527,91 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int i = 0; i < 16; ++i) Ls[(b0 + i) * LS_LD + j] = acc[i];
             }
             named_bar_sync(NB_SOLVE, 128);
-            // level 1: blocks (1,0) and (3,2): X = -T_aa (L_ab T_bb), 16x16 each
+            // Block merges on tf32 mma.sync tiles, one 8-column strip per warp, fp32 in
+            // shared memory: M = L_ab T_b (strip), then X = -T_a M (strip) -> T's block (a, b).
             {
-                const int pair = r >> 6, rr = r & 63;
-                const int a0 = 16 + 32 * pair, b0 = 32 * pair;   // (a, b) = (1, 0) or (3, 2)
-                const int i = rr >> 2, q4 = (rr & 3) * 4;
-                float m[4] = {0.f, 0.f, 0.f, 0.f};
+                const int w = warp - 4, g = lane >> 2, q = lane & 3;
+                float *rt = Rt + w * 32 * 8;                 // this warp's [32][8] strip of M
+                auto lda = [&](uint32_t (&a)[4], const float *base, int ld) {
+                    a[0] = to_tf32(base[g * ld + q]);
+                    a[1] = to_tf32(base[(g + 8) * ld + q]);
+                    a[2] = to_tf32(base[g * ld + q + 4]);
+                    a[3] = to_tf32(base[(g + 8) * ld + q + 4]);
+                };
+                auto ldb = [&](uint32_t (&b)[2], const float *base, int ld) {
+                    b[0] = to_tf32(base[q * ld + g]);
+                    b[1] = to_tf32(base[(q + 4) * ld + g]);
+                };
+                auto std_ = [&](float *base, int ld, const float (&d)[4], float sgn) {
+                    base[g * ld + 2 * q] = sgn * d[0];
+                    base[g * ld + 2 * q + 1] = sgn * d[1];
+                    base[(g + 8) * ld + 2 * q] = sgn * d[2];
+                    base[(g + 8) * ld + 2 * q + 1] = sgn * d[3];
+                };
+                // level 1: blocks (1,0) and (3,2), 16x16 each; warp w: pair w >> 1, strip w & 1
+                {
+                    const int pair = w >> 1, j = w & 1;
+                    const int a0 = 16 + 32 * pair, b0 = 32 * pair;
+                    float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k4 = 0; k4 < 16; k4 += 4) {
-                    const float4 l4 = ldsf4(Ls + (a0 + i) * LS_LD + b0 + k4);
-                    const float lk[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float4 tr = ldsf4(Ls + (b0 + k4 + e) * LS_LD + b0 + q4);
-                        m[0] = fmaf(lk[e], tr.x, m[0]);
-                        m[1] = fmaf(lk[e], tr.y, m[1]);
-                        m[2] = fmaf(lk[e], tr.z, m[2]);
-                        m[3] = fmaf(lk[e], tr.w, m[3]);
+                    for (int kk = 0; kk < 16; kk += 8) {
+                        uint32_t a[4], b[2];
+                        lda(a, Ls + a0 * LS_LD + b0 + kk, LS_LD);
+                        ldb(b, Ls + (b0 + kk) * LS_LD + b0 + 8 * j, LS_LD);
+                        mma_tf32_16x8x8(m, a, b);
                     }
+                    std_(rt, 8, m, 1.f);
+                    __syncwarp();
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int kk = 0; kk < 16; kk += 8) {
+                        uint32_t a[4], b[2];
+                        lda(a, Ls + a0 * LS_LD + a0 + kk, LS_LD);
+                        ldb(b, rt + kk * 8, 8);
+                        mma_tf32_16x8x8(x, a, b);
+                    }
+                    // the sibling strip's warp may still read L_ab: store X after everyone
+                    named_bar_sync(NB_SOLVE, 128);
+                    std_(Ls + a0 * LS_LD + b0 + 8 * j, LS_LD, x, -1.f);
                 }
-                stsf4(Rt + pair * 16 * 16 + i * 16 + q4, make_float4(m[0], m[1], m[2], m[3]));
                 named_bar_sync(NB_SOLVE, 128);
-                float x[4] = {0.f, 0.f, 0.f, 0.f};
+                // level 2: rows 32..63 x cols 0..31; warp w owns strip w (cols 8w..8w+7)
+                {
+                    const int k_lo = w >= 2 ? 16 : 0;        // T_A is zero in rows 0..15 of cols 16..31
+                    __syncwarp();
+                    float m[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-                for (int k4 = 0; k4 < 16; k4 += 4) {
-                    const float4 t4 = ldsf4(Ls + (a0 + i) * LS_LD + a0 + k4);
-                    const float tk[4] = {t4.x, t4.y, t4.z, t4.w};
+                    for (int kk = 0; kk < 32; kk += 8) {
+                        if (kk < k_lo) continue;
+                        uint32_t b[2];
+                        ldb(b, Ls + kk * LS_LD + 8 * w, LS_LD);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float4 mr = ldsf4(Rt + pair * 16 * 16 + (k4 + e) * 16 + q4);
-                        x[0] = fmaf(-tk[e], mr.x, x[0]);
-                        x[1] = fmaf(-tk[e], mr.y, x[1]);
-                        x[2] = fmaf(-tk[e], mr.z, x[2]);
-                        x[3] = fmaf(-tk[e], mr.w, x[3]);
+                        for (int mt = 0; mt < 2; ++mt) {
+                            uint32_t a[4];
+                            lda(a, Ls + (32 + 16 * mt) * LS_LD + kk, LS_LD);
+                            mma_tf32_16x8x8(m[mt], a, b);
+                        }
                     }
-                }
-                stsf4(Ls + (a0 + i) * LS_LD + b0 + q4, make_float4(x[0], x[1], x[2], x[3]));
-            }
-            named_bar_sync(NB_SOLVE, 128);
-            // level 2: rows 32..63 x cols 0..31: X = -T_B (L_BA T_A), 32x32 each.
-            // Warp w owns 8 columns (8w..8w+7), lane = row.
-            {
-                const int w = warp - 4, i = lane, c0 = 8 * w;
-                const int k_lo = w >= 2 ? 16 : 0;        // T_A is zero in rows 0..15 of cols 16..31
-                float m[8];
+                    std_(rt, 8, m[0], 1.f);
+                    std_(rt + 16 * 8, 8, m[1], 1.f);
+                    __syncwarp();
+                    float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) m[e] = 0.f;
+                    for (int kk = 0; kk < 32; kk += 8) {
+                        uint32_t b[2];
+                        ldb(b, rt + kk * 8, 8);
 #pragma unroll
-                for (int k4 = 0; k4 < 32; k4 += 4) {
-                    if (k4 < k_lo) continue;
-                    const float4 l4 = ldsf4(Ls + (32 + i) * LS_LD + k4);
-                    const float lk[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float4 ta = ldsf4(Ls + (k4 + e) * LS_LD + c0);
-                        const float4 tb = ldsf4(Ls + (k4 + e) * LS_LD + c0 + 4);
-                        m[0] = fmaf(lk[e], ta.x, m[0]);
-                        m[1] = fmaf(lk[e], ta.y, m[1]);
-                        m[2] = fmaf(lk[e], ta.z, m[2]);
-                        m[3] = fmaf(lk[e], ta.w, m[3]);
-                        m[4] = fmaf(lk[e], tb.x, m[4]);
-                        m[5] = fmaf(lk[e], tb.y, m[5]);
-                        m[6] = fmaf(lk[e], tb.z, m[6]);
-                        m[7] = fmaf(lk[e], tb.w, m[7]);
+                        for (int mt = 0; mt < 2; ++mt) {
+                            if (mt == 0 && kk >= 16) continue;   // T_B is zero above its diagonal blocks
+                            uint32_t a[4];
+                            lda(a, Ls + (32 + 16 * mt) * LS_LD + 32 + kk, LS_LD);
+                            mma_tf32_16x8x8(x[mt], a, b);
+                        }
                     }
+                    named_bar_sync(NB_SOLVE, 128);      // every warp is done reading L_BA
+                    std_(Ls + 32 * LS_LD + 8 * w, LS_LD, x[0], -1.f);
+                    std_(Ls + 48 * LS_LD + 8 * w, LS_LD, x[1], -1.f);
                 }
-                stsf4(Rt + i * RT_LD + c0, make_float4(m[0], m[1], m[2], m[3]));
-                stsf4(Rt + i * RT_LD + c0 + 4, make_float4(m[4], m[5], m[6], m[7]));
-                named_bar_sync(NB_SOLVE, 128);
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = 0.f;
-#pragma unroll
-                for (int k4 = 0; k4 < 32; k4 += 4) {
-                    const float4 t4 = ldsf4(Ls + (32 + i) * LS_LD + 32 + k4);
-                    const float tk[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float4 ma = ldsf4(Rt + (k4 + e) * RT_LD + c0);
-                        const float4 mb = ldsf4(Rt + (k4 + e) * RT_LD + c0 + 4);
-                        x[0] = fmaf(-tk[e], ma.x, x[0]);
-                        x[1] = fmaf(-tk[e], ma.y, x[1]);
-                        x[2] = fmaf(-tk[e], ma.z, x[2]);
-                        x[3] = fmaf(-tk[e], ma.w, x[3]);
-                        x[4] = fmaf(-tk[e], mb.x, x[4]);
-                        x[5] = fmaf(-tk[e], mb.y, x[5]);
-                        x[6] = fmaf(-tk[e], mb.z, x[6]);
-                        x[7] = fmaf(-tk[e], mb.w, x[7]);
-                    }
-                }
-                stsf4(Ls + (32 + i) * LS_LD + c0, make_float4(x[0], x[1], x[2], x[3]));
-                stsf4(Ls + (32 + i) * LS_LD + c0 + 4, make_float4(x[4], x[5], x[6], x[7]));
             }
             named_bar_sync(NB_SOLVE, 128);
             // (c) T diag(beta gamma), rows by threads 0..63. The row is computed into registers
@@ -627,10 +667,10 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[B_WB]);
-            // (e) P into the V stage of this chunk, free once U^T(c) is done (x_full(c));
+            // (e) P into the V stage of this chunk, free once U^T(c) is done (u_full(c));
             // S(c) reads it, and the stage is reloaded only after S(c) completes
             ok = true;
-            if (r == 0) ok = mbar_wait_bounded(&bar[B_XFULL], c & 1, abort_flag, kWaitLimit);
+            if (r == 0) ok = mbar_wait_bounded(&bar[B_UFULL], c & 1, abort_flag, kWaitLimit);
             if (!named_bar_and(NB_SOLVE, 128, ok)) break;
             if (r >= 64) {
                 uint8_t *pdst = smem + OFF_V + (c & 1) * V_STAGE;

@@ -269,6 +269,28 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128-byte-swizzled tile.
 __device__ __forceinline__ uint32_t sw128_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
+// ---------------------------------------------------------------- warp-level MMA
+// D = A x B + D for one 16x8x8 tile, tf32 inputs, fp32 accumulate (mma.sync). Used for
+// the small block products of the triangular solve, where the M >= 64 of tcgen05 does
+// not fit. Fragment ownership (g = lane / 4, q = lane % 4):
+//   A 16x8 row-major: a0 (g, q), a1 (g+8, q), a2 (g, q+4), a3 (g+8, q+4)
+//   B 8x8 (k x n):    b0 (q, g), b1 (q+4, g)
+//   D 16x8:           d0 (g, 2q), d1 (g, 2q+1), d2 (g+8, 2q), d3 (g+8, 2q+1)
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+{
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
 // 2^x with the SM's approximate base-2 exponential instruction (denormal results flush
 // to zero). Every argument here is <= 0, so results lie in [0, 1].
 __device__ __forceinline__ float fast_exp2(float x)
