@@ -104,6 +104,23 @@ def _check(fn: str, code: int):
         raise GdnError(fn, code)
 
 
+_workspaces = {}
+
+
+def _workspace(device, nbytes):
+    """Device scratch for gdn_chunk_fwd, kept per device and grown on demand. One buffer
+    serves every call on a device: the library indexes it by SM id, so calls on
+    different streams do not collide."""
+    if nbytes == 0:
+        return None
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(idx)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[idx] = ws
+    return ws
+
+
 def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0,
               cu_seqlens_host=None, out=None, final_state=True, y_dtype=torch.float32):
     """Chunked prefill over packed sequences. Returns (y, S_T or None).
@@ -136,7 +153,7 @@ def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0
            if final_state else None)
     L = lib()
     ws_bytes = L.gdn_chunk_fwd_workspace_bytes(n_seq, N, H, dk, dv, chunk)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device) if ws_bytes else None
+    ws = _workspace(q.device, ws_bytes)
     rc = L.gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), code, _ptr(log_alpha), _ptr(beta), _ptr(S0),
                          _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), n_seq, H, dk, dv,
                          int(chunk), float(scale), _ptr(y), _dtype_code(y), _ptr(S_T), _ptr(ws),

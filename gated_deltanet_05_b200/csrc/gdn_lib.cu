@@ -59,6 +59,23 @@ bool make_map(CUtensorMap *map, const void *base, int64_t n_tok, int H)
     return r == CUDA_SUCCESS;
 }
 
+// 3-D map over the [n_tok][H][128] output y (fp32 or bf16), box {128, 1, 32}: one
+// warpgroup's 32 token rows of one head, no swizzle (the staging tile is row-major).
+bool make_y_map(CUtensorMap *map, void *base, int64_t n_tok, int H, bool f32)
+{
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t es = f32 ? 4 : 2;
+    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)n_tok};
+    cuuint64_t strides[2] = {128 * es, (cuuint64_t)H * 128 * es};
+    cuuint32_t box[3] = {128, 1, 32};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int g_smem_optin = -1;
 
 int smem_optin()
@@ -91,23 +108,40 @@ gdn_status launch_chunk_f32(const void *q, const void *k, const void *v, const f
     return launch_status();
 }
 
+// Number of SM ids of the current device (the tensor-core kernel's workspace has one
+// region per SM id); 0 if the device cannot be queried.
+int device_sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
 template <typename TY>
 gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const float *la,
                               const float *beta, const float *S0, const int32_t *cu, int n_seq,
-                              int64_t n_tok, int H, float scale, void *y, float *S_T,
-                              cudaStream_t st)
+                              int64_t n_tok, int H, float scale, void *y, float *S_T, void *ws,
+                              size_t ws_bytes, cudaStream_t st)
 {
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, n_tok, H) || !make_map(&mk, k, n_tok, H) || !make_map(&mv, v, n_tok, H))
+    const int n_sm = device_sm_count();
+    if (n_sm <= 0) return GDN_ERR_CUDA;
+    if (!ws || !aligned(ws, 128) || ws_bytes < (size_t)n_sm * gdn::sm100::kWsBytesPerSm)
+        return GDN_ERR_INVALID_ARG;
+    CUtensorMap mq, mk, mv, my;
+    if (!make_map(&mq, q, n_tok, H) || !make_map(&mk, k, n_tok, H) || !make_map(&mv, v, n_tok, H) ||
+        !make_y_map(&my, y, n_tok, H, sizeof(TY) == 4))
         return GDN_ERR_CUDA;
     const int smem = (int)gdn::sm100::SMEM_BYTES;
     if (smem > smem_optin()) return GDN_ERR_UNSUPPORTED;
     auto kern = gdn::sm100::chunk_fwd_bf16_kernel<TY>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return GDN_ERR_CUDA;
-    const unsigned grid = (unsigned)((int64_t)n_seq * H);
-    kern<<<grid, gdn::sm100::kThreads, smem, st>>>(mq, mk, mv, la, beta, S0, cu, n_seq, H, scale,
-                                                   static_cast<TY *>(y), S_T);
+    // one cluster of two CTAs (solver, chain) per (sequence, head) chain
+    const unsigned grid = (unsigned)(2 * (int64_t)n_seq * H);
+    kern<<<grid, gdn::sm100::kThreads, smem, st>>>(mq, mk, mv, my, la, beta, S0, cu, n_seq, H, scale,
+                                                   static_cast<TY *>(y), S_T,
+                                                   static_cast<uint8_t *>(ws), n_sm);
     return launch_status();
 }
 
@@ -133,8 +167,9 @@ int gdn_version(void) { return 100; }
 size_t gdn_chunk_fwd_workspace_bytes(int n_seq, int64_t total_tokens, int H, int d_k, int d_v,
                                      int chunk)
 {
-    (void)n_seq; (void)total_tokens; (void)H; (void)d_k; (void)d_v; (void)chunk;
-    return 0;
+    (void)n_seq; (void)total_tokens; (void)H;
+    if (d_k != 128 || d_v != 128 || chunk != 64) return 0;
+    return (size_t)device_sm_count() * gdn::sm100::kWsBytesPerSm;
 }
 
 gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
@@ -144,7 +179,6 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype 
                          gdn_dtype y_dtype, float *S_T, void *workspace, size_t workspace_bytes,
                          void *stream)
 {
-    (void)workspace; (void)workspace_bytes;
     if (n_seq < 0 || H <= 0 || !cu_seqlens_host || (n_seq > 0 && !cu_seqlens_dev))
         return GDN_ERR_INVALID_ARG;
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
@@ -164,11 +198,12 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype 
     if ((int64_t)n_seq * H * (d_v / (d_v < 32 ? d_v : 32)) > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     cudaStream_t st = as_stream(stream);
     const bool y32 = y_dtype == GDN_F32;
-    if (in_dtype == GDN_BF16 && d_k == 128 && d_v == 128 && chunk == 64)
+    if (in_dtype == GDN_BF16 && d_k == 128 && d_v == 128 && chunk == 64 && n_tok > 0)
         return y32 ? launch_chunk_sm100<float>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev, n_seq,
-                                               n_tok, H, scale, y, S_T, st)
+                                               n_tok, H, scale, y, S_T, workspace, workspace_bytes, st)
                    : launch_chunk_sm100<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev,
-                                                       n_seq, n_tok, H, scale, y, S_T, st);
+                                                       n_seq, n_tok, H, scale, y, S_T, workspace,
+                                                       workspace_bytes, st);
 #define GDN_F32_PATH(T, TY)                                                                        \
     launch_chunk_f32<T, TY>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev, n_seq, H, d_k, d_v, chunk, \
                             scale, y, S_T, st)

@@ -67,10 +67,12 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// The bounded waits below are out of line: they are called from many sites and kept
+// out of the instruction cache's way.
 // Waits for the phase of `bar` with the given parity to complete. Gives up (returns
 // false) after ~limit_cycles SM clocks or as soon as *abort becomes non-zero; on a
 // timeout it records kErrTimeout in the device error word and sets *abort.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+__device__ __noinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort, long long limit_cycles)
 {
     if (mbar_try_wait(bar, parity))
@@ -91,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 
 // Waits for a phase to complete, ignoring any abort request (used to drain async work
 // before the CTA exits). Returns false after ~limit_cycles.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, long long limit_cycles)
+__device__ __noinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, long long limit_cycles)
 {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity))
@@ -149,6 +151,17 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *desc, ui
         : "memory");
 }
 
+// 3-D tiled store of one box from shared memory, tracked by this thread's bulk
+// async-group. Coordinates are element indices, innermost first, all >= 0; rows of the
+// box beyond the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_3d(const void *desc, const void *smem_src, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(desc)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 // Bulk (non-tensor) copy shared -> global, tracked by this thread's bulk async-group.
 // Both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_store_s2g(void *gdst, const void *ssrc, uint32_t bytes)
@@ -162,6 +175,149 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // All of this thread's bulk copies have completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// ---------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Shared-memory address of the same offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_peer(uint32_t local_smem_addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem_addr), "r"(rank));
+    return r;
+}
+
+// Arrive (release at cluster scope) on an mbarrier of another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+// Relaxed variant: for signals that publish no memory writes of the arriving thread (so
+// it does not wait for the thread's outstanding stores).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote_relaxed(uint32_t remote_bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(remote_bar),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t remote_bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(remote_bar),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Waits, with cluster-scope acquire, for a phase of a local mbarrier that another CTA of
+// the cluster signals. Bounded like mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __noinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                          long long limit_cycles)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (*abort) return false;
+        if (clock64() - t0 > limit_cycles) {
+            *abort = 1;
+            raise_error(kErrTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Bulk copy from this CTA's shared memory into another CTA's shared memory of the
+// cluster; completion is counted as transaction bytes on the destination's mbarrier.
+// No multicast. Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_copy_s2peer(uint32_t remote_dst, const void *local_src, uint32_t bytes,
+                                                 uint32_t remote_bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+                     "r"(remote_dst),
+                 "r"(smem_u32(local_src)), "r"(bytes), "r"(remote_bar)
+                 : "memory");
+}
+// 32-bit load from another CTA's shared memory (address from map_to_peer).
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t remote_addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote_addr) : "memory");
+    return v;
+}
+
+// Bulk copy global -> this CTA's shared memory, completing as transaction bytes on `bar`.
+// Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load_g2s(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(sdst)),
+                 "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Bulk copies of this thread: at most one group not yet complete.
+__device__ __forceinline__ void bulk_wait_all_but_1() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
+// Orders this thread's generic-proxy view of global memory with async-proxy (bulk/TMA)
+// accesses.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t smid()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t p;
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.b32 %0, 1, 0, e;\n\t}" : "=r"(p));
+    return p != 0;
+}
+
+// 32-bit store into another CTA's shared memory (address from map_to_peer).
+__device__ __forceinline__ void st_cluster_u32(uint32_t remote_addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote_addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 // ---------------------------------------------------------------- tcgen05 / TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t *smem_slot, uint32_t n_cols)
@@ -191,6 +347,112 @@ __device__ __forceinline__ void mma_f16kind_ss(uint32_t d_tmem, uint64_t a_desc,
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] x B[smem desc], kind::f16. A is M x K with row m in TMEM lane m and
+// two 16-bit K elements per 32-bit column (lower K index in the low half); a K step of 16
+// advances the A address by 8 columns. A is K-major by construction (descriptor bit 15 = 0).
+__device__ __forceinline__ void mma_f16kind_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Leader-predicated forms: executed by a whole converged warp with warp-uniform operands
+// (so they stay in uniform registers); only the lane with `leader` != 0 issues. Keeping the
+// warp converged avoids per-lane operand loops around these instructions.
+__device__ __forceinline__ void mma_ss_lead(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, l;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 l, %5, 0;\n\t"
+        "@l tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_lead(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, l;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 l, %5, 0;\n\t"
+        "@l tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_lead(uint64_t *bar, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %1, 0;\n\t"
+        "@l tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
+        "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_lead(void *smem_dst, const void *desc, uint64_t *bar, int c0, int c1,
+                                                 int c2, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %6, 0;\n\t"
+        "@l cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_lead(uint64_t *bar, uint32_t bytes, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %2, 0;\n\t"
+        "@l mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+        "r"(bytes), "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_load_g2s_lead(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar,
+                                                   uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %4, 0;\n\t"
+        "@l cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(
+            smem_u32(sdst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_lead(uint64_t *bar, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %1, 0;\n\t"
+        "@l mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(bar)),
+        "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote_lead(uint32_t remote_bar, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %1, 0;\n\t"
+        "@l mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n\t}" ::"r"(remote_bar),
+        "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_store_s2g_lead(void *gdst, const void *ssrc, uint32_t bytes, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %3, 0;\n\t"
+        "@l cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t}" ::"l"(gdst),
+        "r"(smem_u32(ssrc)), "r"(bytes), "r"(leader)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote_relaxed_lead(uint32_t remote_bar, uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %1, 0;\n\t"
+        "@l mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];\n\t}" ::"r"(remote_bar),
+        "r"(leader)
         : "memory");
 }
 

@@ -84,8 +84,12 @@ typedef enum {
  *   y           [N_tok, H, d_v]  out, in y_dtype (GDN_F32 or GDN_BF16, independent of
  *               in_dtype; a bf16 y is the round-to-nearest-even of the fp32 result)
  *   S_T         [n_seq, H, d_v, d_k] fp32 out (final state per sequence), or NULL
- *   workspace   device scratch of workspace_bytes >= gdn_chunk_fwd_workspace_bytes(..)
- *               (may be NULL when that is 0)
+ *   workspace   device scratch of workspace_bytes >= gdn_chunk_fwd_workspace_bytes(..),
+ *               128-byte aligned (may be NULL when that is 0). The tensor-core path uses
+ *               it as a ring of fp16 K tiles per SM id (SM count x 64 KB on the current
+ *               device); no initial contents are needed and nothing is left in
+ *               it. Calls on different streams may share one workspace (each SM id's
+ *               region is used by at most one cluster at a time). Caller-owned.
  *
  * Paths: bf16 inputs with d_k = d_v = 128 and chunk = 64 run the sm_100a tensor-core
  * kernel (tcgen05 MMA with TMEM accumulators, TMA loads, fp32 state carry; bf16 inputs
@@ -93,6 +97,9 @@ typedef enum {
  * convert exactly -- which requires |q|, |k|, |v| and the state entries below 65504);
  * every other supported case runs the CUDA-core fp32 chunk kernel.
  */
+/* Scratch bytes gdn_chunk_fwd needs for these sizes on the current device: SM count x
+ * 64 KB when d_k = d_v = 128 and chunk = 64 (the tensor-core path; sized for any input
+ * dtype), else 0. Returns 0 when no device can be queried. */
 size_t gdn_chunk_fwd_workspace_bytes(int n_seq, int64_t total_tokens, int H, int d_k, int d_v,
                                      int chunk);
 

@@ -44,7 +44,11 @@ def test_status_strings_and_version(L):
         assert L.gdn_status_string(code).decode() == name
     assert L.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
     assert L.gdn_version() == 100
-    assert L.gdn_chunk_fwd_workspace_bytes(4, 16384, 16, 128, 128, 64) == 0
+    # only the tensor-core path (d_k = d_v = 128, chunk 64) uses scratch: one K ring
+    # per SM id (none without a device)
+    assert L.gdn_chunk_fwd_workspace_bytes(4, 16384, 16, 64, 64, 64) == 0
+    assert L.gdn_chunk_fwd_workspace_bytes(4, 16384, 16, 128, 128, 32) == 0
+    assert L.gdn_chunk_fwd_workspace_bytes(4, 16384, 16, 128, 128, 64) % (4 * 16384) == 0
 
 
 def _cu(vals):
@@ -82,6 +86,7 @@ def test_chunk_fwd_rejects_bad_arguments(L):
     assert _chunk(L, y=ctypes.c_void_p(0x10008)) == 1       # misaligned output
     assert _chunk(L, la=ctypes.c_void_p(0x10002)) == 1      # misaligned gate
     assert _chunk(L, n_seq=0, cuh=_cu([0])) == 0            # nothing to do
+    assert _chunk(L) != 0                                   # tensor-core path without its workspace
 
 
 def test_decode_and_gate_norm_reject_bad_arguments(L):
