@@ -18,7 +18,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "decode_step", "gate_norm", "device_error", "lib", "LIB_PATH",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "decode_step", "gate_norm", "device_error", "lib", "LIB_PATH",
            "GdnError", "EXPORTED_SYMBOLS", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn_b200.so")
@@ -27,7 +27,8 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
           4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_DEVICE_CHECK"}
 GDN_F32, GDN_BF16 = 0, 1
 
-EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_decode_step",
+EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc",
+                    "gdn_decode_step",
                     "gdn_gate_norm", "gdn_status_string", "gdn_device_error", "gdn_version")
 
 
@@ -59,6 +60,9 @@ def lib():
         L.gdn_chunk_fwd.restype = i32
         L.gdn_chunk_fwd.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                     f32, vp, i32, vp, vp, ctypes.c_size_t, vp]
+        L.gdn_chunk_fwd_noalloc.restype = i32
+        L.gdn_chunk_fwd_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                            i32, f32, vp, i32, vp, vp]
         L.gdn_decode_step.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, vp, vp]
         L.gdn_gate_norm.restype = i32
@@ -121,20 +125,12 @@ def _workspace(device, nbytes):
     return ws
 
 
-def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0,
-              cu_seqlens_host=None, out=None, final_state=True, y_dtype=torch.float32):
-    """Chunked prefill over packed sequences. Returns (y, S_T or None).
-
-    q, k [N, H, d_k] and v [N, H, d_v] (fp32 or bf16, same dtype); log_alpha, beta [N, H]
-    fp32; cu_seqlens [n_seq + 1] int32 (device); S0 [n_seq, H, d_v, d_k] fp32 or None.
-    y is returned in y_dtype (float32 by default; bfloat16 gives the round-to-nearest-even
-    of the same fp32 result).
-    """
+def _chunk_setup(q, k, v, log_alpha, beta, cu_seqlens, S0, cu_seqlens_host, out, final_state,
+                 state_out, y_dtype):
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (log_alpha, "log_alpha"), (beta, "beta"),
                  (cu_seqlens, "cu_seqlens")):
         _cuda(t, n)
     _cuda(S0, "S0")
-    code = _dtype_code(q)
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share one dtype")
     if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
@@ -149,16 +145,49 @@ def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0
     cu_h = cu_seqlens_host.to(torch.int32).contiguous()
     y = out if out is not None else torch.empty((N, H, dv), dtype=y_dtype, device=q.device)
     _cuda(y, "out")
-    S_T = (torch.empty((n_seq, H, dv, dk), dtype=torch.float32, device=q.device)
-           if final_state else None)
+    S_T = None
+    if final_state:
+        S_T = (state_out if state_out is not None
+               else torch.empty((n_seq, H, dv, dk), dtype=torch.float32, device=q.device))
+        _cuda(S_T, "state_out")
+    args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+            _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), n_seq, H, dk, dv)
+    return args, y, S_T, cu_h
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0,
+              cu_seqlens_host=None, out=None, final_state=True, y_dtype=torch.float32,
+              state_out=None):
+    """Chunked prefill over packed sequences. Returns (y, S_T or None).
+
+    q, k [N, H, d_k] and v [N, H, d_v] (fp32 or bf16, same dtype); log_alpha, beta [N, H]
+    fp32; cu_seqlens [n_seq + 1] int32 (device); S0 [n_seq, H, d_v, d_k] fp32 or None.
+    y is returned in y_dtype (float32 by default; bfloat16 gives the round-to-nearest-even
+    of the same fp32 result). out / state_out may supply the output tensors.
+    """
+    args, y, S_T, cu_h = _chunk_setup(q, k, v, log_alpha, beta, cu_seqlens, S0, cu_seqlens_host,
+                                      out, final_state, state_out, y_dtype)
     L = lib()
-    ws_bytes = L.gdn_chunk_fwd_workspace_bytes(n_seq, N, H, dk, dv, chunk)
+    n_seq, H, dk, dv = args[9], args[10], args[11], args[12]
+    ws_bytes = L.gdn_chunk_fwd_workspace_bytes(n_seq, q.shape[0], H, dk, dv, chunk)
     ws = _workspace(q.device, ws_bytes)
-    rc = L.gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), code, _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                         _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), n_seq, H, dk, dv,
-                         int(chunk), float(scale), _ptr(y), _dtype_code(y), _ptr(S_T), _ptr(ws),
-                         ws_bytes, _stream(q.device))
+    rc = L.gdn_chunk_fwd(*args, int(chunk), float(scale), _ptr(y), _dtype_code(y), _ptr(S_T),
+                         _ptr(ws), ws_bytes, _stream(q.device))
     _check("gdn_chunk_fwd", rc)
+    return y, S_T
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0,
+                      cu_seqlens_host=None, out=None, final_state=True, y_dtype=torch.float32,
+                      state_out=None):
+    """chunk_fwd through gdn_chunk_fwd_noalloc: the library call allocates nothing (its
+    scratch is a fixed device array of the library). Pass out / state_out (and a host
+    cu_seqlens) for a call that allocates nothing on this side either."""
+    args, y, S_T, cu_h = _chunk_setup(q, k, v, log_alpha, beta, cu_seqlens, S0, cu_seqlens_host,
+                                      out, final_state, state_out, y_dtype)
+    rc = lib().gdn_chunk_fwd_noalloc(*args, int(chunk), float(scale), _ptr(y), _dtype_code(y),
+                                     _ptr(S_T), _stream(q.device))
+    _check("gdn_chunk_fwd_noalloc", rc)
     return y, S_T
 
 

@@ -118,6 +118,12 @@ int device_sm_count()
     return n;
 }
 
+// Fixed scratch of gdn_chunk_fwd_noalloc: the tensor-core kernel's K ring for up to
+// kNoAllocMaxSms SM ids, as a file-scope device array (one copy per device, created with
+// the module; never allocated by a call).
+constexpr int kNoAllocMaxSms = 160;
+static __device__ __align__(256) uint8_t g_noalloc_ws[(size_t)kNoAllocMaxSms * gdn::sm100::kWsBytesPerSm];
+
 template <typename TY>
 gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const float *la,
                               const float *beta, const float *S0, const int32_t *cu, int n_seq,
@@ -211,6 +217,26 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype 
         return y32 ? GDN_F32_PATH(__nv_bfloat16, float) : GDN_F32_PATH(__nv_bfloat16, __nv_bfloat16);
     return y32 ? GDN_F32_PATH(float, float) : GDN_F32_PATH(float, __nv_bfloat16);
 #undef GDN_F32_PATH
+}
+
+gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                 int n_seq, int H, int d_k, int d_v, int chunk, float scale, void *y,
+                                 gdn_dtype y_dtype, float *S_T, void *stream)
+{
+    // the fixed array covers kNoAllocMaxSms SM ids of the current device
+    size_t need = 0;
+    if (d_k == 128 && d_v == 128 && chunk == 64) {
+        const int n_sm = device_sm_count();
+        if (n_sm <= 0) return GDN_ERR_CUDA;
+        if (n_sm > kNoAllocMaxSms) return GDN_ERR_UNSUPPORTED;
+        need = (size_t)n_sm * gdn::sm100::kWsBytesPerSm;
+    }
+    void *ws = nullptr;
+    if (need > 0 && cudaGetSymbolAddress(&ws, g_noalloc_ws) != cudaSuccess) return GDN_ERR_CUDA;
+    return gdn_chunk_fwd(q, k, v, in_dtype, log_alpha, beta, S0, cu_seqlens_dev, cu_seqlens_host, n_seq, H,
+                         d_k, d_v, chunk, scale, y, y_dtype, S_T, ws, need, stream);
 }
 
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype in_dtype,

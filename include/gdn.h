@@ -111,6 +111,26 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype 
                          size_t workspace_bytes, void *stream);
 
 /*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd without a caller workspace, for callers that
+ * may not allocate (no counterpart in the pages: a deployment convenience, not part of
+ * the method).
+ *
+ * Same arguments, results and errors as gdn_chunk_fwd, minus workspace. The scratch of
+ * the tensor-core path is a fixed file-scope device array of the library (one per
+ * device, 160 SM ids x 64 KB = 10 MB, reached through cudaGetSymbolAddress); the call
+ * allocates and frees nothing. A device with more than 160 SMs returns
+ * GDN_ERR_UNSUPPORTED. The array is shared by every call in the process: overlapping
+ * calls on different streams do not race only because each SM id's region is used by at
+ * most one cluster at a time (one cluster's solver CTA occupies an SM), the same
+ * property that lets gdn_chunk_fwd callers share one workspace.
+ */
+gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                 int n_seq, int H, int d_k, int d_v, int chunk, float scale,
+                                 void *y, gdn_dtype y_dtype, float *S_T, void *stream);
+
+/*
  * gdn_decode_step -- one token for each of n_seq * H independent chains, in place.
  *
  * Defines: the same four-line update (joezjh.github.io notes, "Gated DeltaNet 核心机制")
