@@ -121,9 +121,11 @@ constexpr uint32_t OFF_BAR = OFF_DEC + 8 * 64 * 4;
 enum {
     B_K_FULL = 0, B_K_EMPTY = B_K_FULL + kStages, B_QV_FULL = B_K_EMPTY + kStages,
     B_QV_EMPTY = B_QV_FULL + kQVStages, B_CONV = B_QV_EMPTY + kQVStages, B_RECV = B_CONV + kQVStages,
-    B_K_READY = B_RECV + kRecv, B_WFULL = B_K_READY + kRing, B_WB, B_UD, B_SB, B_SACC, B_XFULL, B_SFULL,
-    B_DRAIN, N_BAR
+    B_K_READY = B_RECV + kRecv, B_WFULL = B_K_READY + kRing, B_XFULL, B_SFULL, B_DRAIN, N_BAR
 };
+// named barriers: 1, 2 epilogue groups, 3 converters; the epilogue (256 threads, arrive)
+// hands the two critical products to the issuer warp (32 threads, sync) through
+constexpr int NB_S_TRIG = 4, NB_X_TRIG = 5, NB_TRIG_THREADS = 288;
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BAR * 8;           // tmem base, abort, sequence, operand copies sent[2][kRecv]
 constexpr uint32_t SMEM_USED = OFF_MISC + 48;
 // TMEM columns (128 lanes): fp32 state, Y^T double buffer, W^T, U~^T, and the fp16 A
@@ -243,7 +245,6 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         } else {
             for (int b = 0; b < ch::N_BAR; ++b) {
                 uint32_t count = 1;
-                if (b == ch::B_WB || b == ch::B_UD || b == ch::B_SB || b == ch::B_SACC) count = 256;
                 if (b >= ch::B_CONV && b < ch::B_CONV + kQVStages) count = 64;
                 mbar_init(&bar[b], count);
             }
@@ -279,12 +280,16 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         return (int)(rem < kC ? rem : kC);
     };
     auto fail = [&]() { st_cluster_u32(peer_abort, 1u); };
+    // Bounded waits. A non-blocking test goes first: a blocking try_wait on a phase that
+    // has already completed still costs a few hundred cycles.
     auto wait = [&](int b, int parity) -> bool {
+        if (mbar_test(&bar[b], (uint32_t)parity & 1u)) return true;
         if (mbar_wait_bounded(&bar[b], (uint32_t)parity & 1u, abort_flag, kWaitLimit)) return true;
         fail();
         return false;
     };
     auto wait_cl = [&](int b, int parity) -> bool {
+        if (mbar_test_cluster(&bar[b], (uint32_t)parity & 1u)) return true;
         if (mbar_wait_cluster_bounded(&bar[b], (uint32_t)parity & 1u, abort_flag, kWaitLimit)) return true;
         fail();
         return false;
@@ -693,10 +698,10 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // inputs are normally there before X(c) completes, and W(c+1) runs on the tensor
             // pipe while the epilogue turns U~(c) into S(c)'s operands). The order also keeps
             // every TMEM accumulator single-writer:
-            //   W(c+1): K and solver operands of c+1 arrived; -W^T(c) read out (waited for X(c))
-            //   S(c):   U~ operands of c in TMEM, the state rescaled
-            //   U(c+1): Q and V of c+1 converted; U~(c) read out (waited for S(c))
-            //   X(c+1): -W^T(c+1) in shared memory, the state copy of c+1 in TMEM
+            //   W(c+1): K and solver operands of c+1 arrived; -W^T(c) read out (before X(c))
+            //   S(c):   U~ operands of c in TMEM, the state rescaled (S trigger)
+            //   U(c+1): Q and V of c+1 converted; U~(c) read out (before S(c))
+            //   X(c+1): -W^T(c+1) in shared memory, the state copy of c+1 in TMEM (X trigger)
             if (n_chunks > 0) {
                 const uint32_t lead = elect_one();
                 const uint32_t id_wu = idesc_f32acc(kFmtF16, 128, 64, 1, 0);
@@ -739,8 +744,16 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         mma_ss_lead(tmem + TM_U, vt + GDN_DOFF(kk * 2048), tb + GDN_DOFF(kk * 32), id_wu, kk > 0, lead);
                     return true;
                 };
+                // X(c) and S(c) start when the epilogue has stored their operands: a named
+                // barrier (the epilogue arrives without waiting) wakes this warp faster than an
+                // mbarrier wait. The epilogue always makes one last arrival on each trigger when
+                // it leaves early, so these never wait for good; an abort is checked after each.
+                auto trigger = [&](int nb_id) -> bool {
+                    named_bar_sync(nb_id, NB_TRIG_THREADS);
+                    return !__any_sync(0xffffffffu, *abort_flag != 0);
+                };
                 auto issue_X = [&](int c) -> bool {
-                    if (!wait_w(B_WB, c) || !wait_w(B_SB, c)) return false;
+                    if (!trigger(NB_X_TRIG)) return false;
                     tc_fence_after();
                     const uint64_t q0 = dq0 + GDN_DOFF((c % kQVStages) * QV_STAGE);
                     const uint32_t ty = tmem + TM_Y + (c & 1) * 64;
@@ -757,7 +770,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     return true;
                 };
                 auto issue_S = [&](int c) -> bool {
-                    if (!wait_w(B_UD, c) || !wait_w(B_SACC, c)) return false;
+                    if (!trigger(NB_S_TRIG)) return false;
                     tc_fence_after();
                     const uint64_t kb = dkt0 + GDN_DOFF((c % kStages) * K_BYTES);     // K as [s][k]: MN-major B
                     const uint64_t pp = dop0 + GDN_DOFF((c % kRecv) * TP_BYTES + 16384);
@@ -859,7 +872,6 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(&bar[B_WB]);
                 return true;
             };
             float g_lo = 0.f, g_hi = 0.f;
@@ -900,11 +912,15 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(&bar[B_SB]);
-                    mbar_arrive(&bar[B_SACC]);
                 }
             }
+            // triggers given to the issuer (each is taken n_chunks times in a complete run)
+            int n_strig = 0, n_xtrig = 0;
             bool alive = n_chunks > 0 && do_wb(0);
+            if (alive) {                          // X(0): state copy of S0 and -W^T(0) in place
+                named_bar_arrive(NB_X_TRIG, NB_TRIG_THREADS);
+                ++n_xtrig;
+            }
             for (int c = 0; alive && c < n_chunks; ++c) {
                 const int64_t tok0 = bos + (int64_t)c * kC;
                 const int n_valid = chunk_valid(c);
@@ -947,7 +963,8 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     tmem_wait_st();
                 }
                 tc_fence_before();
-                mbar_arrive(&bar[B_UD]);
+                named_bar_arrive(NB_S_TRIG, NB_TRIG_THREADS);   // S(c)
+                ++n_strig;
                 // -W^T of the next chunk while S(c) runs
                 if (!last && !do_wb(c + 1)) break;
                 // E3: the fp16 state copy of S_{c+1} and the fp32 state rescaled by the next
@@ -982,9 +999,6 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         }
                         tmem_st_x16(tmem + lane_base + TM_SB + 32 * hh, pa);
                         tmem_st_x16(tmem + lane_base + TM_SB + 32 * hh + 16, pb);
-                        tmem_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(&bar[B_SB]);
                         // S(c) has completed, so has every read of this chunk's operand slot: the
                         // solver may refill it (the signal publishes no data of this thread)
                         if (hh == 0 && r == 0)
@@ -999,7 +1013,8 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         tmem_st_x32(tmem + lane_base + TM_S + 64 * hh + 32, sb);
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(&bar[B_SACC]);
+                        named_bar_arrive(NB_X_TRIG, NB_TRIG_THREADS);   // X(c+1)
+                        ++n_xtrig;
                     }
                 }
                 // y: tokens [32 hh, 32 hh + 32) of Y^T (lane v of each warp). A full chunk goes
@@ -1032,6 +1047,10 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 g_lo = n_lo;
                 g_hi = n_hi;
             }
+            // leaving early (abort): one last arrival on each trigger the issuer may still be
+            // waiting for
+            if (n_strig < n_chunks) named_bar_arrive(NB_S_TRIG, NB_TRIG_THREADS);
+            if (n_xtrig < n_chunks) named_bar_arrive(NB_X_TRIG, NB_TRIG_THREADS);
             if (r == 0) bulk_wait_all();          // y stores complete before the CTA exits
         }
     }

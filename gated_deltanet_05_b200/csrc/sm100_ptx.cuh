@@ -117,6 +117,13 @@ __device__ __forceinline__ void named_bar_sync(int id, int n_threads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n_threads) : "memory");
 }
 
+// Arrive on a named barrier without waiting (the waiting side uses named_bar_sync with
+// the same thread count).
+__device__ __forceinline__ void named_bar_arrive(int id, int n_threads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n_threads) : "memory");
+}
+
 // Named barrier that also ANDs a predicate over the participating threads: every
 // thread gets the same answer, so a group can take a uniform decision.
 __device__ __forceinline__ bool named_bar_and(int id, int n_threads, bool pred)
