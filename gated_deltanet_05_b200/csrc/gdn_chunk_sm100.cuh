@@ -938,10 +938,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     if (c + 2 < n_chunks) load_la(c + 2);
                 }
                 const float gC_next = last ? 1.f : fast_exp2(__shfl_sync(0xffffffffu, n_hi, 31));
-                // E2: U~^T -> fp16 A operands in TMEM (plain and decayed), 32 columns s per half.
-                // (The barrier also tells the group that the previous y store has read its
-                // staging tile.)
-                if (r == 0) bulk_wait_read();
+                // E2: U~^T -> fp16 A operands in TMEM (plain and decayed), 32 columns s per half
                 if (!group_wait(B_XFULL, c)) break;
                 tc_fence_after();
                 {
@@ -1026,6 +1023,10 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     tmem_ld_x32(tmem + lane_base + TM_Y + (c & 1) * 64 + 32 * hh, ya);
                     tmem_wait_ld();
                     if (n_valid == kC) {
+                        // the previous chunk's store has read the staging tile (it had a whole
+                        // chunk to do so)
+                        if (r == 0) bulk_wait_read();
+                        named_bar_sync(nb, 128);
                         TY *ys = reinterpret_cast<TY *>(smem + OFF_YST + hh * YST_HALF);
 #pragma unroll
                         for (int jt = 0; jt < 32; ++jt) ys[jt * kD + r] = from_f32<TY>(__uint_as_float(ya[jt]));
