@@ -18,7 +18,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "decode_step", "gate_norm", "device_error", "lib", "LIB_PATH",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "selftest_bounded_wait", "decode_step", "gate_norm", "device_error", "lib", "LIB_PATH",
            "GdnError", "EXPORTED_SYMBOLS", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn_b200.so")
@@ -28,7 +28,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc",
-                    "gdn_decode_step",
+                    "gdn_selftest_bounded_wait", "gdn_decode_step",
                     "gdn_gate_norm", "gdn_status_string", "gdn_device_error", "gdn_version")
 
 
@@ -63,6 +63,8 @@ def lib():
         L.gdn_chunk_fwd_noalloc.restype = i32
         L.gdn_chunk_fwd_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                             i32, f32, vp, i32, vp, vp]
+        L.gdn_selftest_bounded_wait.restype = i32
+        L.gdn_selftest_bounded_wait.argtypes = [i64, i32, vp]
         L.gdn_decode_step.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, vp, vp]
         L.gdn_gate_norm.restype = i32
@@ -225,6 +227,15 @@ def gate_norm(y, z, w, eps=1e-6, out=None, out_dtype=None):
                              dv, float(eps), _ptr(o), _dtype_code(o), _stream(y.device))
     _check("gdn_gate_norm", rc)
     return o
+
+
+def selftest_bounded_wait(limit_cycles=2_000_000, mode=0, device=None):
+    """Runs the kernels' bounded wait on the device (see gdn_selftest_bounded_wait) and
+    returns the device error status it leaves: "GDN_ERR_TIMEOUT" for mode 0 (the wait ran
+    out), "GDN_OK" for modes 1 (aborted by another thread) and 2 (completed)."""
+    dev = device if device is not None else torch.cuda.current_device()
+    _check("gdn_selftest_bounded_wait", lib().gdn_selftest_bounded_wait(int(limit_cycles), int(mode), _stream(dev)))
+    return device_error(dev)
 
 
 def device_error(device=None) -> str:

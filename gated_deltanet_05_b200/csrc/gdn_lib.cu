@@ -118,6 +118,36 @@ int device_sm_count()
     return n;
 }
 
+// Device check of the kernels' bounded mbarrier wait (gdn_selftest_bounded_wait). Thread 0
+// waits on a phase of a fresh barrier; mode 0: nothing completes it (the wait must give up
+// after `limit` cycles and record a timeout); mode 1: thread 32 raises the abort flag after
+// a short delay (the wait must return early without recording anything); mode 2: thread 32
+// completes the phase (the wait must succeed). Only the timeout records an error.
+__global__ void selftest_wait_kernel(long long limit, int mode)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        gdn::sm100::mbar_init(&bar, 1);
+        abort_flag = 0;
+        gdn::sm100::fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const bool ok = gdn::sm100::mbar_wait_bounded(&bar, 0, &abort_flag, limit);
+        // a wait that returned the wrong answer for its mode is an internal-check failure
+        if (ok != (mode == 2)) gdn::raise_error(gdn::kErrCheck);
+    } else if (threadIdx.x == 32 && mode != 0) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < 20000) {}
+        if (mode == 1) {
+            *reinterpret_cast<volatile int *>(&abort_flag) = 1;
+        } else {
+            gdn::sm100::mbar_arrive(&bar);
+        }
+    }
+}
+
 // Fixed scratch of gdn_chunk_fwd_noalloc: the tensor-core kernel's K ring for up to
 // kNoAllocMaxSms SM ids, as a file-scope device array (one copy per device, created with
 // the module; never allocated by a call).
@@ -237,6 +267,14 @@ gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gd
     if (need > 0 && cudaGetSymbolAddress(&ws, g_noalloc_ws) != cudaSuccess) return GDN_ERR_CUDA;
     return gdn_chunk_fwd(q, k, v, in_dtype, log_alpha, beta, S0, cu_seqlens_dev, cu_seqlens_host, n_seq, H,
                          d_k, d_v, chunk, scale, y, y_dtype, S_T, ws, need, stream);
+}
+
+gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *stream)
+{
+    if (limit_cycles < 1 || limit_cycles > 2000000000LL || mode < 0 || mode > 2) return GDN_ERR_INVALID_ARG;
+    if (mode == 1 && limit_cycles < 1000000) return GDN_ERR_INVALID_ARG;   // the abort must come first
+    selftest_wait_kernel<<<1, 64, 0, as_stream(stream)>>>((long long)limit_cycles, mode);
+    return launch_status();
 }
 
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype in_dtype,

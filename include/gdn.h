@@ -131,6 +131,21 @@ gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gd
                                  void *y, gdn_dtype y_dtype, float *S_T, void *stream);
 
 /*
+ * gdn_selftest_bounded_wait -- runs the bounded mbarrier wait that every prefill-kernel
+ * role uses, on the device, in one small CTA (failure handling; no counterpart in the
+ * pages). Thread 0 waits on a barrier phase:
+ *   mode 0: nothing completes it. After limit_cycles SM clocks the wait gives up and records
+ *           GDN_ERR_TIMEOUT in the device error word, and the kernel exits normally.
+ *   mode 1: another thread raises the kernel's abort flag after ~20K cycles. The wait returns
+ *           at once and records nothing. limit_cycles >= 1e6 so that the abort comes first.
+ *   mode 2: another thread completes the phase. The wait succeeds and records nothing.
+ * A wait that returns the wrong answer for its mode records GDN_ERR_DEVICE_CHECK.
+ * limit_cycles in [1, 2e9] (the kernels use 2e9, about 1 s). Asynchronous on `stream`; read
+ * the outcome with gdn_device_error. GDN_ERR_INVALID_ARG for out-of-range arguments.
+ */
+gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *stream);
+
+/*
  * gdn_decode_step -- one token for each of n_seq * H independent chains, in place.
  *
  * Defines: the same four-line update (joezjh.github.io notes, "Gated DeltaNet 核心机制")

@@ -89,6 +89,13 @@ def test_chunk_fwd_rejects_bad_arguments(L):
     assert _chunk(L) != 0                                   # tensor-core path without its workspace
 
 
+def test_selftest_rejects_bad_arguments(L):
+    assert L.gdn_selftest_bounded_wait(0, 0, None) == 1          # limit out of range
+    assert L.gdn_selftest_bounded_wait(3_000_000_000, 0, None) == 1
+    assert L.gdn_selftest_bounded_wait(1000, 3, None) == 1       # unknown mode
+    assert L.gdn_selftest_bounded_wait(1000, 1, None) == 1       # abort needs a long limit
+
+
 def test_decode_and_gate_norm_reject_bad_arguments(L):
     dec = lambda **kw: L.gdn_decode_step(kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 0), FAKE,
                                          FAKE, kw.get("S", FAKE), kw.get("n", 4), kw.get("H", 2),
