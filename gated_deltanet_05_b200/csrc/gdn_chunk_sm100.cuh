@@ -71,7 +71,8 @@ namespace sm100 {
 constexpr int kC = 64;       // chunk length
 constexpr int kD = 128;      // d_k = d_v
 constexpr int kThreads = 384;
-constexpr int kStages = 3;   // TMA ring depth of both CTAs
+constexpr int kStages = 3;   // K ring depth of the chain CTA
+constexpr int kSvStages = 2; // K/Q TMA ring depth of the solver CTA
 constexpr int kRing = 4;     // K/Q chunks in flight through global memory, per solver SM
 constexpr int kRecv = 2;     // solver-operand slots in the chain CTA
 constexpr int kQVStages = 2; // Q/V ring of the chain CTA
@@ -84,23 +85,23 @@ constexpr size_t kWsBytesPerSm = (size_t)kRing * K_BYTES;
 
 // ---------------------------------------------------------------- solver CTA layout
 namespace sv {
-constexpr uint32_t OFF_QK = 0;          // kStages x 32 KB, bf16 as loaded, then fp16 in place
+constexpr uint32_t OFF_QK = 0;          // kSvStages x 32 KB, bf16 as loaded, then fp16 in place
 constexpr uint32_t QK_STAGE = 32768;
-constexpr uint32_t OFF_SEND = OFF_QK + kStages * QK_STAGE;   // per solve group: one chunk's operands
+constexpr uint32_t OFF_SEND = OFF_QK + kSvStages * QK_STAGE; // per solve group: two chunks' operands
 constexpr int LS_LD = 68;
 constexpr uint32_t LS_BYTES = 64 * LS_LD * 4;                // fp32 [64][68]: L, then T in place
-constexpr uint32_t OFF_LS = OFF_SEND + 2 * TP_BYTES;
+constexpr uint32_t OFF_LS = OFF_SEND + 4 * TP_BYTES;
 constexpr uint32_t RT_BYTES = 4 * 32 * 8 * 4;                // merge temp: [32][8] fp32 per warp
 constexpr uint32_t OFF_RT = OFF_LS + 2 * LS_BYTES;
 constexpr uint32_t GATES_BYTES = 4 * 64 * 4;                 // {g2, gamma, beta, 2^(m - g2)}[64]
 constexpr uint32_t OFF_GATES = OFF_RT + 2 * RT_BYTES;
 constexpr uint32_t OFF_BAR = OFF_GATES + 2 * GATES_BYTES;
 enum {
-    B_FULL = 0, B_EMPTY = B_FULL + kStages, B_CREADY = B_EMPTY + kStages, B_GFULL = B_CREADY + kStages,
+    B_FULL = 0, B_EMPTY = B_FULL + kSvStages, B_CREADY = B_EMPTY + kSvStages, B_GFULL = B_CREADY + kSvStages,
     // RECV_EMPTY: chain slot of chunk c free again, one barrier per c % (2 kRecv) so that
-    // each has a single waiting solve group; LANDED: a group's send buffer copied out
+    // each has a single waiting solve group; LANDED: the send buffer of chunk c % 4 copied out
     B_GEMPTY = B_GFULL + 2, B_RECV_EMPTY = B_GEMPTY + 2, B_LANDED = B_RECV_EMPTY + 2 * kRecv,
-    B_SCR_EMPTY = B_LANDED + 2, B_DRAIN = B_SCR_EMPTY + kRing, N_BAR
+    B_SCR_EMPTY = B_LANDED + 4, B_DRAIN = B_SCR_EMPTY + kRing, N_BAR
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BAR * 8;           // tmem base, abort flag, sequence, smid
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
@@ -309,12 +310,12 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     tma_prefetch_desc(&tm_q);
                     tma_prefetch_desc(&tm_k);
                 }
-                int issued[kStages] = {};
+                int issued[kSvStages] = {};
 #pragma unroll 1
                 for (int c = 0; c < n_chunks; ++c) {
-                    const int st = c % kStages;
+                    const int st = c % kSvStages;
                     // the stage is free once its fp16 K tile has been copied out
-                    if (c >= kStages && !wait_w(B_EMPTY + st, c / kStages - 1)) break;
+                    if (c >= kSvStages && !wait_w(B_EMPTY + st, c / kSvStages - 1)) break;
                     const int tok = (int)(bos + (int64_t)c * kC);
                     uint8_t *qk = smem + OFF_QK + st * QK_STAGE;
                     mbar_arrive_expect_tx_lead(&bar[B_FULL + st], QK_STAGE, lead);
@@ -324,8 +325,8 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     tma_load_3d_lead(qk + 24576, &tm_q, &bar[B_FULL + st], 64, head, tok, lead);
                     issued[st] = c + 1;
                 }
-                for (int st = 0; st < kStages; ++st)
-                    if (issued[st] > 0) mbar_wait_drain(&bar[B_FULL + st], ((issued[st] - 1) / kStages) & 1, kWaitLimit);
+                for (int st = 0; st < kSvStages; ++st)
+                    if (issued[st] > 0) mbar_wait_drain(&bar[B_FULL + st], ((issued[st] - 1) / kSvStages) & 1, kWaitLimit);
             }
         } else if (warp == 1) {
             // ============================================================ G = [K; Q] K^T issuer
@@ -335,8 +336,8 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const uint64_t dqk0 = sdesc_sw128(sbase + OFF_QK, 16, 1024);
 #pragma unroll 1
                 for (int c = 0; c < n_chunks; ++c) {
-                    const int st = c % kStages;
-                    if (!wait_w(B_FULL + st, c / kStages)) break;
+                    const int st = c % kSvStages;
+                    if (!wait_w(B_FULL + st, c / kSvStages)) break;
                     if (c >= 2 && !wait_w(B_GEMPTY + (c & 1), (c >> 1) - 1)) break;
                     tc_fence_after();
                     const uint64_t base = dqk0 + GDN_DOFF(st * QK_STAGE);
@@ -362,9 +363,9 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint32_t lead = elect_one();    // in warp 2: the lane that issues the ring stores
             int stored = 0;
             for (int c = 0; c < n_chunks; ++c) {
-                const int st = c % kStages;
+                const int st = c % kSvStages;
                 bool ok = true;
-                if (u == 0) ok = wait(B_CREADY + st, c / kStages);
+                if (u == 0) ok = wait(B_CREADY + st, c / kSvStages);
                 if (!named_bar_and(5, 64, ok)) break;
                 uint8_t *qk = smem + OFF_QK + st * QK_STAGE;
                 // A whole 128-byte row is rewritten, so the swizzle does not matter; the
@@ -415,7 +416,6 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             float *Rt = reinterpret_cast<float *>(smem + OFF_RT + j * RT_BYTES);
             float *g2s = reinterpret_cast<float *>(smem + OFF_GATES + j * GATES_BYTES);
             float *gam = g2s + 64, *bet = g2s + 128, *bfac = g2s + 192;
-            uint8_t *send = smem + OFF_SEND + j * TP_BYTES;
             const bool gate_warp = (warp & 3) == 0;
             // log alpha and beta of this group's next chunk, loaded one chunk ahead
             float la0 = 0.f, la1 = 0.f, be0 = 0.f, be1 = 0.f;
@@ -445,11 +445,12 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     bfac[lane + 32] = fast_exp2(mid - g_hi);
                     if (c + 2 < n_chunks) load_gates(c + 2);
                 }
-                // (a) the send buffer is free once its previous copy (chunk c - 2) has landed;
-                // G rows: K K^T (lanes 0..63), Q K^T (lanes 64..127)
+                // (a) the group's two send buffers alternate: this one is free once its previous
+                // copy (chunk c - 4) has landed; G rows: K K^T (lanes 0..63), Q K^T (lanes 64..127)
+                uint8_t *send = smem + OFF_SEND + (c & 3) * TP_BYTES;
                 bool ok = true;
                 if (r == 0) {
-                    if (c >= 2) ok = wait_cl(B_LANDED + j, (c >> 1) - 1);
+                    if (c >= 4) ok = wait_cl(B_LANDED + (c & 3), (c >> 2) - 1);
                     if (ok) ok = wait(B_GFULL + j, c >> 1);
                 }
                 if (!named_bar_and(nb, 128, ok)) break;
@@ -724,7 +725,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     if (!wait_w(B_K_FULL + c % kStages, c / kStages)) return false;
                     mbar_arrive_remote_relaxed_lead(scr_empty0 + (uint32_t)(c % kRing) * 8u, lead);   // ring slot reusable
                     if (!wait_cl_w(B_RECV + c % kRecv, c / kRecv)) return false;
-                    mbar_arrive_remote_relaxed_lead(landed0 + (uint32_t)(c & 1) * 8u, lead);          // send buffer reusable
+                    mbar_arrive_remote_relaxed_lead(landed0 + (uint32_t)(c & 3) * 8u, lead);          // send buffer reusable
                     tc_fence_after();
                     const uint64_t kt = dkt0 + GDN_DOFF((c % kStages) * K_BYTES);
                     const uint64_t tbg = dop0 + GDN_DOFF((c % kRecv) * TP_BYTES);
