@@ -9,7 +9,9 @@ stores the transpose ([.., d_v, d_k]); `state_to_lib` / `state_from_lib` convert
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py (the
 equivalent update form, brute-force matrix products, invariants, closed forms and
-a hand-worked example).
+a hand-worked example) and, for the featurisation, tests/test_oracle_featurize.py
+(a library convolution, the impulse response, sequence isolation, unit norms and the
+gates' closed forms).
 """
 from __future__ import annotations
 
@@ -50,6 +52,10 @@ def _configure(lib):
     lib.gdn_oracle_gate_norm.restype = ctypes.c_int
     lib.gdn_oracle_gate_norm.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int,
                                          ctypes.c_double, _dp]
+    lib.gdn_oracle_featurize.restype = ctypes.c_int
+    lib.gdn_oracle_featurize.argtypes = ([_dp] * 6 + [ctypes.c_int] + [_dp] * 4 +
+                                         [_i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_double] + [_dp] * 5)
     return lib
 
 
@@ -143,3 +149,33 @@ def gate_norm(y, z, w, eps=1e-6):
                                     _ptr(o)) < 0:
         raise ValueError("gdn_oracle_gate_norm: bad argument")
     return o
+
+
+def featurize(xq, xk, xv, conv_q, conv_k, conv_v, beta_logit, alpha_logit, A, b_alpha,
+              cu_seqlens, eps=1e-6):
+    """Short causal convolution -> SiLU -> L2 norm (q, k) and the two gates, in fp64.
+
+    xq, xk: [N, H, dk]; xv: [N, H, dv]; conv_q, conv_k: [H*dk, W]; conv_v: [H*dv, W]
+    (tap j multiplies the token W-1-j places back); beta_logit, alpha_logit: [N, H];
+    A, b_alpha: [H]. Returns (q, k, v, beta, log_alpha)."""
+    xq, xk, xv = _f64(xq), _f64(xk), _f64(xv)
+    cq, ck, cv = _f64(conv_q), _f64(conv_k), _f64(conv_v)
+    bl, al, A, ba = _f64(beta_logit), _f64(alpha_logit), _f64(A), _f64(b_alpha)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens if not hasattr(cu_seqlens, "numpy")
+                                         else cu_seqlens.numpy(), dtype=np.int64))
+    n_seq = cu.shape[0] - 1
+    N, H, dk = xq.shape
+    dv = xv.shape[2]
+    W = cq.shape[1]
+    assert xk.shape == (N, H, dk) and xv.shape[:2] == (N, H) and int(cu[-1]) == N
+    assert cq.shape == (H * dk, W) and ck.shape == (H * dk, W) and cv.shape == (H * dv, W)
+    assert bl.shape == (N, H) and al.shape == (N, H) and A.shape == (H,) and ba.shape == (H,)
+    q, k = np.zeros((N, H, dk)), np.zeros((N, H, dk))
+    v = np.zeros((N, H, dv))
+    beta, log_alpha = np.zeros((N, H)), np.zeros((N, H))
+    if _load().gdn_oracle_featurize(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(cq), _ptr(ck), _ptr(cv),
+                                    int(W), _ptr(bl), _ptr(al), _ptr(A), _ptr(ba),
+                                    cu.ctypes.data_as(_i64p), n_seq, H, dk, dv, float(eps),
+                                    _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha)) < 0:
+        raise ValueError("gdn_oracle_featurize: bad argument")
+    return q, k, v, beta, log_alpha

@@ -268,3 +268,77 @@ int gdn_oracle_gate_norm(const double *y, const double *z, const double *w, int6
     }
     return 1;
 }
+
+/* ---------------------------------------------------------------- featurisation */
+
+/*
+ * The feature and gate computation in front of the recurrence (joezjh.github.io notes
+ * page "Qwen3.8-Flash-Next", section "GDN 参数化细节", the q/k/v equations and the gate
+ * equations; pwwt.cn translation, section 2.1.1, Figure 2 caption: a short causal
+ * convolution on the projected q, k, v streams, L2 normalisation of q and k only).
+ * The projections W x are inputs here (plain GEMMs outside this step):
+ *
+ *   c_t     = sum_{j < W} w[ch][j] * x_{t - (W-1) + j}     per channel, x = 0 before the
+ *                                                           sequence's first token
+ *   f_t     = SiLU(c_t) = c_t / (1 + exp(-c_t))
+ *   q_t,k_t = f_t / sqrt(sum_ch f_t^2 + eps)               per (token, head), over d
+ *   v_t     = f_t
+ *   beta_t  = 1 / (1 + exp(-beta_logit_t))
+ *   log alpha_t = -exp(A_h) * softplus(alpha_logit_t + b_alpha_h)
+ *
+ * Tap j of a channel's W weights multiplies the token W-1-j places back (the weight
+ * layout of a depthwise PyTorch Conv1d padded by W-1 and cut to its first T outputs).
+ * x*, out*: [n_tok][H][d] (d = dk for q, k and dv for v); conv_*: [H*d][W];
+ * logits, beta, log_alpha: [n_tok][H]; A, b_alpha: [H]. Single threaded.
+ */
+static void featurize_stream(const double *x, const double *cw, int W, const int64_t *cu, int n_seq,
+                             int H, int d, int l2, double eps, double *out)
+{
+    for (int i = 0; i < n_seq; ++i)
+        for (int64_t t = cu[i]; t < cu[i + 1]; ++t)
+            for (int h = 0; h < H; ++h) {
+                double *o = out + ((size_t)t * H + h) * d;
+                for (int c = 0; c < d; ++c) {
+                    const double *w = cw + ((size_t)h * d + c) * W;
+                    double acc = 0.0;
+                    for (int j = 0; j < W; ++j) {
+                        const int64_t s = t - (W - 1) + j;
+                        if (s >= cu[i])
+                            acc += w[j] * x[((size_t)s * H + h) * d + c];
+                    }
+                    o[c] = acc / (1.0 + exp(-acc));
+                }
+                if (l2) {
+                    double ss = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        ss += o[c] * o[c];
+                    const double inv = 1.0 / sqrt(ss + eps);
+                    for (int c = 0; c < d; ++c)
+                        o[c] *= inv;
+                }
+            }
+}
+
+static double softplus(double x) { return x > 0.0 ? x + log1p(exp(-x)) : log1p(exp(x)); }
+
+int gdn_oracle_featurize(const double *xq, const double *xk, const double *xv, const double *conv_q,
+                         const double *conv_k, const double *conv_v, int W, const double *beta_logit,
+                         const double *alpha_logit, const double *A, const double *b_alpha,
+                         const int64_t *cu, int n_seq, int H, int dk, int dv, double eps, double *q,
+                         double *k, double *v, double *beta, double *log_alpha)
+{
+    if (!xq || !xk || !xv || !conv_q || !conv_k || !conv_v || !beta_logit || !alpha_logit || !A ||
+        !b_alpha || !cu || !q || !k || !v || !beta || !log_alpha || W < 1 || n_seq < 0 || H <= 0 ||
+        dk <= 0 || dv <= 0)
+        return -1;
+    featurize_stream(xq, conv_q, W, cu, n_seq, H, dk, 1, eps, q);
+    featurize_stream(xk, conv_k, W, cu, n_seq, H, dk, 1, eps, k);
+    featurize_stream(xv, conv_v, W, cu, n_seq, H, dv, 0, eps, v);
+    for (int64_t t = cu[0]; t < cu[n_seq]; ++t)
+        for (int h = 0; h < H; ++h) {
+            const size_t e = (size_t)t * H + h;
+            beta[e] = 1.0 / (1.0 + exp(-beta_logit[e]));
+            log_alpha[e] = -exp(A[h]) * softplus(alpha_logit[e] + b_alpha[h]);
+        }
+    return 1;
+}

@@ -13,6 +13,7 @@ import types
 import pytest
 
 import oracle
+from tests import test_oracle_featurize as fpins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
@@ -57,6 +58,16 @@ MUTANTS = {
     "norm_mean_off_by_one": [("sqrt(ss / dv + eps)", "sqrt(ss / (dv - 1) + eps)")],
     "gate_silu": [("const double gate = 1.0 / (1.0 + exp(-zr[j]));",
                    "const double gate = zr[j] / (1.0 + exp(-zr[j]));")],
+    # featurisation: taps in the wrong order, a window that crosses sequence starts, no
+    # SiLU, v normalised too, the decay bias dropped, the decay rate not exponentiated
+    "conv_taps_reversed": [("acc += w[j] * x[((size_t)s * H + h) * d + c];",
+                            "acc += w[W - 1 - j] * x[((size_t)s * H + h) * d + c];")],
+    "conv_crosses_sequences": [("if (s >= cu[i])\n", "if (s >= 0)\n")],
+    "no_silu": [("o[c] = acc / (1.0 + exp(-acc));", "o[c] = acc;")],
+    "v_normalised": [("featurize_stream(xv, conv_v, W, cu, n_seq, H, dv, 0, eps, v);",
+                      "featurize_stream(xv, conv_v, W, cu, n_seq, H, dv, 1, eps, v);")],
+    "decay_bias_dropped": [("softplus(alpha_logit[e] + b_alpha[h]);", "softplus(alpha_logit[e]);")],
+    "decay_rate_not_exp": [("log_alpha[e] = -exp(A[h]) * softplus", "log_alpha[e] = -A[h] * softplus")],
 }
 
 PIN_TESTS = [
@@ -70,7 +81,7 @@ PIN_TESTS = [
     pins.test_hand_example,
     pins.test_decode_step_matches_one_token_recurrence,
     pins.test_gate_norm_closed_forms,
-]
+] + fpins.PINS
 
 
 def _mutant_module(tmp_path, name, edits):
@@ -85,7 +96,7 @@ def _mutant_module(tmp_path, name, edits):
                     str(c_path), "-lm", "-lpthread"], check=True)
     lib = oracle._configure(ctypes.CDLL(str(so_path)))
     mod = types.SimpleNamespace()
-    for fn in ("recurrent", "decode_step", "gate_norm"):
+    for fn in ("recurrent", "decode_step", "gate_norm", "featurize"):
         f = getattr(oracle, fn)
 
         def wrapped(*a, _f=f, **kw):
