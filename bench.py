@@ -9,7 +9,8 @@ synthetic draws (workloads/), resident in HBM before the timed region; q, k, v a
 (256 MiB) exceed the 126 MB L2, so no flush is needed between steps.
 
 The decode step (256 sequences x 32 heads, d = 128, 537 MB fp32 state in HBM) is timed
-separately and reported under "decode".
+separately and reported under "decode"; the featurisation step in front of the prefill
+(gdn_featurize on the prefill workload's shape) under "featurize".
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent batch
 (the chains do not interact), so scaling is weak and the data path has no collective;
@@ -334,6 +335,7 @@ def run_ours(args, rank, world, local, pg):
                      "bytes_per_launch": gn_bytes}
 
     decode = None if args.no_decode else bench_decode(args, device, peaks, peak_kind, pg)
+    featurize = bench_featurize(args, device, peaks, peak_kind, pg, rank)
     e2e = bench_e2e(args, inp, device, pg, world)
 
     line = {
@@ -348,6 +350,7 @@ def run_ours(args, rank, world, local, pg):
         "roofline": roofline,
         "gate_norm": gate_norm_obj,
         "decode": decode,
+        "featurize": featurize,
         "e2e": e2e,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
@@ -395,11 +398,88 @@ def bench_decode(args, device, peaks, peak_kind, pg):
     state_bytes = n * H * d * d * 4
     step_bytes = 2 * state_bytes + n * H * (3 * d * 4 + d * 4 + 8)
     gbs = step_bytes / (ms * 1e-3) / 1e9
+
+    # several tokens per call (next_n = 4): one pass over the state for 4 tokens
+    nt = 4
+    staged_t = []
+    for s_ in range(4):
+        xs = [W.make_decode_inputs(w, 1000 + s_ * nt + i) for i in range(nt)]
+        staged_t.append({key: torch.stack([x[key] for x in xs], 1).contiguous().to(device)
+                         for key in ("q", "k", "v", "alpha", "beta")})
+    y_t = torch.empty((n, nt, H, d), dtype=torch.float32, device=device)
+
+    def multi(i):
+        x = staged_t[i % len(staged_t)]
+        gdn.decode_tokens(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S, out=y_t)
+
+    for i in range(max(3, args.warmup)):
+        multi(i)
+    torch.cuda.synchronize(device)
+    barrier(pg, device)
+    a.record(stream)
+    for i in range(steps):
+        multi(i)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms_t = max_over_ranks(pg, a.elapsed_time(b), device) / steps
+    call_bytes = 2 * state_bytes + nt * n * H * (3 * d * 4 + d * 4 + 8)
+    gbs_t = call_bytes / (ms_t * 1e-3) / 1e9
+    status = gdn.device_error(device)
+    if status != "GDN_OK":
+        raise SystemExit(f"device error in the decode leg: {status}")
     return {"workload": "decode fp32 state: 256 seqs x H=32, d_k=d_v=128, one token per step",
             "ms_per_step": ms, "tokens_per_s": n / (ms * 1e-3), "bytes_per_step": step_bytes,
             "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
-            "steps": steps, "l2": "state 537 MB > L2"}
+            "steps": steps, "l2": "state 537 MB > L2",
+            "tokens_4": {"kernel": "gdn::decode_tokens_kernel", "tokens_per_call": nt,
+                         "ms_per_call": ms_t, "tokens_per_s": n * nt / (ms_t * 1e-3),
+                         "bytes_per_call": call_bytes, "achieved": gbs_t, "unit": "GB/s",
+                         "frac": gbs_t / peaks["hbm_gbs"]}}
+
+
+def bench_featurize(args, device, peaks, peak_kind, pg, rank):
+    """The featurisation step in front of the prefill (short conv, SiLU, L2 norm, gates)
+    on the prefill workload's shape: 4 x 4096 tokens, H = 16, d = 128, bf16 streams."""
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    import workloads as W
+    w = W.WORKLOADS["prefill"]
+    inp = W.make_featurize_inputs(w, seed=w.seed + 7 + 1000 * rank)
+    keys = ("xq", "xk", "xv", "conv_q", "conv_k", "conv_v", "beta_logit", "alpha_logit", "A",
+            "b_alpha", "cu_seqlens")
+    dev = [inp[k].to(device) for k in keys]
+    n_tok, H, d = inp["xq"].shape
+    cu_host = inp["cu_seqlens"]
+    out = (torch.empty_like(dev[0]), torch.empty_like(dev[1]), torch.empty_like(dev[2]),
+           torch.empty((n_tok, H), dtype=torch.float32, device=device),
+           torch.empty((n_tok, H), dtype=torch.float32, device=device))
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(3, args.warmup)):
+        gdn.featurize(*dev, cu_seqlens_host=cu_host, out=out)
+    torch.cuda.synchronize(device)
+    steps = max(args.steps, 20)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(pg, device)
+    a.record(stream)
+    for _ in range(steps):
+        gdn.featurize(*dev, cu_seqlens_host=cu_host, out=out)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    status = gdn.device_error(device)
+    if status != "GDN_OK":
+        raise SystemExit(f"device error in the featurisation leg: {status}")
+    ms = max_over_ranks(pg, a.elapsed_time(b), device) / steps
+    # read x (3 streams) + 2 logits, write q, k, v + beta, log alpha; plus the weights
+    step_bytes = n_tok * H * 2 * (3 * d * 2 + 2 * 4) + 3 * H * d * 4 * 4 + 2 * H * 4
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    return {"workload": "featurisation bf16: 4 seqs x 4096 tokens, H=16, d=128, conv width 4",
+            "kernel": "gdn::featurize_kernel (2 launches)", "launch_ms": ms,
+            "bytes_per_launch": step_bytes, "achieved": gbs, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+            "steps": steps, "l2": "inputs 192 MiB > L2"}
 
 
 def bench_e2e(args, inp, device, pg, world):
@@ -466,7 +546,8 @@ def run_case(args):
     """A few launches of one kernel on a named shape, nothing else (for ncu captures):
     --case prefill:S,T,H   (bf16, d=128, chunk 64, fp32 y)
     --case decode:N        (N sequences x 32 heads, d=128, fp32 state)
-    --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)"""
+    --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)
+    --case featurize:S,T,H (bf16, d=128, conv width 4)"""
     import torch
 
     import gated_deltanet_05_b200 as gdn
@@ -496,6 +577,15 @@ def run_case(args):
         wn = (torch.randn(128, generator=g) * 0.02).cuda()
         for _ in range(args.reps):
             gdn.gate_norm(y, z, wn, out_dtype=torch.bfloat16)
+    elif kind == "featurize":
+        n_seq, T, H = dims
+        w = W.Workload("case", "bf16", (T,) * n_seq, H, 128, 128, 64, seed=1)
+        inp = W.make_featurize_inputs(w)
+        keys = ("xq", "xk", "xv", "conv_q", "conv_k", "conv_v", "beta_logit", "alpha_logit", "A",
+                "b_alpha", "cu_seqlens")
+        dev = [inp[k].cuda() for k in keys]
+        for _ in range(args.reps):
+            gdn.featurize(*dev, cu_seqlens_host=inp["cu_seqlens"])
     else:
         raise SystemExit(f"unknown case {args.case}")
     torch.cuda.synchronize()

@@ -7,7 +7,10 @@ importing works but every call raises RuntimeError.
 
     y, S_T = chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64)
     y = decode_step(q, k, v, alpha, beta, S)          # S updated in place
+    y = decode_tokens(q, k, v, alpha, beta, S)        # [n_seq, n, H, d]: n tokens, one pass
     o = gate_norm(y, z, w, eps=1e-6)
+    q, k, v, beta, log_alpha = featurize(xq, xk, xv, conv_q, conv_k, conv_v,
+                                         beta_logit, alpha_logit, A, b_alpha, cu_seqlens)
 
 State tensors use the library's value-major layout [.., d_v, d_k] in fp32.
 """
@@ -18,7 +21,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "selftest_bounded_wait", "decode_step", "gate_norm", "device_error", "lib", "LIB_PATH",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "selftest_bounded_wait", "decode_step", "decode_tokens", "gate_norm", "featurize",
+           "device_error", "lib", "LIB_PATH",
            "GdnError", "EXPORTED_SYMBOLS", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn_b200.so")
@@ -28,8 +32,9 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc",
-                    "gdn_selftest_bounded_wait", "gdn_decode_step",
-                    "gdn_gate_norm", "gdn_status_string", "gdn_device_error", "gdn_version")
+                    "gdn_selftest_bounded_wait", "gdn_decode_step", "gdn_decode_tokens",
+                    "gdn_gate_norm", "gdn_featurize", "gdn_status_string", "gdn_device_error",
+                    "gdn_version")
 
 
 class GdnError(RuntimeError):
@@ -67,8 +72,13 @@ def lib():
         L.gdn_selftest_bounded_wait.argtypes = [i64, i32, vp]
         L.gdn_decode_step.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, vp, vp]
+        L.gdn_decode_tokens.restype = i32
+        L.gdn_decode_tokens.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]
         L.gdn_gate_norm.restype = i32
         L.gdn_gate_norm.argtypes = [vp, i32, vp, i32, vp, i64, i32, f32, vp, i32, vp]
+        L.gdn_featurize.restype = i32
+        L.gdn_featurize.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, i32, i64,
+                                    i32, i32, i32, f32, vp, vp, vp, vp, vp, vp]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_status_string.argtypes = [i32]
         L.gdn_device_error.restype = i32
@@ -207,6 +217,23 @@ def decode_step(q, k, v, alpha, beta, S, scale=1.0, out=None):
     return y
 
 
+def decode_tokens(q, k, v, alpha, beta, S, scale=1.0, out=None):
+    """n consecutive tokens per chain in one pass over the state (S updated in place).
+
+    q, k [n_seq, n, H, d_k], v [n_seq, n, H, d_v] (fp32 or bf16, one dtype); alpha, beta
+    [n_seq, n, H] fp32; S [n_seq, H, d_v, d_k] fp32. Returns y [n_seq, n, H, d_v]."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (alpha, "alpha"), (beta, "beta"), (S, "S")):
+        _cuda(t, nm)
+    code = _dtype_code(q)
+    n_seq, n, H, dk = q.shape
+    dv = v.shape[3]
+    y = out if out is not None else torch.empty((n_seq, n, H, dv), dtype=q.dtype, device=q.device)
+    rc = lib().gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha), _ptr(beta), _ptr(S),
+                                 n_seq, n, H, dk, dv, float(scale), _ptr(y), _stream(q.device))
+    _check("gdn_decode_tokens", rc)
+    return y
+
+
 def gate_norm(y, z, w, eps=1e-6, out=None, out_dtype=None):
     """o = sigmoid(z) * y / sqrt(mean(y^2) + eps) * (1 + w) over the last axis.
 
@@ -227,6 +254,54 @@ def gate_norm(y, z, w, eps=1e-6, out=None, out_dtype=None):
                              dv, float(eps), _ptr(o), _dtype_code(o), _stream(y.device))
     _check("gdn_gate_norm", rc)
     return o
+
+
+def featurize(xq, xk, xv, conv_q, conv_k, conv_v, beta_logit, alpha_logit, A, b_alpha, cu_seqlens,
+              eps=1e-6, cu_seqlens_host=None, out=None):
+    """Short causal convolution -> SiLU -> L2 norm (q, k), and the gates, for packed sequences.
+
+    xq, xk [N, H, d_k] and xv [N, H, d_v] (one dtype, fp32 or bf16): the projected streams;
+    conv_q, conv_k [H*d_k, W] and conv_v [H*d_v, W] fp32 (W <= 4; tap j multiplies the token
+    W-1-j places back); beta_logit, alpha_logit [N, H] fp32; A, b_alpha [H] fp32;
+    cu_seqlens [n_seq + 1] int32 (device). Returns (q, k, v, beta, log_alpha): q, k, v in
+    the input dtype and beta, log_alpha fp32, ready for chunk_fwd. `out` may supply those
+    five tensors."""
+    for t, n in ((xq, "xq"), (xk, "xk"), (xv, "xv"), (conv_q, "conv_q"), (conv_k, "conv_k"),
+                 (conv_v, "conv_v"), (beta_logit, "beta_logit"), (alpha_logit, "alpha_logit"),
+                 (A, "A"), (b_alpha, "b_alpha"), (cu_seqlens, "cu_seqlens")):
+        _cuda(t, n)
+    if xk.dtype != xq.dtype or xv.dtype != xq.dtype:
+        raise TypeError("xq, xk, xv must share one dtype")
+    for t, n in ((conv_q, "conv_q"), (conv_k, "conv_k"), (conv_v, "conv_v"), (beta_logit, "beta_logit"),
+                 (alpha_logit, "alpha_logit"), (A, "A"), (b_alpha, "b_alpha")):
+        if t.dtype != torch.float32:
+            raise TypeError(f"{n} must be float32")
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    N, H, dk = xq.shape
+    dv = xv.shape[2]
+    W = conv_q.shape[1]
+    if tuple(conv_q.shape) != (H * dk, W) or tuple(conv_k.shape) != (H * dk, W) or \
+            tuple(conv_v.shape) != (H * dv, W):
+        raise ValueError("conv weights must be [H*d, W] with one W")
+    n_seq = cu_seqlens.numel() - 1
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.to("cpu")
+    cu_h = cu_seqlens_host.to(torch.int32).contiguous()
+    if out is None:
+        out = (torch.empty_like(xq), torch.empty_like(xk), torch.empty_like(xv),
+               torch.empty((N, H), dtype=torch.float32, device=xq.device),
+               torch.empty((N, H), dtype=torch.float32, device=xq.device))
+    for t, n in zip(out, ("q", "k", "v", "beta", "log_alpha")):
+        _cuda(t, n)
+    q, k, v, beta, log_alpha = out
+    rc = lib().gdn_featurize(_ptr(xq), _ptr(xk), _ptr(xv), _dtype_code(xq), _ptr(conv_q), _ptr(conv_k),
+                             _ptr(conv_v), int(W), _ptr(beta_logit), _ptr(alpha_logit), _ptr(A),
+                             _ptr(b_alpha), _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), n_seq,
+                             N, H, dk, dv, float(eps), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                             _ptr(log_alpha), _stream(xq.device))
+    _check("gdn_featurize", rc)
+    return q, k, v, beta, log_alpha
 
 
 def selftest_bounded_wait(limit_cycles=2_000_000, mode=0, device=None):

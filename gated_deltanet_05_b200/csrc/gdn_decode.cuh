@@ -86,3 +86,119 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
 }
 
 }  // namespace gdn
+
+namespace gdn {
+
+// ---------------------------------------------------------------- several tokens per call
+//
+// n (<= kDecodeMaxTokens) consecutive tokens of every chain in one pass over S: the same
+// update as decode_step_kernel, applied token after token to each row while the row stays
+// in registers, so the state is read and written once per call instead of once per
+// token. A lane holds 16 consecutive elements of a row (LPR = d_k / 16 lanes per row), so
+// each of the two dot products per row and token costs log2(LPR) shuffles. The tokens'
+// k, scale q, v, alpha, beta and k.(scale q) are staged in shared memory first.
+constexpr int kDecodeMaxTokens = 8;
+constexpr int kDecodeTokThreads = 256;
+
+template <int DK, typename T>
+__global__ void __launch_bounds__(kDecodeTokThreads)
+decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                     const float *__restrict__ alpha, const float *__restrict__ beta,
+                     float *__restrict__ S, int n, int H, int dv, float scale, T *__restrict__ y)
+{
+    constexpr int LPR = DK / 16;             // lanes per row, 16 elements each
+    constexpr int RPW = 32 / LPR;            // rows per warp pass
+    constexpr int WARPS = kDecodeTokThreads / 32;
+    constexpr int ROWS_IN_FLIGHT = 2;
+    __shared__ float4 sk[kDecodeMaxTokens][DK / 4], sq[kDecodeMaxTokens][DK / 4];
+    __shared__ float sv[kDecodeMaxTokens][128];
+    __shared__ float sa[kDecodeMaxTokens], sb[kDecodeMaxTokens], skq[kDecodeMaxTokens];
+
+    const int chain = blockIdx.x;            // seq * H + head
+    const int seq = chain / H, head = chain % H;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // token i of this chain sits at row (seq * n + i) * H + head of the [n_seq * n, H, .] inputs
+    auto tok_row = [&](int i) -> size_t { return ((size_t)seq * n + i) * H + head; };
+
+    for (int e = threadIdx.x; e < n * (DK / 4); e += kDecodeTokThreads) {
+        const int i = e / (DK / 4), c4 = e % (DK / 4);
+        sk[i][c4] = load4(k + tok_row(i) * DK + 4 * c4);
+        float4 qq = load4(q + tok_row(i) * DK + 4 * c4);
+        qq.x *= scale; qq.y *= scale; qq.z *= scale; qq.w *= scale;
+        sq[i][c4] = qq;
+    }
+    for (int e = threadIdx.x; e < n * dv; e += kDecodeTokThreads) {
+        const int i = e / dv, j = e % dv;
+        sv[i][j] = to_f32(v[tok_row(i) * dv + j]);
+    }
+    if (threadIdx.x < n) {
+        sa[threadIdx.x] = alpha[tok_row(threadIdx.x)];
+        sb[threadIdx.x] = beta[tok_row(threadIdx.x)];
+    }
+    __syncthreads();
+    if (warp < n) {                           // k_i . (scale q_i), one warp per token
+        float acc = 0.f;
+        for (int c4 = lane; c4 < DK / 4; c4 += 32) {
+            const float4 a = sk[warp][c4], b = sq[warp][c4];
+            acc += a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+        }
+        acc = group_sum<32>(acc);
+        if (lane == 0) skq[warp] = acc;
+    }
+    __syncthreads();
+
+    const int part = lane % LPR, sub = lane / LPR;
+    float *Sc = S + (size_t)chain * dv * DK;
+    const int rows_per_round = WARPS * RPW * ROWS_IN_FLIGHT;
+    for (int base = 0; base < dv; base += rows_per_round) {
+        float s[ROWS_IN_FLIGHT][16];
+        int row[ROWS_IN_FLIGHT];
+#pragma unroll
+        for (int f = 0; f < ROWS_IN_FLIGHT; ++f) {
+            row[f] = base + (f * WARPS + warp) * RPW + sub;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4 x = row[f] < dv ? load4(Sc + (size_t)row[f] * DK + 16 * part + 4 * c)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                s[f][4 * c] = x.x; s[f][4 * c + 1] = x.y; s[f][4 * c + 2] = x.z; s[f][4 * c + 3] = x.w;
+            }
+        }
+#pragma unroll 1
+        for (int i = 0; i < n; ++i) {
+            float kv[16], qv[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4 a = sk[i][4 * part + c], b = sq[i][4 * part + c];
+                kv[4 * c] = a.x; kv[4 * c + 1] = a.y; kv[4 * c + 2] = a.z; kv[4 * c + 3] = a.w;
+                qv[4 * c] = b.x; qv[4 * c + 1] = b.y; qv[4 * c + 2] = b.z; qv[4 * c + 3] = b.w;
+            }
+            const float a = sa[i], b = sb[i], kq = skq[i];
+#pragma unroll
+            for (int f = 0; f < ROWS_IN_FLIGHT; ++f) {
+                float u = 0.f, r = 0.f;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    u = fmaf(s[f][e], kv[e], u);
+                    r = fmaf(s[f][e], qv[e], r);
+                }
+                u = group_sum<LPR>(u);
+                r = group_sum<LPR>(r);
+                const bool valid = row[f] < dv;
+                const float ev = (valid ? sv[i][row[f]] : 0.f) - a * u;
+                const float be = b * ev;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) s[f][e] = fmaf(a, s[f][e], be * kv[e]);
+                if (valid && part == 0) y[tok_row(i) * dv + row[f]] = from_f32<T>(fmaf(a, r, be * kq));
+            }
+        }
+#pragma unroll
+        for (int f = 0; f < ROWS_IN_FLIGHT; ++f)
+            if (row[f] < dv)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    store4(Sc + (size_t)row[f] * DK + 16 * part + 4 * c,
+                           make_float4(s[f][4 * c], s[f][4 * c + 1], s[f][4 * c + 2], s[f][4 * c + 3]));
+    }
+}
+
+}  // namespace gdn

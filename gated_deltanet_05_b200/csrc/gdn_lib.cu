@@ -12,6 +12,7 @@
 #include "gdn_chunk_sm100.cuh"
 #include "gdn_common.cuh"
 #include "gdn_decode.cuh"
+#include "gdn_featurize.cuh"
 #include "gdn_gate_norm.cuh"
 
 namespace {
@@ -316,6 +317,47 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
     return launch_status();
 }
 
+gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                             const float *alpha, const float *beta, float *S, int n_seq,
+                             int n_tokens, int H, int d_k, int d_v, float scale, void *y,
+                             void *stream)
+{
+    if (n_seq < 0 || H <= 0 || n_tokens < 1 || n_tokens > gdn::kDecodeMaxTokens)
+        return GDN_ERR_INVALID_ARG;
+    if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!pow2_in(d_k, 16, 128) || !pow2_in(d_v, 16, 128)) return GDN_ERR_UNSUPPORTED;
+    const int64_t n_chain = (int64_t)n_seq * H;
+    if (n_chain == 0) return GDN_OK;
+    if (n_chain > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !S || !y) return GDN_ERR_INVALID_ARG;
+    const size_t vec = in_dtype == GDN_F32 ? 16 : 8;
+    if (!aligned(q, vec) || !aligned(k, vec) || !aligned(S, 16) || !aligned(alpha, 4) ||
+        !aligned(beta, 4) || !aligned(v, 4) || !aligned(y, 4))
+        return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    const unsigned grid = (unsigned)n_chain;
+#define GDN_DECTOK_CASE(DK)                                                                        \
+    case DK:                                                                                       \
+        if (in_dtype == GDN_F32)                                                                   \
+            gdn::decode_tokens_kernel<DK, float><<<grid, gdn::kDecodeTokThreads, 0, st>>>(         \
+                (const float *)q, (const float *)k, (const float *)v, alpha, beta, S, n_tokens, H, \
+                d_v, scale, (float *)y);                                                           \
+        else                                                                                       \
+            gdn::decode_tokens_kernel<DK, __nv_bfloat16><<<grid, gdn::kDecodeTokThreads, 0, st>>>( \
+                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,      \
+                alpha, beta, S, n_tokens, H, d_v, scale, (__nv_bfloat16 *)y);                      \
+        break;
+    switch (d_k) {
+        GDN_DECTOK_CASE(16)
+        GDN_DECTOK_CASE(32)
+        GDN_DECTOK_CASE(64)
+        GDN_DECTOK_CASE(128)
+    default: return GDN_ERR_UNSUPPORTED;
+    }
+#undef GDN_DECTOK_CASE
+    return launch_status();
+}
+
 gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dtype z_dtype,
                          const float *w, int64_t n_rows, int d_v, float eps, void *o,
                          gdn_dtype o_dtype, void *stream)
@@ -363,6 +405,65 @@ gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dt
     }
 #undef GDN_GN_DV
 #undef GDN_GN
+    return launch_status();
+}
+
+gdn_status gdn_featurize(const void *xq, const void *xk, const void *xv, gdn_dtype dtype,
+                         const float *conv_q, const float *conv_k, const float *conv_v, int W,
+                         const float *beta_logit, const float *alpha_logit, const float *A,
+                         const float *b_alpha, const int32_t *cu_seqlens_dev,
+                         const int32_t *cu_seqlens_host, int n_seq, int64_t n_tok, int H, int d_k,
+                         int d_v, float eps, void *q, void *k, void *v, float *beta,
+                         float *log_alpha, void *stream)
+{
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (n_tok < 0 || n_seq < 1 || H < 1 || W < 1 || W > gdn::kFeatMaxWidth || !(eps >= 0.f))
+        return GDN_ERR_INVALID_ARG;
+    if (!pow2_in(d_k, 16, 128) || !pow2_in(d_v, 16, 128)) return GDN_ERR_UNSUPPORTED;
+    if (cu_seqlens_host) {
+        if (cu_seqlens_host[0] != 0 || cu_seqlens_host[n_seq] != n_tok) return GDN_ERR_INVALID_ARG;
+        for (int i = 0; i < n_seq; ++i)
+            if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return GDN_ERR_INVALID_ARG;
+    }
+    if (n_tok == 0) return GDN_OK;
+    const void *ptrs[] = {xq, xk, xv, conv_q, conv_k, conv_v, beta_logit, alpha_logit, A, b_alpha,
+                          cu_seqlens_dev, q, k, v, beta, log_alpha};
+    for (const void *p : ptrs)
+        if (!p) return GDN_ERR_INVALID_ARG;
+    for (const void *p : {xq, xk, xv, (const void *)q, (const void *)k, (const void *)v})
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    const int64_t n_runs = (n_tok + gdn::kFeatRun - 1) / gdn::kFeatRun;
+    const int warps_per_block = gdn::kFeatThreads / 32;
+    auto blocks_for = [&](int d, int n_streams, bool gates) -> unsigned {
+        const int rpw = 32 / (d / 4);
+        const int64_t n_hg = (H + rpw - 1) / rpw;
+        const int64_t tasks = n_streams * n_runs * n_hg + (gates ? n_runs : 0);
+        return (unsigned)((tasks + warps_per_block - 1) / warps_per_block);
+    };
+    using f32 = float;
+    using b16 = __nv_bfloat16;
+    // launch 1: q and k (L2-normalised); launch 2: v and the gates
+#define GDN_FT(T, D, L2, X0, X1, W0, W1, O0, O1, NS, GATES)                                       \
+    gdn::featurize_kernel<T, D, L2><<<blocks_for(D, NS, GATES), gdn::kFeatThreads, 0, st>>>(      \
+        (const T *)(X0), (const T *)(X1), W0, W1, (T *)(O0), (T *)(O1), NS, W, cu_seqlens_dev, n_seq, \
+        n_tok, H, eps, GATES ? beta_logit : nullptr, alpha_logit, A, b_alpha, beta, log_alpha)
+#define GDN_FT_D(T, d, L2, X0, X1, W0, W1, O0, O1, NS, GATES)                                     \
+    switch (d) {                                                                                 \
+    case 16: GDN_FT(T, 16, L2, X0, X1, W0, W1, O0, O1, NS, GATES); break;                        \
+    case 32: GDN_FT(T, 32, L2, X0, X1, W0, W1, O0, O1, NS, GATES); break;                        \
+    case 64: GDN_FT(T, 64, L2, X0, X1, W0, W1, O0, O1, NS, GATES); break;                        \
+    default: GDN_FT(T, 128, L2, X0, X1, W0, W1, O0, O1, NS, GATES); break;                       \
+    }
+    if (dtype == GDN_BF16) {
+        GDN_FT_D(b16, d_k, true, xq, xk, conv_q, conv_k, q, k, 2, false)
+        GDN_FT_D(b16, d_v, false, xv, xv, conv_v, conv_v, v, v, 1, true)
+    } else {
+        GDN_FT_D(f32, d_k, true, xq, xk, conv_q, conv_k, q, k, 2, false)
+        GDN_FT_D(f32, d_v, false, xv, xv, conv_v, conv_v, v, v, 1, true)
+    }
+#undef GDN_FT_D
+#undef GDN_FT
     return launch_status();
 }
 

@@ -165,6 +165,28 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
                            int d_k, int d_v, float scale, void *y, void *stream);
 
 /*
+ * gdn_decode_tokens -- n_tokens consecutive tokens for each of n_seq * H chains, in place,
+ * in one pass over the state (the multi-token decode of speculative decoding).
+ *
+ * Defines: the update of gdn_decode_step applied token after token (joezjh.github.io
+ * notes, "Gated DeltaNet 核心机制"); the result equals n_tokens calls of gdn_decode_step.
+ * The state is read and written once per call, so the HBM cost per token falls by
+ * n_tokens. Token i of sequence s is row (s * n_tokens + i) of the inputs:
+ *
+ *   q, k   [n_seq * n_tokens, H, d_k] in in_dtype;  v [n_seq * n_tokens, H, d_v] in in_dtype
+ *   alpha  [n_seq * n_tokens, H] fp32 in (0, 1];  beta [n_seq * n_tokens, H] fp32 in [0, 1]
+ *   S      [n_seq, H, d_v, d_k] fp32, read and overwritten with the state after the last token
+ *   y      [n_seq * n_tokens, H, d_v] out, in in_dtype
+ *   1 <= n_tokens <= 8; d_k, d_v each in {16, 32, 64, 128}
+ * The pages run decode with several tokens per step (pwwt.cn translation, Figure 6
+ * settings: next_n = 4) but give no kernel for it.
+ */
+gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                             const float *alpha, const float *beta, float *S, int n_seq,
+                             int n_tokens, int H, int d_k, int d_v, float scale, void *y,
+                             void *stream);
+
+/*
  * gdn_gate_norm -- the output epilogue o = sigmoid(z) * RMSNorm(y) * (1 + w).
  *
  * Defines: the output-gate equation of the joezjh.github.io notes ("GDN 参数化细节")
@@ -180,6 +202,41 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
 gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dtype z_dtype,
                          const float *w, int64_t n_rows, int d_v, float eps, void *o,
                          gdn_dtype o_dtype, void *stream);
+
+/*
+ * gdn_featurize -- the feature and gate step in front of the recurrence.
+ *
+ * Defines: the q/k/v and gate equations of the joezjh.github.io notes ("GDN 参数化细节")
+ * with the projections W x given as inputs, and the pwwt.cn translation (section 2.1.1,
+ * Figure 2): a short causal convolution of each projected stream, SiLU, then an L2 norm
+ * of q and k (not v) per (token, head) over d:
+ *   f_t = SiLU(sum_{j<W} conv[ch][j] * x_{t-(W-1)+j}),  x = 0 before the sequence start
+ *   q_t = f_t / sqrt(|f_t|^2 + eps) (likewise k_t);  v_t = f_t
+ *   beta_t = sigmoid(beta_logit_t);  log_alpha_t = -exp(A_h) * softplus(alpha_logit_t + b_alpha_h)
+ * The window never reaches into an earlier sequence of the packed batch.
+ *
+ *   xq, xk [n_tok, H, d_k], xv [n_tok, H, d_v] in dtype (projected streams)
+ *   conv_q, conv_k [H * d_k, W], conv_v [H * d_v, W] fp32 (tap j multiplies the row
+ *          W - 1 - j tokens back: the layout of a depthwise Conv1d padded by W - 1)
+ *   beta_logit, alpha_logit [n_tok, H] fp32;  A, b_alpha [H] fp32
+ *   cu_seqlens_dev [n_seq + 1] int32 on the device, read by the kernels;
+ *   cu_seqlens_host the same values on the host, or NULL (then unchecked here; tokens
+ *          that the device copy does not cover raise GDN_ERR_DEVICE_CHECK)
+ *   q, k [n_tok, H, d_k], v [n_tok, H, d_v] out, in dtype (the chunk_fwd inputs)
+ *   beta, log_alpha [n_tok, H] out, fp32 (the chunk_fwd gates)
+ *   d_k, d_v in {16, 32, 64, 128}; 1 <= W <= 4; eps >= 0 (1e-6; with eps = 0 an all-zero
+ *   feature row gives NaN)
+ * Outputs must not alias inputs. Two launches on `stream`, no synchronisation.
+ * The pages do not give the convolution width or eps; there is no counterpart of
+ * cu_seqlens on the pages (it delimits the packed sequences).
+ */
+gdn_status gdn_featurize(const void *xq, const void *xk, const void *xv, gdn_dtype dtype,
+                         const float *conv_q, const float *conv_k, const float *conv_v, int W,
+                         const float *beta_logit, const float *alpha_logit, const float *A,
+                         const float *b_alpha, const int32_t *cu_seqlens_dev,
+                         const int32_t *cu_seqlens_host, int n_seq, int64_t n_tok, int H, int d_k,
+                         int d_v, float eps, void *q, void *k, void *v, float *beta,
+                         float *log_alpha, void *stream);
 
 /* A static, human-readable name for a status code. */
 const char *gdn_status_string(gdn_status status);

@@ -120,6 +120,54 @@ def test_decode_and_gate_norm_reject_bad_arguments(L):
     assert gn(rows=0) == 0
 
 
+def test_decode_tokens_rejects_bad_arguments(L):
+    dt = lambda **kw: L.gdn_decode_tokens(kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 0), FAKE, FAKE,
+                                          kw.get("S", FAKE), kw.get("n", 4), kw.get("nt", 4),
+                                          kw.get("H", 2), kw.get("dk", 128), kw.get("dv", 128), 1.0,
+                                          FAKE, None)
+    assert dt(nt=0) == 1
+    assert dt(nt=9) == 1
+    assert dt(n=-1) == 1
+    assert dt(H=0) == 1
+    assert dt(dt=2) == 1
+    assert dt(dk=256) == 2
+    assert dt(dv=24) == 2
+    assert dt(q=None) == 1
+    assert dt(S=ctypes.c_void_p(0x10004)) == 1
+    assert dt(n=0) == 0
+
+
+def test_featurize_rejects_bad_arguments(L):
+    cu_ok = (ctypes.c_int32 * 3)(0, 5, 12)
+    cu_bad = (ctypes.c_int32 * 3)(0, 7, 5)           # decreasing
+    cu_short = (ctypes.c_int32 * 3)(0, 5, 11)        # does not reach n_tok
+
+    def ft(**kw):
+        cu = kw.get("cu", cu_ok)
+        return L.gdn_featurize(kw.get("xq", FAKE), FAKE, FAKE, kw.get("dt", 1), FAKE, FAKE, FAKE,
+                               kw.get("W", 4), FAKE, FAKE, FAKE, FAKE, FAKE,
+                               ctypes.cast(cu, ctypes.c_void_p) if cu is not None else None,
+                               kw.get("n_seq", 2), kw.get("n_tok", 12), kw.get("H", 2),
+                               kw.get("dk", 128), kw.get("dv", 128), kw.get("eps", 1e-6),
+                               kw.get("q", FAKE), FAKE, FAKE, FAKE, FAKE, None)
+    assert ft(dt=3) == 1
+    assert ft(W=0) == 1
+    assert ft(W=5) == 1
+    assert ft(H=0) == 1
+    assert ft(n_seq=0) == 1
+    assert ft(n_tok=-1) == 1
+    assert ft(eps=-1.0) == 1
+    assert ft(eps=float("nan")) == 1
+    assert ft(dk=256) == 2
+    assert ft(dv=48) == 2
+    assert ft(cu=cu_bad) == 1
+    assert ft(cu=cu_short) == 1
+    assert ft(xq=None) == 1
+    assert ft(q=None) == 1
+    assert ft(q=ctypes.c_void_p(0x10008)) == 1     # not 16-byte aligned
+    assert ft(n_tok=0, cu=(ctypes.c_int32 * 3)(0, 0, 0)) == 0
+
+
 def test_binding_has_no_cpu_fallback(monkeypatch):
     """Calls on CPU tensors raise instead of computing anything."""
     import torch

@@ -1,0 +1,110 @@
+"""GPU parity of the multi-token decode (gdn_decode_tokens) against the fp64 oracle.
+
+n tokens per chain and call are n steps of the recurrence started from the current state,
+so the oracle is the token-by-token recurrence over sequences of n tokens with S0 = the
+state. Bar: max|got - ref| / rms(ref) on every y and on the final state, fp32 <= 1e-4,
+bf16 inputs <= 2e-2 on the fp32 state; a bf16 y is held to one bf16 rounding of the exact
+value per element (|d| <= 2^-8 |ref| + 1e-4 rms(ref)). Cases: every d (16..128), d_k != d_v,
+1..8 tokens, odd head counts, a 400-token run of 100 calls of 4 tokens, and agreement with
+n calls of gdn_decode_step.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests.helpers import TOL, f64, rel_err
+
+gdn = pytest.importorskip("gated_deltanet_05_b200")
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+    yield
+    assert gdn.device_error() == "GDN_OK"
+
+
+def _tokens(n_seq, n, H, dk, dv, dtype, seed):
+    """Inputs of n decode steps: [n_seq, n, H, .] (steps drawn with the decode generator)."""
+    w = W.WORKLOADS["decode"]
+    steps = [W.make_decode_inputs(w, seed * 100 + i, n_seq=n_seq, H=H, d=dk) for i in range(n)]
+    vs = [W.make_decode_inputs(w, seed * 100 + 50 + i, n_seq=n_seq, H=H, d=dv)["v"] for i in range(n)]
+    cast = (lambda t: t.to(torch.bfloat16)) if dtype == "bf16" else (lambda t: t)
+    q = cast(torch.stack([s["q"] for s in steps], 1))
+    k = cast(torch.stack([s["k"] for s in steps], 1))
+    v = cast(torch.stack(vs, 1))
+    alpha = torch.stack([s["alpha"] for s in steps], 1)
+    beta = torch.stack([s["beta"] for s in steps], 1)
+    return q, k, v, alpha, beta
+
+
+def _oracle(q, k, v, alpha, beta, S_lib):
+    """y [n_seq, n, H, dv] and the final state (library layout) from the fp64 recurrence."""
+    n_seq, n, H, dk = q.shape
+    dv = v.shape[3]
+    flat = lambda t, d: t.reshape(n_seq * n, H, d)
+    cu = np.arange(0, n_seq * n + 1, n, dtype=np.int64)
+    la = np.log(f64(alpha).reshape(n_seq * n, H))
+    y, S_T, _ = oracle.recurrent(flat(q, dk), flat(k, dk), flat(v, dv), la, beta.reshape(n_seq * n, H),
+                                 cu, S0=oracle.state_from_lib(S_lib))
+    return y.reshape(n_seq, n, H, dv), oracle.state_to_lib(S_T)
+
+
+@pytest.mark.parametrize("n_seq,n,H,dk,dv,dtype", [
+    (3, 4, 2, 128, 128, "f32"), (2, 1, 3, 64, 64, "f32"), (5, 8, 1, 32, 32, "f32"),
+    (2, 3, 3, 16, 16, "f32"), (2, 5, 2, 32, 64, "f32"), (2, 2, 2, 128, 64, "f32"),
+    (4, 4, 2, 128, 128, "bf16"), (3, 7, 5, 64, 64, "bf16"),
+])
+def test_decode_tokens_parity(n_seq, n, H, dk, dv, dtype):
+    q, k, v, alpha, beta = _tokens(n_seq, n, H, dk, dv, dtype, seed=n_seq * 10 + n)
+    g = torch.Generator().manual_seed(n)
+    S0 = (torch.randn(n_seq, H, dv, dk, generator=g) * 0.05).float()
+    S = S0.cuda()
+    y = gdn.decode_tokens(q.cuda(), k.cuda(), v.cuda(), alpha.cuda(), beta.cuda(), S)
+    torch.cuda.synchronize()
+    y_ref, S_ref = _oracle(q, k, v, alpha, beta, S0.numpy().astype(np.float64))
+    tol = TOL[dtype]
+    if dtype == "bf16":
+        # y is returned in bf16: each element within one rounding of the exact value
+        rms = float(np.sqrt(np.mean(y_ref * y_ref)))
+        assert (np.abs(f64(y) - y_ref) <= 2.0 ** -8 * np.abs(y_ref) + 1e-4 * rms).all()
+    else:
+        assert rel_err(f64(y), y_ref) <= tol
+    assert rel_err(f64(S), S_ref) <= tol
+
+
+def test_decode_tokens_long_run():
+    """100 calls of 4 tokens (400 steps) from a zero state, fp32, against one oracle run."""
+    n_seq, n, H, d, calls = 4, 4, 2, 128, 100
+    q, k, v, alpha, beta = _tokens(n_seq, n * calls, H, d, d, "f32", seed=7)
+    S = torch.zeros(n_seq, H, d, d, device="cuda")
+    ys = []
+    for c in range(calls):
+        sl = slice(c * n, (c + 1) * n)
+        ys.append(gdn.decode_tokens(q[:, sl].contiguous().cuda(), k[:, sl].contiguous().cuda(),
+                                    v[:, sl].contiguous().cuda(), alpha[:, sl].contiguous().cuda(),
+                                    beta[:, sl].contiguous().cuda(), S).cpu())
+    y = torch.cat(ys, 1)
+    y_ref, S_ref = _oracle(q, k, v, alpha, beta, np.zeros((n_seq, H, d, d)))
+    assert rel_err(f64(y), y_ref) <= TOL["f32"]
+    assert rel_err(f64(S), S_ref) <= TOL["f32"]
+
+
+def test_decode_tokens_matches_single_steps():
+    n_seq, n, H, d = 8, 4, 4, 128
+    q, k, v, alpha, beta = _tokens(n_seq, n, H, d, d, "f32", seed=3)
+    S0 = torch.randn(n_seq, H, d, d) * 0.05
+    S_a, S_b = S0.cuda(), S0.cuda()
+    y_a = gdn.decode_tokens(q.cuda(), k.cuda(), v.cuda(), alpha.cuda(), beta.cuda(), S_a)
+    y_b = torch.stack([gdn.decode_step(q[:, i].contiguous().cuda(), k[:, i].contiguous().cuda(),
+                                       v[:, i].contiguous().cuda(), alpha[:, i].contiguous().cuda(),
+                                       beta[:, i].contiguous().cuda(), S_b) for i in range(n)], 1)
+    torch.cuda.synchronize()
+    assert rel_err(f64(y_a), f64(y_b)) <= 1e-5
+    assert rel_err(f64(S_a), f64(S_b)) <= 1e-5

@@ -18,6 +18,12 @@ benchmark workloads of this library:
   decode    fp32 state, 256 sequences, H=32, d=128, one token per step
 
 Draw order within one workload: q, k, v, beta logits, A, u, S0, z, w.
+
+The featurisation step in front of the recurrence takes the projected streams instead
+(make_featurize_inputs): xq, xk, xv ~ N(0, 1) in the workload dtype, depthwise
+convolution weights ~ N(0, 1/W) fp32 with W = 4 taps, beta and alpha logits ~ N(0, 1),
+A ~ U(A_range) per head and b_alpha ~ N(0, 0.25) per head; draw order xq, xk, xv,
+conv_q, conv_k, conv_v, beta logits, A, alpha logits, b_alpha.
 """
 from __future__ import annotations
 
@@ -27,7 +33,7 @@ import numpy as np
 import torch
 
 __all__ = [
-    "Workload", "WORKLOADS", "make_prefill_inputs", "make_decode_inputs",
+    "Workload", "WORKLOADS", "make_prefill_inputs", "make_decode_inputs", "make_featurize_inputs",
     "varlen_lengths", "to_f64",
 ]
 
@@ -146,6 +152,33 @@ def make_prefill_inputs(w: Workload, lengths=None, seed=None, with_gate: bool = 
         out["z"] = _normal(rng, (n_tok, H, dv), w.dtype)
         out["w_norm"] = torch.from_numpy((rng.standard_normal(dv) * 0.02).astype(np.float32))
     return out
+
+
+def make_featurize_inputs(w: Workload, lengths=None, seed=None, width: int = 4) -> dict:
+    """Projected streams and gate logits of one prefill workload, for the featurisation step.
+
+    xq, xk : [N_tok, H, d_k], xv : [N_tok, H, d_v] in w.dtype
+    conv_q, conv_k : [H*d_k, width], conv_v : [H*d_v, width] fp32
+    beta_logit, alpha_logit : [N_tok, H] fp32 ; A, b_alpha : [H] fp32 ; cu_seqlens int32
+    """
+    lengths = tuple(w.lengths if lengths is None else lengths)
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    n_tok = int(sum(lengths))
+    H, dk, dv = w.H, w.d_k, w.d_v
+    xq = _normal(rng, (n_tok, H, dk), w.dtype)
+    xk = _normal(rng, (n_tok, H, dk), w.dtype)
+    xv = _normal(rng, (n_tok, H, dv), w.dtype)
+    conv = [torch.from_numpy((rng.standard_normal((H * d, width)) / np.sqrt(width)).astype(np.float32))
+            for d in (dk, dk, dv)]
+    beta_logit = rng.standard_normal((n_tok, H)).astype(np.float32)
+    A = rng.uniform(w.A_range[0], w.A_range[1], size=(H,)).astype(np.float32)
+    alpha_logit = rng.standard_normal((n_tok, H)).astype(np.float32)
+    b_alpha = (rng.standard_normal(H) * 0.5).astype(np.float32)
+    return dict(xq=xq, xk=xk, xv=xv, conv_q=conv[0], conv_k=conv[1], conv_v=conv[2],
+                beta_logit=torch.from_numpy(beta_logit), alpha_logit=torch.from_numpy(alpha_logit),
+                A=torch.from_numpy(A), b_alpha=torch.from_numpy(b_alpha),
+                cu_seqlens=torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32),
+                H=H, d_k=dk, d_v=dv, dtype=w.dtype, lengths=lengths)
 
 
 def make_decode_inputs(w: Workload, step: int, n_seq=None, H=None, d=None) -> dict:
