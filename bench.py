@@ -547,7 +547,8 @@ def run_case(args):
     --case prefill:S,T,H   (bf16, d=128, chunk 64, fp32 y)
     --case decode:N        (N sequences x 32 heads, d=128, fp32 state)
     --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)
-    --case featurize:S,T,H (bf16, d=128, conv width 4)"""
+    --case featurize:S,T,H (bf16, d=128, conv width 4)
+    --case decode_tokens:N,T (N sequences x 32 heads, d=128, T tokens per call)"""
     import torch
 
     import gated_deltanet_05_b200 as gdn
@@ -569,6 +570,15 @@ def run_case(args):
         S = torch.zeros(n, 32, 128, 128, device="cuda")
         for _ in range(args.reps):
             gdn.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S)
+    elif kind == "decode_tokens":
+        n, nt = dims
+        w = W.WORKLOADS["decode"]
+        xs = [W.make_decode_inputs(w, i, n_seq=n) for i in range(nt)]
+        x = {key: torch.stack([xi[key] for xi in xs], 1).contiguous().cuda()
+             for key in ("q", "k", "v", "alpha", "beta")}
+        S = torch.zeros(n, 32, 128, 128, device="cuda")
+        for _ in range(args.reps):
+            gdn.decode_tokens(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S)
     elif kind == "gate_norm":
         (rows,) = dims
         g = torch.Generator().manual_seed(0)
