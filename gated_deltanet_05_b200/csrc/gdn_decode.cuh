@@ -109,7 +109,7 @@ decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
     constexpr int LPR = DK / 16;             // lanes per row, 16 elements each
     constexpr int RPW = 32 / LPR;            // rows per warp pass
     constexpr int WARPS = kDecodeTokThreads / 32;
-    constexpr int ROWS_IN_FLIGHT = 2;
+    constexpr int ROWS_IN_FLIGHT = 4;        // 128 rows of d_k = 128 in one round
     __shared__ float4 sk[kDecodeMaxTokens][DK / 4], sq[kDecodeMaxTokens][DK / 4];
     __shared__ float sv[kDecodeMaxTokens][128];
     __shared__ float sa[kDecodeMaxTokens], sb[kDecodeMaxTokens], skq[kDecodeMaxTokens];

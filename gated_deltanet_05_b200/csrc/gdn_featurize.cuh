@@ -25,7 +25,7 @@ namespace gdn {
 
 constexpr int kFeatThreads = 128;
 constexpr int kFeatRun = 32;      // tokens per warp task
-constexpr int kFeatBatch = 8;     // rows loaded ahead
+constexpr int kFeatBatch = 4;     // rows loaded ahead
 constexpr int kFeatMaxWidth = 4;  // convolution taps
 
 // SiLU with the fast exponential and division intrinsics (relative error ~1e-6, well inside
@@ -54,7 +54,7 @@ __device__ __forceinline__ void raw_to_f32(const uint2 &r, float (&x)[4])
 // One launch covers n_streams streams of width D (q and k with L2 = true; v with
 // L2 = false) and, when beta_logit is given, the gates.
 template <typename T, int D, bool L2>
-__global__ void __launch_bounds__(kFeatThreads, 4)
+__global__ void __launch_bounds__(kFeatThreads, 6)
 featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float *__restrict__ w0,
                  const float *__restrict__ w1, T *__restrict__ o0, T *__restrict__ o1, int n_streams,
                  int W, const int32_t *__restrict__ cu, int n_seq, int64_t n_tok, int H, float eps,
