@@ -3,7 +3,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = chunked prefill (gdn_chunk_fwd) + the sigmoid-gate zero-centred RMSNorm
-epilogue (gdn_gate_norm) over one batch of the prefill workload: 4 sequences x 4096
+epilogue (gdn_gate_norm) over one batch of the prefill workload; the same step as one
+launch with the epilogue fused into the prefill's output stage (gdn_chunk_fwd_gated) is
+timed beside it under "fused_step". The workload: 4 sequences x 4096
 tokens, H = 16, d_k = d_v = 128, chunk 64, bf16 q/k/v, fp32 state. Inputs are seeded
 synthetic draws (workloads/), resident in HBM before the timed region; q, k, v and z
 (256 MiB) exceed the 126 MB L2, so no flush is needed between steps.
@@ -51,10 +53,11 @@ def flops_per_token_head(chunk: int, d: int) -> float:
     return 10.0 * chunk * d + 6.0 * d * d + chunk * chunk / 3.0
 
 
-def prefill_bytes_per_token_head(in_elem: int, y_elem: int, d: int) -> float:
-    """Minimal HBM bytes per (token, head): read q, k, v (3 d in_elem), write y (d y_elem),
-    read log_alpha and beta (8 bytes)."""
-    return 3 * in_elem * d + y_elem * d + 8.0
+def prefill_bytes_per_token_head(in_elem: int, y_elem: int, d: int, z_elem: int = 0) -> float:
+    """Minimal HBM bytes per (token, head): read q, k, v (3 d in_elem), write y or o
+    (d y_elem), read z when the gate-norm is fused (d z_elem), read log_alpha and beta
+    (8 bytes)."""
+    return 3 * in_elem * d + y_elem * d + z_elem * d + 8.0
 
 
 def load_peaks():
@@ -264,6 +267,7 @@ def run_ours(args, rank, world, local, pg):
     stream = torch.cuda.current_stream(device)
 
     def step(ev=None):
+        # the whole hot path: chunked prefill (fp32 y), then the gate-norm epilogue
         if ev is not None:
             ev[0].record(stream)
         gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
@@ -274,6 +278,13 @@ def run_ours(args, rank, world, local, pg):
         gdn.gate_norm(y, dev["z"], dev["w_norm"], out=o)
         if ev is not None:
             ev[2].record(stream)
+
+    def fused_step(ev):
+        ev[0].record(stream)
+        gdn.chunk_fwd_gated(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                            dev["cu_seqlens"], dev["z"], dev["w_norm"], chunk=C,
+                            cu_seqlens_host=cu_host, out=o, final_state=True)
+        ev[1].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -301,6 +312,12 @@ def run_ours(args, rank, world, local, pg):
     elapsed_ms = max_over_ranks(pg, elapsed_ms, device)
     chunk_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     gn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # the same step as one launch with the gate-norm fused into the prefill's output stage
+    fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(20)]
+    for e in fevs:
+        fused_step(e)
+    torch.cuda.synchronize(device)
+    fused_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in fevs)
     ms_per_step = elapsed_ms / args.steps
     tokens_per_step = n_tok * world
     value = tokens_per_step / (ms_per_step * 1e-3)
@@ -333,6 +350,9 @@ def run_ours(args, rank, world, local, pg):
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gn_bytes / (gn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "bytes_per_launch": gn_bytes}
+    fused = {"ms_per_step": fused_ms,
+             "note": "the same step as one gdn_chunk_fwd_gated launch (gate-norm in the prefill's "
+                     "output stage), 20 steps"}
 
     decode = None if args.no_decode else bench_decode(args, device, peaks, peak_kind, pg)
     featurize = bench_featurize(args, device, peaks, peak_kind, pg, rank)
@@ -349,6 +369,7 @@ def run_ours(args, rank, world, local, pg):
                    "l2": "no flush: q, k, v, z are 256 MiB per step, above the 126 MB L2"},
         "roofline": roofline,
         "gate_norm": gate_norm_obj,
+        "fused_step": fused,
         "decode": decode,
         "featurize": featurize,
         "e2e": e2e,
@@ -545,6 +566,7 @@ def cpu_baseline(inp, H, min_seconds=10.0, max_reps=12):
 def run_case(args):
     """A few launches of one kernel on a named shape, nothing else (for ncu captures):
     --case prefill:S,T,H   (bf16, d=128, chunk 64, fp32 y)
+    --case prefill_gated:S,T,H (the same with the fused gate-norm, bf16 z and o)
     --case decode:N        (N sequences x 32 heads, d=128, fp32 state)
     --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)
     --case featurize:S,T,H (bf16, d=128, conv width 4)
@@ -564,6 +586,14 @@ def run_case(args):
         for _ in range(args.reps):
             gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
                           cu_seqlens_host=inp["cu_seqlens"])
+    elif kind == "prefill_gated":
+        n_seq, T, H = dims
+        w = W.Workload("case", "bf16", (T,) * n_seq, H, 128, 128, 64, seed=1)
+        inp = W.make_prefill_inputs(w)
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        for _ in range(args.reps):
+            gdn.chunk_fwd_gated(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
+                                d["z"], d["w_norm"], cu_seqlens_host=inp["cu_seqlens"])
     elif kind == "decode":
         (n,) = dims
         x = {k: v.cuda() for k, v in W.make_decode_inputs(W.WORKLOADS["decode"], 0, n_seq=n).items()}

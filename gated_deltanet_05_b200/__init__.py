@@ -6,6 +6,7 @@ stream. There is no CPU path: if the shared library is missing or fails to load,
 importing works but every call raises RuntimeError.
 
     y, S_T = chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64)
+    o, S_T = chunk_fwd_gated(q, k, v, log_alpha, beta, cu_seqlens, z, w)   # fused gate-norm
     y = decode_step(q, k, v, alpha, beta, S)          # S updated in place
     y = decode_tokens(q, k, v, alpha, beta, S)        # [n_seq, n, H, d]: n tokens, one pass
     o = gate_norm(y, z, w, eps=1e-6)
@@ -21,7 +22,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "selftest_bounded_wait", "decode_step", "decode_tokens", "gate_norm", "featurize",
+__all__ = ["chunk_fwd", "chunk_fwd_gated", "chunk_fwd_noalloc", "selftest_bounded_wait", "decode_step", "decode_tokens", "gate_norm", "featurize",
            "device_error", "lib", "LIB_PATH",
            "GdnError", "EXPORTED_SYMBOLS", "STATUS"]
 
@@ -31,7 +32,8 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
           4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_DEVICE_CHECK"}
 GDN_F32, GDN_BF16 = 0, 1
 
-EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc",
+EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_fwd_gated",
+                    "gdn_chunk_fwd_noalloc",
                     "gdn_selftest_bounded_wait", "gdn_decode_step", "gdn_decode_tokens",
                     "gdn_gate_norm", "gdn_featurize", "gdn_status_string", "gdn_device_error",
                     "gdn_version")
@@ -65,6 +67,9 @@ def lib():
         L.gdn_chunk_fwd.restype = i32
         L.gdn_chunk_fwd.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                     f32, vp, i32, vp, vp, ctypes.c_size_t, vp]
+        L.gdn_chunk_fwd_gated.restype = i32
+        L.gdn_chunk_fwd_gated.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                          f32, vp, vp, f32, vp, i32, vp, vp, ctypes.c_size_t, vp]
         L.gdn_chunk_fwd_noalloc.restype = i32
         L.gdn_chunk_fwd_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                             i32, f32, vp, i32, vp, vp]
@@ -187,6 +192,31 @@ def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0
                          _ptr(ws), ws_bytes, _stream(q.device))
     _check("gdn_chunk_fwd", rc)
     return y, S_T
+
+
+def chunk_fwd_gated(q, k, v, log_alpha, beta, cu_seqlens, z, w, eps=1e-6, S0=None, chunk=64,
+                    scale=1.0, cu_seqlens_host=None, out=None, final_state=True,
+                    o_dtype=torch.bfloat16, state_out=None):
+    """chunk_fwd with the output epilogue fused in: returns (o, S_T or None), where
+    o = sigmoid(z) * y / sqrt(mean(y^2) + eps) * (1 + w) per (token, head) and y is the
+    chunk_fwd output (never written). Tensor-core path only: bf16 q, k, v and z, d = 128,
+    chunk 64 (other shapes raise GdnError GDN_ERR_UNSUPPORTED). w [d_v] fp32."""
+    _cuda(z, "z")
+    _cuda(w, "w")
+    if z.dtype != torch.bfloat16 or z.shape != v.shape:
+        raise TypeError("z must be bfloat16 with v's shape")
+    if w.dtype != torch.float32 or w.numel() != v.shape[-1]:
+        raise TypeError("w must be float32 [d_v]")
+    args, o, S_T, cu_h = _chunk_setup(q, k, v, log_alpha, beta, cu_seqlens, S0, cu_seqlens_host,
+                                      out, final_state, state_out, o_dtype)
+    L = lib()
+    n_seq, H, dk, dv = args[9], args[10], args[11], args[12]
+    ws_bytes = L.gdn_chunk_fwd_workspace_bytes(n_seq, q.shape[0], H, dk, dv, chunk)
+    ws = _workspace(q.device, ws_bytes)
+    rc = L.gdn_chunk_fwd_gated(*args, int(chunk), float(scale), _ptr(z), _ptr(w), float(eps), _ptr(o),
+                               _dtype_code(o), _ptr(S_T), _ptr(ws), ws_bytes, _stream(q.device))
+    _check("gdn_chunk_fwd_gated", rc)
+    return o, S_T
 
 
 def chunk_fwd_noalloc(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0,

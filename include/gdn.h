@@ -146,6 +146,29 @@ gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gd
 gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *stream);
 
 /*
+ * gdn_chunk_fwd_gated -- gdn_chunk_fwd with the output epilogue fused into its y stage:
+ * o = sigmoid(z) * RMSNorm(y) * (1 + w) per (token, head), as gdn_gate_norm defines it,
+ * written instead of y (y itself never reaches memory).
+ *
+ * Defines: the chunked prefill of gdn_chunk_fwd followed by the output-gate equation of
+ * the joezjh.github.io notes ("GDN 参数化细节") with the zero-centred RMSNorm of the pwwt.cn
+ * translation (section 2.1.1); the same arguments as gdn_chunk_fwd, plus
+ *   z      [n_tok, H, d_v] bf16 (the projected gate logits)
+ *   w      [d_v] fp32 (stored zero-centred weight; the scale is 1 + w);  eps >= 0 (1e-6)
+ *   o      [n_tok, H, d_v] out, o_dtype (GDN_F32 or GDN_BF16), in place of y
+ * Only the tensor-core path: in_dtype GDN_BF16, d_k = d_v = 128, chunk = 64; anything else
+ * returns GDN_ERR_UNSUPPORTED (call gdn_chunk_fwd then gdn_gate_norm). The workspace is
+ * that of gdn_chunk_fwd. The result equals gdn_chunk_fwd + gdn_gate_norm up to fp32
+ * rounding order.
+ */
+gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                               const float *log_alpha, const float *beta, const float *S0,
+                               const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                               int n_seq, int H, int d_k, int d_v, int chunk, float scale,
+                               const void *z, const float *w, float eps, void *o, gdn_dtype o_dtype,
+                               float *S_T, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdn_decode_step -- one token for each of n_seq * H independent chains, in place.
  *
  * Defines: the same four-line update (joezjh.github.io notes, "Gated DeltaNet 核心机制")

@@ -120,6 +120,32 @@ def test_decode_and_gate_norm_reject_bad_arguments(L):
     assert gn(rows=0) == 0
 
 
+def test_chunk_fwd_gated_rejects_bad_arguments(L):
+    cu = (ctypes.c_int32 * 3)(0, 64, 100)
+    cu_bad = (ctypes.c_int32 * 3)(0, 64, 10)
+
+    def g(**kw):
+        c = kw.get("cu", cu)
+        return L.gdn_chunk_fwd_gated(FAKE, FAKE, FAKE, kw.get("dt", 1), FAKE, FAKE, None, FAKE,
+                                     ctypes.cast(c, ctypes.c_void_p), kw.get("n_seq", 2), kw.get("H", 2),
+                                     kw.get("dk", 128), kw.get("dv", 128), kw.get("chunk", 64), 1.0,
+                                     kw.get("z", FAKE), kw.get("w", FAKE), kw.get("eps", 1e-6),
+                                     kw.get("o", FAKE), kw.get("odt", 1), None, FAKE, 1 << 24, None)
+    assert g(dt=0) == 2            # fp32 inputs: the fused epilogue is tensor-core only
+    assert g(dk=64) == 2
+    assert g(chunk=32) == 2
+    assert g(dt=4) == 1
+    assert g(odt=3) == 1
+    assert g(eps=-1.0) == 1
+    assert g(H=0) == 1
+    assert g(cu=cu_bad) == 1
+    assert g(z=None) == 1
+    assert g(w=None) == 1
+    assert g(o=None) == 1
+    assert g(o=ctypes.c_void_p(0x10008)) == 1
+    assert g(n_seq=0) == 0
+
+
 def test_decode_tokens_rejects_bad_arguments(L):
     dt = lambda **kw: L.gdn_decode_tokens(kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 0), FAKE, FAKE,
                                           kw.get("S", FAKE), kw.get("n", 4), kw.get("nt", 4),
