@@ -16,7 +16,6 @@
 // so several 512-byte rows per warp are in flight. One CTA of 8 warps owns a chain.
 #pragma once
 #include "gdn_common.cuh"
-#include "sm100_ptx.cuh"
 
 namespace gdn {
 
@@ -199,206 +198,6 @@ decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
                 for (int c = 0; c < 4; ++c)
                     store4(Sc + (size_t)row[f] * DK + 16 * part + 4 * c,
                            make_float4(s[f][4 * c], s[f][4 * c + 1], s[f][4 * c + 2], s[f][4 * c + 3]));
-    }
-}
-
-}  // namespace gdn
-
-namespace gdn {
-
-// ---------------------------------------------------------------- several tokens, state streamed
-//
-// The same computation as decode_tokens_kernel for d_k = d_v = 128, with the state streamed
-// through shared memory: a persistent CTA per SM walks chains blockIdx.x, + gridDim.x, ...
-// and keeps two chain buffers. While it computes chain c from one buffer, the bulk copy of
-// the next chain's 64 KB state and of its tokens' q, k, v rows fills the other, and the
-// bulk store of chain c's updated state drains behind it. The loads, the arithmetic and
-// the stores of different chains overlap, so the kernel can run at the rate of HBM instead
-// of the latency of one warp's loads. Every wait is bounded (~1 s); a timeout records
-// kErrTimeout and every thread leaves together.
-constexpr int kDecStreamThreads = 512;
-constexpr int kDecStreamD = 128;
-constexpr uint32_t kDecStateBytes = kDecStreamD * kDecStreamD * 4;            // 64 KB
-
-template <typename T> struct DecStreamLayout {
-    static constexpr uint32_t ROW = kDecStreamD * sizeof(T);                      // one q/k/v row
-    static constexpr uint32_t TOK = 3 * kDecodeMaxTokens * ROW;                   // q | k | v rows
-    static constexpr uint32_t BUF = kDecStateBytes + TOK + 2 * kDecodeMaxTokens * 4;   // + alpha, beta
-    static constexpr uint32_t OFF_BAR = 2 * BUF;
-    static constexpr uint32_t SMEM = OFF_BAR + 64 + 2 * kDecodeMaxTokens * 4;    // bars, abort, k.q
-};
-
-template <typename T>
-__device__ __forceinline__ void load16(const T *p, float (&x)[16]);
-template <>
-__device__ __forceinline__ void load16<float>(const float *p, float (&x)[16])
-{
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const float4 f = *reinterpret_cast<const float4 *>(p + 4 * c);
-        x[4 * c] = f.x; x[4 * c + 1] = f.y; x[4 * c + 2] = f.z; x[4 * c + 3] = f.w;
-    }
-}
-template <>
-__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[16])
-{
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        const uint4 r = *reinterpret_cast<const uint4 *>(p + 8 * c);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
-            x[8 * c + 2 * i] = f.x;
-            x[8 * c + 2 * i + 1] = f.y;
-        }
-    }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kDecStreamThreads, 1)
-decode_tokens_stream_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                            const float *__restrict__ alpha, const float *__restrict__ beta,
-                            float *__restrict__ S, int n, int H, int n_chain, float scale,
-                            T *__restrict__ y)
-{
-    using L = DecStreamLayout<T>;
-    constexpr int D = kDecStreamD;
-    constexpr int LPR = D / 16;                 // 8 lanes per row, 16 elements each
-    constexpr int RPW = 32 / LPR;               // 4 rows per warp pass
-    constexpr int WARPS = kDecStreamThreads / 32;
-    constexpr int RIF = D / (WARPS * RPW);      // 2 passes cover the 128 rows
-    extern __shared__ __align__(128) uint8_t dsm[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + L::OFF_BAR);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(dsm + L::OFF_BAR + 16);
-    float *skq = reinterpret_cast<float *>(dsm + L::OFF_BAR + 64);   // [2][kDecodeMaxTokens]
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int part = lane % LPR, sub = lane / LPR;
-
-    auto buf = [&](int b) -> uint8_t * { return dsm + (size_t)b * L::BUF; };
-    auto tok_row = [&](int chain, int i) -> size_t { return ((size_t)(chain / H) * n + i) * H + chain % H; };
-    // one elected thread: the state and the tokens' rows of `chain` into buffer b
-    auto issue_loads = [&](int chain, int b) {
-        uint8_t *B = buf(b);
-        sm100::mbar_arrive_expect_tx(&full[b], kDecStateBytes + 3u * n * L::ROW);
-        sm100::bulk_load_g2s(B, S + (size_t)chain * D * D, kDecStateBytes, &full[b]);
-        for (int i = 0; i < n; ++i) {
-            const size_t r = tok_row(chain, i);
-            sm100::bulk_load_g2s(B + kDecStateBytes + (0 * kDecodeMaxTokens + i) * L::ROW, q + r * D, L::ROW, &full[b]);
-            sm100::bulk_load_g2s(B + kDecStateBytes + (1 * kDecodeMaxTokens + i) * L::ROW, k + r * D, L::ROW, &full[b]);
-            sm100::bulk_load_g2s(B + kDecStateBytes + (2 * kDecodeMaxTokens + i) * L::ROW, v + r * D, L::ROW, &full[b]);
-        }
-    };
-    float *gates0 = reinterpret_cast<float *>(buf(0) + kDecStateBytes + L::TOK);
-    float *gates1 = reinterpret_cast<float *>(buf(1) + kDecStateBytes + L::TOK);
-
-    int chain = blockIdx.x;
-    if (tid == 0) {
-        sm100::mbar_init(&full[0], 1);
-        sm100::mbar_init(&full[1], 1);
-        *abort_flag = 0;
-        sm100::fence_mbarrier_init();
-    }
-    // alpha, beta of the first chain (plain loads; later chains are prefetched)
-    if (chain < n_chain && tid < 2 * n)
-        gates0[(tid < n ? 0 : kDecodeMaxTokens) + tid % n] = (tid < n ? alpha : beta)[tok_row(chain, tid % n)];
-    __syncthreads();
-    if (tid == 0 && chain < n_chain) issue_loads(chain, 0);
-
-    int it = 0;
-    bool next_in_flight = false;                 // a load into the other buffer not yet waited for
-    for (; chain < n_chain; ++it, chain += gridDim.x) {
-        const int b = it & 1;
-        const int next = chain + gridDim.x;
-        next_in_flight = next < n_chain;
-        uint8_t *B = buf(b);
-        float *gates = b ? gates1 : gates0;
-        float *gates_next = b ? gates0 : gates1;
-        // the other buffer: its state has been stored (read by the copy engine) -> refill
-        if (tid == 0 && next < n_chain) {
-            sm100::bulk_wait_read();
-            issue_loads(next, b ^ 1);
-        }
-        float g_next = 0.f;
-        if (next < n_chain && tid < 2 * n)
-            g_next = (tid < n ? alpha : beta)[tok_row(next, tid % n)];
-        bool ok = sm100::mbar_test(&full[b], (uint32_t)(it >> 1) & 1u) ||
-                  sm100::mbar_wait_bounded(&full[b], (uint32_t)(it >> 1) & 1u, abort_flag, 2000000000LL);
-        if (__syncthreads_or(!ok)) break;
-        const T *qs = reinterpret_cast<const T *>(B + kDecStateBytes);
-        const T *ks = qs + kDecodeMaxTokens * D;
-        const T *vs = ks + kDecodeMaxTokens * D;
-        float *St = reinterpret_cast<float *>(B);
-        float *kq = skq + b * kDecodeMaxTokens;
-        if (warp < n) {                          // k_i . (scale q_i), one warp per token
-            float a4[4], c4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                a4[e] = to_f32(ks[warp * D + 4 * lane + e]);
-                c4[e] = to_f32(qs[warp * D + 4 * lane + e]);
-            }
-            float acc = a4[0] * c4[0] + a4[1] * c4[1] + a4[2] * c4[2] + a4[3] * c4[3];
-            acc = group_sum<32>(acc) * scale;
-            if (lane == 0) kq[warp] = acc;
-        }
-        __syncthreads();
-        float s[RIF][16];
-        int row[RIF];
-#pragma unroll
-        for (int f = 0; f < RIF; ++f) {
-            row[f] = (f * WARPS + warp) * RPW + sub;
-            const float *src = St + row[f] * D + 16 * part;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float4 x = *reinterpret_cast<const float4 *>(src + 4 * c);
-                s[f][4 * c] = x.x; s[f][4 * c + 1] = x.y; s[f][4 * c + 2] = x.z; s[f][4 * c + 3] = x.w;
-            }
-        }
-#pragma unroll 1
-        for (int i = 0; i < n; ++i) {
-            float kv[16], qv[16];
-            load16<T>(ks + i * D + 16 * part, kv);
-            load16<T>(qs + i * D + 16 * part, qv);
-            const float a = gates[i], bb = gates[kDecodeMaxTokens + i], kqi = kq[i];
-            const size_t yrow = tok_row(chain, i) * D;
-#pragma unroll
-            for (int f = 0; f < RIF; ++f) {
-                float u = 0.f, r = 0.f;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    u = fmaf(s[f][e], kv[e], u);
-                    r = fmaf(s[f][e], qv[e], r);
-                }
-                u = group_sum<LPR>(u);
-                r = group_sum<LPR>(r) * scale;
-                const float ev = to_f32(vs[i * D + row[f]]) - a * u;
-                const float be = bb * ev;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) s[f][e] = fmaf(a, s[f][e], be * kv[e]);
-                if (part == 0) y[yrow + row[f]] = from_f32<T>(fmaf(a, r, be * kqi));
-            }
-        }
-#pragma unroll
-        for (int f = 0; f < RIF; ++f) {
-            float *dst = St + row[f] * D + 16 * part;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<float4 *>(dst + 4 * c) =
-                    make_float4(s[f][4 * c], s[f][4 * c + 1], s[f][4 * c + 2], s[f][4 * c + 3]);
-        }
-        sm100::fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            sm100::bulk_store_s2g(S + (size_t)chain * D * D, St, kDecStateBytes);
-            sm100::bulk_commit();
-        }
-        if (next < n_chain && tid < 2 * n) gates_next[(tid < n ? 0 : kDecodeMaxTokens) + tid % n] = g_next;
-    }
-    if (tid == 0) {
-        // after a timeout, the copy into the other buffer lands before the CTA exits
-        if (chain < n_chain && next_in_flight)
-            sm100::mbar_wait_drain(&full[(it & 1) ^ 1], (uint32_t)((it + 1) >> 1) & 1u, 2000000000LL);
-        sm100::bulk_wait_all();               // the last stores complete before the CTA exits
     }
 }
 

@@ -377,27 +377,6 @@ gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dt
         !aligned(beta, 4) || !aligned(v, 4) || !aligned(y, 4))
         return GDN_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
-    // d = 128 with 16-byte aligned rows: persistent CTAs stream the state through shared memory
-    if (d_k == 128 && d_v == 128 && aligned(q, 16) && aligned(k, 16) && aligned(v, 16)) {
-        const int n_sm = device_sm_count();
-        if (n_sm <= 0) return GDN_ERR_CUDA;
-        const unsigned grid = (unsigned)(n_chain < n_sm ? n_chain : n_sm);
-#define GDN_DECSTREAM(T)                                                                           \
-    {                                                                                              \
-        const int smem = (int)gdn::DecStreamLayout<T>::SMEM;                                       \
-        auto kern = gdn::decode_tokens_stream_kernel<T>;                                           \
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
-            return GDN_ERR_CUDA;                                                                   \
-        kern<<<grid, gdn::kDecStreamThreads, smem, st>>>((const T *)q, (const T *)k, (const T *)v, alpha, \
-                                                         beta, S, n_tokens, H, (int)n_chain, scale, (T *)y); \
-    }
-        if (in_dtype == GDN_F32)
-            GDN_DECSTREAM(float)
-        else
-            GDN_DECSTREAM(__nv_bfloat16)
-#undef GDN_DECSTREAM
-        return launch_status();
-    }
     const unsigned grid = (unsigned)n_chain;
 #define GDN_DECTOK_CASE(DK)                                                                        \
     case DK:                                                                                       \

@@ -5,9 +5,8 @@ so the oracle is the token-by-token recurrence over sequences of n tokens with S
 state. Bar: max|got - ref| / rms(ref) on every y and on the final state, fp32 <= 1e-4,
 bf16 inputs <= 2e-2 on the fp32 state; a bf16 y is held to one bf16 rounding of the exact
 value per element (|d| <= 2^-8 |ref| + 1e-4 rms(ref)). Cases: every d (16..128), d_k != d_v,
-1..8 tokens, odd head counts, more chains than SMs (the d = 128 kernel's persistent CTAs
-cycle their two buffers), a 400-token run of 100 calls of 4 tokens, and agreement with n
-calls of gdn_decode_step.
+1..8 tokens, odd head counts, more chains than SMs, a 400-token run of 100 calls of 4
+tokens, and agreement with n calls of gdn_decode_step.
 """
 import numpy as np
 import pytest
@@ -61,8 +60,7 @@ def _oracle(q, k, v, alpha, beta, S_lib):
     (3, 4, 2, 128, 128, "f32"), (2, 1, 3, 64, 64, "f32"), (5, 8, 1, 32, 32, "f32"),
     (2, 3, 3, 16, 16, "f32"), (2, 5, 2, 32, 64, "f32"), (2, 2, 2, 128, 64, "f32"),
     (4, 4, 2, 128, 128, "bf16"), (3, 7, 5, 64, 64, "bf16"),
-    # more chains than SMs: each persistent CTA of the d = 128 kernel walks several chains
-    # through both of its shared-memory buffers
+    # more chains than SMs
     (40, 4, 8, 128, 128, "f32"), (30, 3, 10, 128, 128, "bf16"), (97, 8, 5, 128, 128, "f32"),
 ])
 def test_decode_tokens_parity(n_seq, n, H, dk, dv, dtype):
