@@ -11,7 +11,9 @@ Parity status: every function here is pinned by tests/test_oracle_pins.py (the
 equivalent update form, brute-force matrix products, invariants, closed forms and
 a hand-worked example) and, for the featurisation, tests/test_oracle_featurize.py
 (a library convolution, the impulse response, sequence isolation, unit norms and the
-gates' closed forms).
+gates' closed forms) and, for the gradients, tests/test_oracle_backward.py (central finite
+differences of the forward oracle, torch autograd of an independent fp64 restatement,
+and closed forms with the gates switched off).
 """
 from __future__ import annotations
 
@@ -52,6 +54,9 @@ def _configure(lib):
     lib.gdn_oracle_gate_norm.restype = ctypes.c_int
     lib.gdn_oracle_gate_norm.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int,
                                          ctypes.c_double, _dp]
+    lib.gdn_oracle_backward.restype = ctypes.c_int
+    lib.gdn_oracle_backward.argtypes = ([_dp] * 6 + [_i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_double] + [_dp] * 8)
     lib.gdn_oracle_featurize.restype = ctypes.c_int
     lib.gdn_oracle_featurize.argtypes = ([_dp] * 6 + [ctypes.c_int] + [_dp] * 4 +
                                          [_i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -179,3 +184,26 @@ def featurize(xq, xk, xv, conv_q, conv_k, conv_v, beta_logit, alpha_logit, A, b_
                                     _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_alpha)) < 0:
         raise ValueError("gdn_oracle_featurize: bad argument")
     return q, k, v, beta, log_alpha
+
+
+def backward(q, k, v, log_alpha, beta, cu_seqlens, dy, S0=None, dS_T=None, scale=1.0):
+    """Gradients of L = sum_t <dy_t, y_t> + <dS_T, S_T> for the token recurrence, in fp64.
+
+    Shapes as recurrent(); dy [N, H, dv]; dS_T, S0 [n_seq, H, dk, dv] (pages' orientation)
+    or None. Returns (dq, dk, dv, dlog_alpha, dbeta, dS0)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, b, dy = _f64(log_alpha), _f64(beta), _f64(dy)
+    S0, dS_T = _f64(S0), _f64(dS_T)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens if not hasattr(cu_seqlens, "numpy")
+                                         else cu_seqlens.numpy(), dtype=np.int64))
+    n_seq = cu.shape[0] - 1
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    assert dy.shape == (N, H, dv) and int(cu[-1]) == N
+    out = [np.zeros((N, H, dk)), np.zeros((N, H, dk)), np.zeros((N, H, dv)), np.zeros((N, H)),
+           np.zeros((N, H)), np.zeros((n_seq, H, dk, dv))]
+    if _load().gdn_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(S0),
+                                   cu.ctypes.data_as(_i64p), n_seq, H, dk, dv, float(scale),
+                                   _ptr(dy), _ptr(dS_T), *[_ptr(o) for o in out]) < 0:
+        raise ValueError("gdn_oracle_backward: bad argument")
+    return tuple(out)

@@ -342,3 +342,166 @@ int gdn_oracle_featurize(const double *xq, const double *xk, const double *xv, c
         }
     return 1;
 }
+
+/* ---------------------------------------------------------------- backward */
+
+/*
+ * Gradients of the token recurrence above (the reverse-mode adjoint of its four lines,
+ * taken step by step in reverse order). Given dy_t = dL/dy_t for every token and
+ * dS_T = dL/dS_T for the final state of every sequence (NULL: zero), with G = dL/dS_t
+ * carried backwards from G = dS_T:
+ *
+ *   y_t = S_t^T (scale q_t):       G += scale q_t dy_t^T;   dq_t = scale S_t dy_t
+ *   S_t = S~_t + beta_t k_t e_t^T: dbeta_t = k_t^T G e_t;   dk_t = beta_t G e_t;
+ *                                  de_t = beta_t G^T k_t;   G~ = G
+ *   e_t = v_t - S~_t^T k_t:        dv_t = de_t;   G~ -= k_t de_t^T;   dk_t -= S~_t de_t
+ *   S~_t = alpha_t S_{t-1}:        dalpha_t = <G~, S_{t-1}>;   G = alpha_t G~
+ *
+ * and dlog_alpha_t = alpha_t dalpha_t, dS0 = G after the first token. The states S_t are
+ * recomputed forward from a copy kept every kCkpt tokens (the same operations in the same
+ * order as the forward pass, so the same values). Layouts as gdn_oracle_recurrent; dS_T,
+ * dS0 [n_seq][H][dk][dv] in the pages' orientation. Single threaded.
+ */
+enum { kCkpt = 64 };
+
+static void forward_step(double *S_out, const double *S_in, const double *kt, const double *vt,
+                         double alpha, double beta, int dk, int dv, double *e)
+{
+    for (int a = 0; a < dk * dv; ++a)
+        S_out[a] = alpha * S_in[a];
+    for (int b = 0; b < dv; ++b) {
+        double acc = 0.0;
+        for (int a = 0; a < dk; ++a)
+            acc += S_out[a * dv + b] * kt[a];
+        e[b] = vt[b] - acc;
+    }
+    for (int a = 0; a < dk; ++a)
+        for (int b = 0; b < dv; ++b)
+            S_out[a * dv + b] += beta * kt[a] * e[b];
+}
+
+int gdn_oracle_backward(const double *q, const double *k, const double *v, const double *log_alpha,
+                        const double *beta, const double *S0, const int64_t *cu, int n_seq, int H,
+                        int dk, int dv, double scale, const double *dy, const double *dS_T,
+                        double *dq, double *dk_out, double *dv_out, double *dlog_alpha,
+                        double *dbeta, double *dS0)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !cu || !dy || !dq || !dk_out || !dv_out ||
+        !dlog_alpha || !dbeta || n_seq < 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return -1;
+    const size_t SZ = (size_t)dk * dv;
+    int64_t max_len = 0;
+    for (int i = 0; i < n_seq; ++i)
+        if (cu[i + 1] - cu[i] > max_len)
+            max_len = cu[i + 1] - cu[i];
+    const int64_t n_ck = max_len / kCkpt + 1;
+    double *ck = (double *)malloc(sizeof(double) * SZ * (size_t)n_ck);
+    double *seg = (double *)malloc(sizeof(double) * SZ * (kCkpt + 1));
+    double *G = (double *)malloc(sizeof(double) * SZ);
+    double *Gt = (double *)malloc(sizeof(double) * SZ);
+    double *e = (double *)malloc(sizeof(double) * dv);
+    double *de = (double *)malloc(sizeof(double) * dv);
+    int rc = (ck && seg && G && Gt && e && de) ? 1 : -1;
+    for (int i = 0; rc > 0 && i < n_seq; ++i)
+        for (int h = 0; h < H; ++h) {
+            const int64_t bos = cu[i], T = cu[i + 1] - cu[i];
+            const size_t soff = ((size_t)i * H + h) * SZ;
+            /* forward: keep S at t = 0, kCkpt, 2 kCkpt, ... */
+            if (S0)
+                memcpy(seg, S0 + soff, sizeof(double) * SZ);
+            else
+                memset(seg, 0, sizeof(double) * SZ);
+            memcpy(ck, seg, sizeof(double) * SZ);
+            for (int64_t t = 0; t < T; ++t) {
+                const size_t r = (size_t)(bos + t) * H + h;
+                forward_step(seg + SZ, seg, k + r * dk, v + r * dv, exp(log_alpha[r]), beta[r], dk, dv, e);
+                memcpy(seg, seg + SZ, sizeof(double) * SZ);
+                if ((t + 1) % kCkpt == 0)
+                    memcpy(ck + (size_t)((t + 1) / kCkpt) * SZ, seg, sizeof(double) * SZ);
+            }
+            /* backward, one checkpoint segment at a time from the end */
+            if (dS_T)
+                memcpy(G, dS_T + soff, sizeof(double) * SZ);
+            else
+                memset(G, 0, sizeof(double) * SZ);
+            for (int64_t s0 = (T == 0 ? 0 : (T - 1) / kCkpt * kCkpt); s0 >= 0 && T > 0; s0 -= kCkpt) {
+                const int64_t s1 = s0 + kCkpt < T ? s0 + kCkpt : T;
+                /* seg[j] = S_{s0 + j}, j = 0 .. s1 - s0 */
+                memcpy(seg, ck + (size_t)(s0 / kCkpt) * SZ, sizeof(double) * SZ);
+                for (int64_t t = s0; t < s1; ++t) {
+                    const size_t r = (size_t)(bos + t) * H + h;
+                    forward_step(seg + (size_t)(t - s0 + 1) * SZ, seg + (size_t)(t - s0) * SZ, k + r * dk,
+                                 v + r * dv, exp(log_alpha[r]), beta[r], dk, dv, e);
+                }
+                for (int64_t t = s1 - 1; t >= s0; --t) {
+                    const size_t r = (size_t)(bos + t) * H + h;
+                    const double *St = seg + (size_t)(t - s0 + 1) * SZ;      /* S_t */
+                    const double *Sp = seg + (size_t)(t - s0) * SZ;          /* S_{t-1} */
+                    const double *qt = q + r * dk, *kt = k + r * dk, *vt = v + r * dv, *dyt = dy + r * dv;
+                    const double alpha = exp(log_alpha[r]), bt = beta[r];
+                    double *dqt = dq + r * dk, *dkt = dk_out + r * dk, *dvt = dv_out + r * dv;
+                    /* y_t = S_t^T (scale q_t) */
+                    for (int a = 0; a < dk; ++a) {
+                        double acc = 0.0;
+                        for (int b = 0; b < dv; ++b)
+                            acc += St[a * dv + b] * dyt[b];
+                        dqt[a] = scale * acc;
+                    }
+                    for (int a = 0; a < dk; ++a)
+                        for (int b = 0; b < dv; ++b)
+                            G[a * dv + b] += scale * qt[a] * dyt[b];
+                    /* e_t and S~_t = alpha S_{t-1} */
+                    for (int b = 0; b < dv; ++b) {
+                        double acc = 0.0;
+                        for (int a = 0; a < dk; ++a)
+                            acc += alpha * Sp[a * dv + b] * kt[a];
+                        e[b] = vt[b] - acc;
+                    }
+                    /* S_t = S~_t + beta k e^T */
+                    double db = 0.0;
+                    for (int a = 0; a < dk; ++a) {
+                        double ge = 0.0;
+                        for (int b = 0; b < dv; ++b)
+                            ge += G[a * dv + b] * e[b];
+                        db += kt[a] * ge;
+                        dkt[a] = bt * ge;
+                    }
+                    dbeta[r] = db;
+                    for (int b = 0; b < dv; ++b) {
+                        double acc = 0.0;
+                        for (int a = 0; a < dk; ++a)
+                            acc += G[a * dv + b] * kt[a];
+                        de[b] = bt * acc;
+                        dvt[b] = de[b];
+                    }
+                    /* e = v - S~^T k */
+                    for (int a = 0; a < dk * dv; ++a)
+                        Gt[a] = G[a];
+                    for (int a = 0; a < dk; ++a) {
+                        double sd = 0.0;
+                        for (int b = 0; b < dv; ++b) {
+                            Gt[a * dv + b] -= kt[a] * de[b];
+                            sd += alpha * Sp[a * dv + b] * de[b];
+                        }
+                        dkt[a] -= sd;
+                    }
+                    /* S~ = alpha S_{t-1} */
+                    double dal = 0.0;
+                    for (int a = 0; a < dk * dv; ++a) {
+                        dal += Gt[a] * Sp[a];
+                        G[a] = alpha * Gt[a];
+                    }
+                    dlog_alpha[r] = alpha * dal;
+                }
+            }
+            if (dS0)
+                memcpy(dS0 + soff, G, sizeof(double) * SZ);
+        }
+    free(ck);
+    free(seg);
+    free(G);
+    free(Gt);
+    free(e);
+    free(de);
+    return rc;
+}

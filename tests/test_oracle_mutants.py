@@ -13,6 +13,7 @@ import types
 import pytest
 
 import oracle
+from tests import test_oracle_backward as bpins
 from tests import test_oracle_featurize as fpins
 from tests import test_oracle_pins as pins
 
@@ -68,6 +69,14 @@ MUTANTS = {
                       "featurize_stream(xv, conv_v, W, cu, n_seq, H, dv, 1, eps, v);")],
     "decay_bias_dropped": [("softplus(alpha_logit[e] + b_alpha[h]);", "softplus(alpha_logit[e]);")],
     "decay_rate_not_exp": [("log_alpha[e] = -exp(A[h]) * softplus", "log_alpha[e] = -A[h] * softplus")],
+    # gradients: the output term dropped from the state adjoint, the error term's sign, the
+    # decay gradient against the new state, the decay missing from the carried adjoint, the
+    # key gradient's error part dropped
+    "bwd_no_output_term": [("                            G[a * dv + b] += scale * qt[a] * dyt[b];\n", "")],
+    "bwd_error_term_sign": [("Gt[a * dv + b] -= kt[a] * de[b];", "Gt[a * dv + b] += kt[a] * de[b];")],
+    "bwd_dalpha_new_state": [("dal += Gt[a] * Sp[a];", "dal += Gt[a] * St[a];")],
+    "bwd_carry_without_decay": [("G[a] = alpha * Gt[a];", "G[a] = Gt[a];")],
+    "bwd_dk_error_part_dropped": [("                        dkt[a] -= sd;\n", "")],
 }
 
 PIN_TESTS = [
@@ -81,7 +90,7 @@ PIN_TESTS = [
     pins.test_hand_example,
     pins.test_decode_step_matches_one_token_recurrence,
     pins.test_gate_norm_closed_forms,
-] + fpins.PINS
+] + fpins.PINS + bpins.PINS
 
 
 def _mutant_module(tmp_path, name, edits):
@@ -96,7 +105,7 @@ def _mutant_module(tmp_path, name, edits):
                     str(c_path), "-lm", "-lpthread"], check=True)
     lib = oracle._configure(ctypes.CDLL(str(so_path)))
     mod = types.SimpleNamespace()
-    for fn in ("recurrent", "decode_step", "gate_norm", "featurize"):
+    for fn in ("recurrent", "decode_step", "gate_norm", "featurize", "backward"):
         f = getattr(oracle, fn)
 
         def wrapped(*a, _f=f, **kw):
