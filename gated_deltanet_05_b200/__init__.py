@@ -22,7 +22,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_gated", "chunk_fwd_noalloc", "selftest_bounded_wait", "decode_step", "decode_tokens", "gate_norm", "featurize",
+__all__ = ["chunk_fwd", "chunk_fwd_gated", "chunk_fwd_noalloc", "backward", "selftest_bounded_wait", "decode_step", "decode_tokens", "gate_norm", "featurize",
            "device_error", "lib", "LIB_PATH",
            "GdnError", "EXPORTED_SYMBOLS", "STATUS"]
 
@@ -33,7 +33,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_fwd_gated",
-                    "gdn_chunk_fwd_noalloc",
+                    "gdn_chunk_fwd_noalloc", "gdn_backward_workspace_bytes", "gdn_backward",
                     "gdn_selftest_bounded_wait", "gdn_decode_step", "gdn_decode_tokens",
                     "gdn_gate_norm", "gdn_featurize", "gdn_status_string", "gdn_device_error",
                     "gdn_version")
@@ -70,6 +70,11 @@ def lib():
         L.gdn_chunk_fwd_gated.restype = i32
         L.gdn_chunk_fwd_gated.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                           f32, vp, vp, f32, vp, i32, vp, vp, ctypes.c_size_t, vp]
+        L.gdn_backward_workspace_bytes.restype = ctypes.c_size_t
+        L.gdn_backward_workspace_bytes.argtypes = [vp, i32, i32, i32, i32]
+        L.gdn_backward.restype = i32
+        L.gdn_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp, vp,
+                                   vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.gdn_chunk_fwd_noalloc.restype = i32
         L.gdn_chunk_fwd_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                             i32, f32, vp, i32, vp, vp]
@@ -217,6 +222,40 @@ def chunk_fwd_gated(q, k, v, log_alpha, beta, cu_seqlens, z, w, eps=1e-6, S0=Non
                                _dtype_code(o), _ptr(S_T), _ptr(ws), ws_bytes, _stream(q.device))
     _check("gdn_chunk_fwd_gated", rc)
     return o, S_T
+
+
+def backward(q, k, v, log_alpha, beta, cu_seqlens, dy, S0=None, dS_T=None, scale=1.0,
+             cu_seqlens_host=None):
+    """Gradients of L = sum <dy, y> + <dS_T, S_T> through the prefill.
+
+    Inputs as chunk_fwd; dy [N, H, d_v] in q's dtype; dS_T [n_seq, H, d_v, d_k] fp32 or None.
+    Returns (dq, dk, dv, dlog_alpha, dbeta, dS0), all fp32 (dS0 in the state layout)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (log_alpha, "log_alpha"), (beta, "beta"),
+                 (cu_seqlens, "cu_seqlens"), (dy, "dy")):
+        _cuda(t, n)
+    _cuda(S0, "S0")
+    _cuda(dS_T, "dS_T")
+    if k.dtype != q.dtype or v.dtype != q.dtype or dy.dtype != q.dtype:
+        raise TypeError("q, k, v, dy must share one dtype")
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    n_seq = cu_seqlens.numel() - 1
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.to("cpu")
+    cu_h = cu_seqlens_host.to(torch.int32).contiguous()
+    L = lib()
+    ws_bytes = L.gdn_backward_workspace_bytes(ctypes.c_void_p(cu_h.data_ptr()), n_seq, H, dk, dv)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    f = dict(dtype=torch.float32, device=q.device)
+    dq, dkk, dvv = torch.empty((N, H, dk), **f), torch.empty((N, H, dk), **f), torch.empty((N, H, dv), **f)
+    dla, db = torch.empty((N, H), **f), torch.empty((N, H), **f)
+    dS0 = torch.empty((n_seq, H, dv, dk), **f)
+    rc = L.gdn_backward(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                        _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), n_seq, H, dk, dv, float(scale),
+                        _ptr(dy), _ptr(dS_T), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla), _ptr(db), _ptr(dS0),
+                        _ptr(ws), ws_bytes, _stream(q.device))
+    _check("gdn_backward", rc)
+    return dq, dkk, dvv, dla, db, dS0
 
 
 def chunk_fwd_noalloc(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0,

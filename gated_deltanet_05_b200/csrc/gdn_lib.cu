@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "gdn.h"
+#include "gdn_backward.cuh"
 #include "gdn_chunk_f32.cuh"
 #include "gdn_chunk_sm100.cuh"
 #include "gdn_common.cuh"
@@ -290,6 +291,66 @@ gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_
     return launch_chunk_sm100<__nv_bfloat16, true>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev, n_seq,
                                                    n_tok, H, scale, o, S_T, workspace, workspace_bytes, st,
                                                    z, w, eps);
+}
+
+size_t gdn_backward_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, int H, int d_k, int d_v)
+{
+    if (!cu_seqlens_host || n_seq <= 0 || H <= 0 || d_k <= 0 || d_v <= 0) return 0;
+    int64_t max_len = 0;
+    for (int i = 0; i < n_seq; ++i) {
+        const int64_t l = (int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i];
+        if (l > max_len) max_len = l;
+    }
+    return (size_t)n_seq * H * gdn::bwd_ws_floats_per_chain(max_len, d_k, d_v) * sizeof(float);
+}
+
+gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                        const float *log_alpha, const float *beta, const float *S0,
+                        const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int n_seq,
+                        int H, int d_k, int d_v, float scale, const void *dy, const float *dS_T,
+                        float *dq, float *dk, float *dv, float *dlog_alpha, float *dbeta, float *dS0,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (n_seq < 0 || H <= 0 || !cu_seqlens_host || (n_seq > 0 && !cu_seqlens_dev))
+        return GDN_ERR_INVALID_ARG;
+    if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!pow2_in(d_k, 16, 128) || !pow2_in(d_v, 16, 128)) return GDN_ERR_UNSUPPORTED;
+    if (cu_seqlens_host[0] != 0) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < n_seq; ++i)
+        if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return GDN_ERR_INVALID_ARG;
+    if (n_seq == 0) return GDN_OK;
+    if ((int64_t)n_seq * H > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    const int64_t n_tok = cu_seqlens_host[n_seq];
+    if (n_tok > 0 && (!q || !k || !v || !log_alpha || !beta || !dy || !dq || !dk || !dv ||
+                      !dlog_alpha || !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_backward_workspace_bytes(cu_seqlens_host, n_seq, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(S0, 4) || !aligned(dS_T, 4) || !aligned(dS0, 4)) return GDN_ERR_INVALID_ARG;
+    int64_t max_len = 0;
+    for (int i = 0; i < n_seq; ++i)
+        if ((int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i] > max_len)
+            max_len = (int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i];
+    cudaStream_t st = as_stream(stream);
+    const int smem = (int)(sizeof(float) * (2 * (size_t)d_v * (d_k + 1) + 2 * d_k + 4 * d_v + gdn::kBwdThreads / 32));
+    if (smem > smem_optin()) return GDN_ERR_UNSUPPORTED;
+    const unsigned grid = (unsigned)((int64_t)n_seq * H);
+#define GDN_BWD(T)                                                                                 \
+    {                                                                                              \
+        auto kern = gdn::gdn_backward_kernel<T>;                                                   \
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+            return GDN_ERR_CUDA;                                                                   \
+        kern<<<grid, gdn::kBwdThreads, smem, st>>>((const T *)q, (const T *)k, (const T *)v, log_alpha, beta, \
+                                                   S0, cu_seqlens_dev, H, d_k, d_v, scale, (const T *)dy, dS_T, \
+                                                   dq, dk, dv, dlog_alpha, dbeta, dS0,             \
+                                                   static_cast<float *>(workspace), max_len);      \
+    }
+    if (in_dtype == GDN_F32)
+        GDN_BWD(float)
+    else
+        GDN_BWD(__nv_bfloat16)
+#undef GDN_BWD
+    return launch_status();
 }
 
 gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gdn_dtype in_dtype,

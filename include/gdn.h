@@ -169,6 +169,31 @@ gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_
                                float *S_T, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gdn_backward -- gradients of the chunked prefill's result with respect to its inputs.
+ *
+ * Defines: the reverse-mode adjoint of the token recurrence (joezjh.github.io notes,
+ * "Gated DeltaNet 核心机制"; the pages report a backward kernel but print none) for
+ * L = sum_t <dy_t, y_t> + <dS_T, S_T>:
+ *   q, k, v, in_dtype, log_alpha, beta, S0, cu_seqlens_*, n_seq, H, d_k, d_v, scale: as for
+ *          gdn_chunk_fwd (S0 may be NULL: zeros)
+ *   dy     [n_tok, H, d_v] in in_dtype;  dS_T [n_seq, H, d_v, d_k] fp32 or NULL (zero)
+ *   dq, dk [n_tok, H, d_k], dv [n_tok, H, d_v], dlog_alpha, dbeta [n_tok, H] fp32 out
+ *   dS0    [n_seq, H, d_v, d_k] fp32 out, or NULL
+ *   workspace: gdn_backward_workspace_bytes(...) bytes, 16-byte aligned (state copies every
+ *          64 tokens plus one recomputed 64-token segment per chain)
+ *   d_k, d_v in {16, 32, 64, 128}
+ * One CTA per chain on CUDA cores in fp32: the correctness-first form of the backward.
+ */
+size_t gdn_backward_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, int H, int d_k,
+                                    int d_v);
+gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
+                        const float *log_alpha, const float *beta, const float *S0,
+                        const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int n_seq,
+                        int H, int d_k, int d_v, float scale, const void *dy, const float *dS_T,
+                        float *dq, float *dk, float *dv, float *dlog_alpha, float *dbeta, float *dS0,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdn_decode_step -- one token for each of n_seq * H independent chains, in place.
  *
  * Defines: the same four-line update (joezjh.github.io notes, "Gated DeltaNet 核心机制")

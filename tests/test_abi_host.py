@@ -120,6 +120,30 @@ def test_decode_and_gate_norm_reject_bad_arguments(L):
     assert gn(rows=0) == 0
 
 
+def test_backward_rejects_bad_arguments(L):
+    cu = (ctypes.c_int32 * 3)(0, 64, 100)
+    assert L.gdn_backward_workspace_bytes(ctypes.cast(cu, ctypes.c_void_p), 2, 2, 128, 128) == \
+        2 * 2 * (64 // 64 + 1 + 65) * 128 * 128 * 4
+    assert L.gdn_backward_workspace_bytes(None, 2, 2, 128, 128) == 0
+
+    def bw(**kw):
+        c = kw.get("cu", cu)
+        return L.gdn_backward(FAKE, FAKE, FAKE, kw.get("dt", 0), FAKE, FAKE, None, FAKE,
+                              ctypes.cast(c, ctypes.c_void_p) if c is not None else None,
+                              kw.get("n_seq", 2), kw.get("H", 2), kw.get("dk", 128), kw.get("dv", 128),
+                              1.0, kw.get("dy", FAKE), None, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                              kw.get("ws", FAKE), kw.get("wsb", 1 << 30), None)
+    assert bw(dt=2) == 1
+    assert bw(dk=24) == 2
+    assert bw(H=0) == 1
+    assert bw(cu=None) == 1
+    assert bw(cu=(ctypes.c_int32 * 3)(0, 64, 10)) == 1
+    assert bw(dy=None) == 1
+    assert bw(wsb=1000) == 1
+    assert bw(ws=None) == 1
+    assert bw(n_seq=0) == 0
+
+
 def test_chunk_fwd_gated_rejects_bad_arguments(L):
     cu = (ctypes.c_int32 * 3)(0, 64, 100)
     cu_bad = (ctypes.c_int32 * 3)(0, 64, 10)
