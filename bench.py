@@ -356,6 +356,7 @@ def run_ours(args, rank, world, local, pg):
 
     decode = None if args.no_decode else bench_decode(args, device, peaks, peak_kind, pg)
     featurize = bench_featurize(args, device, peaks, peak_kind, pg, rank)
+    backward = bench_backward(args, inp, device, pg) if world == 1 else None
     e2e = bench_e2e(args, inp, device, pg, world)
 
     line = {
@@ -372,6 +373,7 @@ def run_ours(args, rank, world, local, pg):
         "fused_step": fused,
         "decode": decode,
         "featurize": featurize,
+        "backward": backward,
         "e2e": e2e,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
@@ -501,6 +503,39 @@ def bench_featurize(args, device, peaks, peak_kind, pg, rank):
             "bytes_per_launch": step_bytes, "achieved": gbs, "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
             "steps": steps, "l2": "inputs 192 MiB > L2"}
+
+
+def bench_backward(args, inp, device, pg):
+    """The backward (gdn_backward) on the prefill workload, a few launches. Guarded: a
+    failure here is reported in the line instead of ending the run."""
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    try:
+        dev = {k: inp[k].to(device) for k in ("q", "k", "v", "log_alpha", "beta", "cu_seqlens", "z")}
+        dy = dev["z"]                           # any bf16 [N, H, d_v] cotangent
+        cu_host = inp["cu_seqlens"]
+        run = lambda: gdn.backward(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                                   dev["cu_seqlens"], dy, cu_seqlens_host=cu_host)
+        run()
+        torch.cuda.synchronize(device)
+        reps = 3
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        barrier(pg, device)
+        a.record()
+        for _ in range(reps):
+            run()
+        b.record()
+        torch.cuda.synchronize(device)
+        ms = max_over_ranks(pg, a.elapsed_time(b), device) / reps
+        status = gdn.device_error(device)
+        n_tok = inp["q"].shape[0]
+        return {"kernel": "gdn::gdn_backward_kernel (fp32, one CTA per chain)", "ms_per_launch": ms,
+                "tokens_per_s": n_tok / (ms * 1e-3), "launches": reps, "status": status,
+                "workload": "prefill shape: 4 x 4096 tokens, H=16, d=128, bf16 inputs"}
+    except Exception as exc:                      # reported, not raised
+        return {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
 
 def bench_e2e(args, inp, device, pg, world):
