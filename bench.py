@@ -53,11 +53,10 @@ def flops_per_token_head(chunk: int, d: int) -> float:
     return 10.0 * chunk * d + 6.0 * d * d + chunk * chunk / 3.0
 
 
-def prefill_bytes_per_token_head(in_elem: int, y_elem: int, d: int, z_elem: int = 0) -> float:
-    """Minimal HBM bytes per (token, head): read q, k, v (3 d in_elem), write y or o
-    (d y_elem), read z when the gate-norm is fused (d z_elem), read log_alpha and beta
-    (8 bytes)."""
-    return 3 * in_elem * d + y_elem * d + z_elem * d + 8.0
+def prefill_bytes_per_token_head(in_elem: int, y_elem: int, d: int) -> float:
+    """Minimal HBM bytes per (token, head): read q, k, v (3 d in_elem), write y (d y_elem),
+    read log_alpha and beta (8 bytes)."""
+    return 3 * in_elem * d + y_elem * d + 8.0
 
 
 def load_peaks():
