@@ -1,8 +1,9 @@
 /*
  * gdn.h -- C ABI of the B200 (sm_100a) gated delta rule library, libgdn_b200.so.
  *
- * The library computes the Gated DeltaNet token mixer's gated delta rule and its
- * output epilogue, as defined on the joezjh.github.io notes page "Qwen3.8-Flash-Next"
+ * The library computes the Gated DeltaNet token mixer's gated delta rule (chunked prefill,
+ * one- and several-token decode, and the gradients), its output epilogue and the feature
+ * and gate step in front of it, as defined on the joezjh.github.io notes page "Qwen3.8-Flash-Next"
  * (section "Gated DeltaNet 核心机制", the four-line update rule and its equivalent
  * form; section "GDN 参数化细节", the output-gate equation) and on the pwwt.cn
  * translation of the report (section 2.1.1, "sigmoid output gate", "zero-centred
