@@ -9,7 +9,6 @@ o = sigmoid(z) * RMSNorm(y) * (1 + w) is checked two ways:
 Lengths cover full chunks, partial last chunks whose second half is empty (n <= 32), an
 empty sequence and S0 != 0; the full prefill workload is checked on sampled chains.
 """
-import numpy as np
 import pytest
 import torch
 

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import workloads as W
-from tests.helpers import TOL, f64, oracle_prefill, rel_err, subset, to_dev
+from tests.helpers import TOL, f64, oracle_prefill, rel_err, to_dev
 
 gdn = pytest.importorskip("gated_deltanet_05_b200")
 
