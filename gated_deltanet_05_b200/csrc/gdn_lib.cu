@@ -560,10 +560,10 @@ gdn_status gdn_featurize(const void *xq, const void *xk, const void *xv, gdn_dty
     }
     if (dtype == GDN_BF16) {
         GDN_FT_D(b16, d_k, true, xq, xk, conv_q, conv_k, q, k, 2, false)
-        GDN_FT_D(b16, d_v, false, xv, xv, conv_v, conv_v, v, v, 1, true)
+        GDN_FT_D(b16, d_v, false, xv, nullptr, conv_v, nullptr, v, nullptr, 1, true)
     } else {
         GDN_FT_D(f32, d_k, true, xq, xk, conv_q, conv_k, q, k, 2, false)
-        GDN_FT_D(f32, d_v, false, xv, xv, conv_v, conv_v, v, v, 1, true)
+        GDN_FT_D(f32, d_v, false, xv, nullptr, conv_v, nullptr, v, nullptr, 1, true)
     }
 #undef GDN_FT_D
 #undef GDN_FT
