@@ -12,7 +12,9 @@ synthetic draws (workloads/), resident in HBM before the timed region; q, k, v a
 
 The decode step (256 sequences x 32 heads, d = 128, 537 MB fp32 state in HBM) is timed
 separately and reported under "decode"; the featurisation step in front of the prefill
-(gdn_featurize on the prefill workload's shape) under "featurize".
+(gdn_featurize on the prefill workload's shape) under "featurize"; the prefill alone on
+the long-context workload (one 65,536-token sequence, H = 32, S0 != 0) and on the packed
+variable-length batch (8 sequences, H = 16) under "prefill_long" and "prefill_varlen".
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent batch
 (the chains do not interact), so scaling is weak and the data path has no collective;
@@ -40,7 +42,7 @@ if ROOT not in sys.path:
 METRIC = "GDN prefill tokens/s + % tensor peak; decode-step state GB/s vs HBM peak"
 UNIT = "tokens/s"
 WORKLOAD = ("prefill bf16: 4 seqs x 4096 tokens, H=16, d_k=d_v=128, chunk 64, fp32 state, "
-            "fp32 y, then sigmoid-gate zero-centred RMSNorm (bf16 z and o)")
+            "bf16 y, then sigmoid-gate zero-centred RMSNorm (bf16 z and o)")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["gated_deltanet_05_b200/csrc/gdn_chunk_sm100.cuh",
                   "gated_deltanet_05_b200/csrc/sm100_ptx.cuh"]
@@ -261,12 +263,12 @@ def run_ours(args, rank, world, local, pg):
     n_tok = int(inp["cu_seqlens"][-1])
     dev = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     cu_host = inp["cu_seqlens"]
-    y = torch.empty((n_tok, H, d), dtype=torch.float32, device=device)
+    y = torch.empty((n_tok, H, d), dtype=torch.bfloat16, device=device)
     o = torch.empty((n_tok, H, d), dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step(ev=None):
-        # the whole hot path: chunked prefill (fp32 y), then the gate-norm epilogue
+        # the whole hot path: chunked prefill (bf16 y), then the gate-norm epilogue
         if ev is not None:
             ev[0].record(stream)
         gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
@@ -324,7 +326,7 @@ def run_ours(args, rank, world, local, pg):
     peaks, peak_kind = load_peaks()
     token_heads = n_tok * H
     flops = flops_per_token_head(C, d) * token_heads
-    algo_bytes = prefill_bytes_per_token_head(2, 4, d) * token_heads + len(w.lengths) * H * d * d * 4
+    algo_bytes = prefill_bytes_per_token_head(2, 2, d) * token_heads + len(w.lengths) * H * d * d * 4
     chunk_s = chunk_ms * 1e-3
     tflops = flops / chunk_s / 1e12
     gbs = algo_bytes / chunk_s / 1e9
@@ -344,7 +346,7 @@ def run_ours(args, rank, world, local, pg):
                    "flops_per_launch": flops,
                    "flops_per_token_head": flops_per_token_head(C, d)},
     }
-    gn_bytes = (4 + 2 + 2) * n_tok * H * d + 4 * d          # y fp32, z and o bf16
+    gn_bytes = (2 + 2 + 2) * n_tok * H * d + 4 * d          # y, z and o bf16
     gate_norm_obj = {"launch_ms": gn_ms, "achieved": gn_bytes / (gn_ms * 1e-3) / 1e9,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gn_bytes / (gn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -353,6 +355,9 @@ def run_ours(args, rank, world, local, pg):
              "note": "the same step as one gdn_chunk_fwd_gated launch (gate-norm in the prefill's "
                      "output stage), 20 steps"}
 
+    shapes = {} if args.no_shapes else {
+        "long": bench_prefill_shape(args, "long", device, peaks, peak_kind, pg, rank),
+        "varlen": bench_prefill_shape(args, "varlen", device, peaks, peak_kind, pg, rank)}
     decode = None if args.no_decode else bench_decode(args, device, peaks, peak_kind, pg)
     featurize = bench_featurize(args, device, peaks, peak_kind, pg, rank)
     backward = bench_backward(args, inp, device, pg) if world == 1 else None
@@ -368,6 +373,8 @@ def run_ours(args, rank, world, local, pg):
                    "heads": H, "d_k": d, "d_v": d, "chunk": C, "parallelism": f"dp{world}",
                    "l2": "no flush: q, k, v, z are 256 MiB per step, above the 126 MB L2"},
         "roofline": roofline,
+        "prefill_long": shapes.get("long"),
+        "prefill_varlen": shapes.get("varlen"),
         "gate_norm": gate_norm_obj,
         "fused_step": fused,
         "decode": decode,
@@ -381,6 +388,62 @@ def run_ours(args, rank, world, local, pg):
         line["cpu_baseline"] = cpu_baseline(inp, H)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def bench_prefill_shape(args, name, device, peaks, peak_kind, pg, rank):
+    """gdn_chunk_fwd alone (bf16 y, S_T written) on another prefill workload: "long" (one
+    65,536-token sequence, H = 32, S0 != 0, A ~ U(-3, 1)) or "varlen" (8 packed sequences
+    of U[512, 8192] tokens, H = 16). Roofline bytes per launch: q, k, v, y in bf16 and the
+    fp32 gates per token-head, plus S_T (and S0 when present) per chain."""
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    import workloads as W
+    w = W.WORKLOADS[name]
+    inp = W.make_prefill_inputs(w, with_gate=False, seed=w.seed + 1000 * rank)
+    dev = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    n_tok = int(inp["cu_seqlens"][-1])
+    n_seq = inp["cu_seqlens"].numel() - 1
+    H, d, C = w.H, w.d_k, w.chunk
+    y = torch.empty((n_tok, H, d), dtype=torch.bfloat16, device=device)
+    S_T = torch.empty((n_seq, H, d, d), dtype=torch.float32, device=device)
+    cu_host = inp["cu_seqlens"]
+    stream = torch.cuda.current_stream(device)
+
+    def run():
+        gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], dev["cu_seqlens"],
+                      S0=dev.get("S0"), chunk=C, cu_seqlens_host=cu_host, out=y, state_out=S_T)
+
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize(device)
+    reps = 10
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(pg, device)
+    a.record(stream)
+    for _ in range(reps):
+        run()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    status = gdn.device_error(device)
+    if status != "GDN_OK":
+        raise SystemExit(f"device error in the {name} prefill leg: {status}")
+    ms = max_over_ranks(pg, a.elapsed_time(b), device) / reps
+    token_heads = n_tok * H
+    n_states = (2 if dev.get("S0") is not None else 1) * n_seq * H
+    algo_bytes = prefill_bytes_per_token_head(2, 2, d) * token_heads + n_states * d * d * 4
+    flops = flops_per_token_head(C, d) * token_heads
+    gbs = algo_bytes / (ms * 1e-3) / 1e9
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"{name} bf16: {n_seq} seq(s), {n_tok} tokens, H={H}, d={d}, chunk {C}, "
+                        f"bf16 y" + (", S0 != 0" if dev.get("S0") is not None else ""),
+            "chains": n_seq * H, "launch_ms": ms, "tokens_per_s": n_tok / (ms * 1e-3),
+            "bytes_per_launch": algo_bytes, "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+            "tensor": {"achieved": tflops, "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                       "flops_per_launch": flops},
+            "launches": reps, "l2": "inputs above the 126 MB L2"}
 
 
 def bench_decode(args, device, peaks, peak_kind, pg):
@@ -558,7 +621,7 @@ def bench_e2e(args, inp, device, pg, world):
         for k in host:
             dev[k].copy_(host[k], non_blocking=True)
         y, _ = gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], cu_dev,
-                             chunk=C, cu_seqlens_host=cu_host)
+                             chunk=C, cu_seqlens_host=cu_host, y_dtype=torch.bfloat16)
         o = gdn.gate_norm(y, dev["z"], w_dev, out_dtype=torch.bfloat16)
         o_host.copy_(o, non_blocking=True)
 
@@ -599,7 +662,7 @@ def cpu_baseline(inp, H, min_seconds=10.0, max_reps=12):
 
 def run_case(args):
     """A few launches of one kernel on a named shape, nothing else (for ncu captures):
-    --case prefill:S,T,H   (bf16, d=128, chunk 64, fp32 y)
+    --case prefill:S,T,H   (bf16, d=128, chunk 64, bf16 y)
     --case prefill_gated:S,T,H (the same with the fused gate-norm, bf16 z and o)
     --case decode:N        (N sequences x 32 heads, d=128, fp32 state)
     --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)
@@ -619,7 +682,7 @@ def run_case(args):
         d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
         for _ in range(args.reps):
             gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"],
-                          cu_seqlens_host=inp["cu_seqlens"])
+                          cu_seqlens_host=inp["cu_seqlens"], y_dtype=torch.bfloat16)
     elif kind == "prefill_gated":
         n_seq, T, H = dims
         w = W.Workload("case", "bf16", (T,) * n_seq, H, 128, 128, 64, seed=1)
@@ -676,6 +739,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-shapes", action="store_true", help="skip the long and varlen prefill legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None, help="profiling case, e.g. prefill:4,4096,16")
     ap.add_argument("--reps", type=int, default=3)

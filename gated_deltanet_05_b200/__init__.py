@@ -81,9 +81,9 @@ def lib():
         L.gdn_selftest_bounded_wait.restype = i32
         L.gdn_selftest_bounded_wait.argtypes = [i64, i32, vp]
         L.gdn_decode_step.restype = i32
-        L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, vp, vp]
+        L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, vp, i32, vp]
         L.gdn_decode_tokens.restype = i32
-        L.gdn_decode_tokens.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]
+        L.gdn_decode_tokens.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, vp]
         L.gdn_gate_norm.restype = i32
         L.gdn_gate_norm.argtypes = [vp, i32, vp, i32, vp, i64, i32, f32, vp, i32, vp]
         L.gdn_featurize.restype = i32
@@ -272,33 +272,41 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, s
     return y, S_T
 
 
-def decode_step(q, k, v, alpha, beta, S, scale=1.0, out=None):
-    """One token per chain; S [n_seq, H, d_v, d_k] fp32 is updated in place. Returns y."""
+def decode_step(q, k, v, alpha, beta, S, scale=1.0, out=None, y_dtype=torch.float32):
+    """One token per chain; S [n_seq, H, d_v, d_k] fp32 is updated in place. Returns y in
+    y_dtype (float32 by default; bfloat16 gives the round-to-nearest-even of the same fp32
+    result), or in out's dtype when out is given."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (alpha, "alpha"), (beta, "beta"), (S, "S")):
         _cuda(t, n)
     code = _dtype_code(q)
     n_seq, H, dk = q.shape
     dv = v.shape[2]
-    y = out if out is not None else torch.empty((n_seq, H, dv), dtype=q.dtype, device=q.device)
+    y = out if out is not None else torch.empty((n_seq, H, dv), dtype=y_dtype, device=q.device)
+    _cuda(y, "out")
     rc = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha), _ptr(beta), _ptr(S),
-                               n_seq, H, dk, dv, float(scale), _ptr(y), _stream(q.device))
+                               n_seq, H, dk, dv, float(scale), _ptr(y), _dtype_code(y),
+                               _stream(q.device))
     _check("gdn_decode_step", rc)
     return y
 
 
-def decode_tokens(q, k, v, alpha, beta, S, scale=1.0, out=None):
+def decode_tokens(q, k, v, alpha, beta, S, scale=1.0, out=None, y_dtype=torch.float32):
     """n consecutive tokens per chain in one pass over the state (S updated in place).
 
     q, k [n_seq, n, H, d_k], v [n_seq, n, H, d_v] (fp32 or bf16, one dtype); alpha, beta
-    [n_seq, n, H] fp32; S [n_seq, H, d_v, d_k] fp32. Returns y [n_seq, n, H, d_v]."""
+    [n_seq, n, H] fp32; S [n_seq, H, d_v, d_k] fp32. Returns y [n_seq, n, H, d_v] in
+    y_dtype (float32 by default; bfloat16 gives the round-to-nearest-even of the same fp32
+    result), or in out's dtype when out is given."""
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (alpha, "alpha"), (beta, "beta"), (S, "S")):
         _cuda(t, nm)
     code = _dtype_code(q)
     n_seq, n, H, dk = q.shape
     dv = v.shape[3]
-    y = out if out is not None else torch.empty((n_seq, n, H, dv), dtype=q.dtype, device=q.device)
+    y = out if out is not None else torch.empty((n_seq, n, H, dv), dtype=y_dtype, device=q.device)
+    _cuda(y, "out")
     rc = lib().gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha), _ptr(beta), _ptr(S),
-                                 n_seq, n, H, dk, dv, float(scale), _ptr(y), _stream(q.device))
+                                 n_seq, n, H, dk, dv, float(scale), _ptr(y), _dtype_code(y),
+                                 _stream(q.device))
     _check("gdn_decode_tokens", rc)
     return y
 

@@ -138,6 +138,10 @@ constexpr uint32_t TM_S = 0, TM_Y = 128, TM_W = 256, TM_U = 320, TM_SB = 384, TM
 
 constexpr uint32_t SMEM_BYTES = (sv::SMEM_USED > ch::SMEM_USED ? sv::SMEM_USED : ch::SMEM_USED) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// At most one CTA of this kernel fits on an SM. The workspace (and the fixed array of the
+// allocation-free entry point) gives each SM id one K-ring region, which is safe for
+// overlapping launches only because no two solver CTAs can share an SM.
+static_assert(2 * SMEM_BYTES > 232448, "one CTA per SM: the per-SM-id workspace regions rely on it");
 static_assert(sv::OFF_SEND % 1024 == 0 && ch::OFF_QV % 1024 == 0 && ch::OFF_RECV % 1024 == 0 &&
                   ch::OFF_WB % 1024 == 0, "swizzle atoms");
 
@@ -188,6 +192,29 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v, float f)
 {
     return make_uint4(pack_f16x2(bf_lo(v.x) * f, bf_hi(v.x) * f), pack_f16x2(bf_lo(v.y) * f, bf_hi(v.y) * f),
                       pack_f16x2(bf_lo(v.z) * f, bf_hi(v.z) * f), pack_f16x2(bf_lo(v.w) * f, bf_hi(v.w) * f));
+}
+
+// Converts row u of n_tiles consecutive 8 KB tiles (64 rows of 128 bytes, bf16 as loaded)
+// to fp16 in place, multiplying the values of the first n_scaled tiles by f; returns the
+// running magnitude maximum of the converted fp16 values (f16x2_absmax). A whole row is
+// rewritten, so the 128-byte swizzle does not matter; the rotated chunk order keeps the
+// eight threads of a row group on distinct banks. Rolled two 16-byte chunks at a time:
+// this code shares the instruction cache with the kernel's other roles.
+__device__ __forceinline__ uint32_t convert_rows_bf16_f16(uint8_t *tiles, int n_tiles, int n_scaled, float f, int u,
+                                                         uint32_t absmax)
+{
+#pragma unroll 1
+    for (int i = 0; i < 8 * n_tiles; i += 2) {
+        uint8_t *row = tiles + (i >> 3) * 8192 + u * 128;
+        const float fi = (i >> 3) < n_scaled ? f : 1.f;
+        const uint32_t o0 = (uint32_t)((((i & 7) + u) & 7) << 4), o1 = (uint32_t)((((i & 7) + 1 + u) & 7) << 4);
+        const uint4 a = lds128(row + o0), b = lds128(row + o1);
+        const uint4 ha = bf16x8_to_f16x8(a, fi), hb = bf16x8_to_f16x8(b, fi);
+        absmax = f16x8_absmax(f16x8_absmax(absmax, ha), hb);
+        sts128(row + o0, ha);
+        sts128(row + o1, hb);
+    }
+    return absmax;
 }
 
 #define GDN_DOFF(bytes) ((uint64_t)((bytes) >> 4))
@@ -285,20 +312,15 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int64_t rem = len - (int64_t)c * kC;
         return (int)(rem < kC ? rem : kC);
     };
-    auto fail = [&]() { st_cluster_u32(peer_abort, 1u); };
     // Bounded waits. A non-blocking test goes first: a blocking try_wait on a phase that
     // has already completed still costs a few hundred cycles.
     auto wait = [&](int b, int parity) -> bool {
-        if (mbar_test(&bar[b], (uint32_t)parity & 1u)) return true;
-        if (mbar_wait_bounded(&bar[b], (uint32_t)parity & 1u, abort_flag, kWaitLimit)) return true;
-        fail();
-        return false;
+        return mbar_test(&bar[b], (uint32_t)parity & 1u) ||
+               mbar_wait_or_abort(&bar[b], (uint32_t)parity & 1u, abort_flag, peer_abort, 0u, kWaitLimit);
     };
     auto wait_cl = [&](int b, int parity) -> bool {
-        if (mbar_test_cluster(&bar[b], (uint32_t)parity & 1u)) return true;
-        if (mbar_wait_cluster_bounded(&bar[b], (uint32_t)parity & 1u, abort_flag, kWaitLimit)) return true;
-        fail();
-        return false;
+        return mbar_test_cluster(&bar[b], (uint32_t)parity & 1u) ||
+               mbar_wait_or_abort(&bar[b], (uint32_t)parity & 1u, abort_flag, peer_abort, 1u, kWaitLimit);
     };
     // the same, called by a whole warp: every lane gets the same answer
     auto wait_w = [&](int b, int parity) -> bool { return __all_sync(0xffffffffu, wait(b, parity)); };
@@ -367,24 +389,16 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint32_t k_ready0 = map_to_peer(sbase + ch::OFF_BAR + ch::B_K_READY * 8, 1);
             const uint32_t lead = elect_one();    // in warp 2: the lane that issues the ring stores
             int stored = 0;
+            uint32_t ovf = 0;                     // magnitude maximum of the converted K values
             for (int c = 0; c < n_chunks; ++c) {
                 const int st = c % kSvStages;
                 bool ok = true;
                 if (u == 0) ok = wait(B_CREADY + st, c / kSvStages);
                 if (!named_bar_and(5, 64, ok)) break;
                 uint8_t *qk = smem + OFF_QK + st * QK_STAGE;
-                // A whole 128-byte row is rewritten, so the swizzle does not matter; the
-                // rotated order keeps the eight threads of a row group on distinct banks.
-                // (Rolled over the rows: this code shares the instruction cache with the solve.)
-#pragma unroll 1
-                for (int w2 = 0; w2 < 2; ++w2) {
-                    uint8_t *row = qk + w2 * 16384 + u * 128;
-                    uint4 v[8];
-#pragma unroll
-                    for (int it = 0; it < 8; ++it) v[it] = lds128(row + (((it + u) & 7) << 4));
-#pragma unroll
-                    for (int it = 0; it < 8; ++it) sts128(row + (((it + u) & 7) << 4), bf16x8_to_f16x8(v[it], 1.f));
-                }
+                // the K tiles are [K d0..63 | Q d0..63 | K d64..127 | Q d64..]: tiles 0 and 2
+                ovf = convert_rows_bf16_f16(qk, 1, 0, 1.f, u, ovf);
+                ovf = convert_rows_bf16_f16(qk + 16384, 1, 0, 1.f, u, ovf);
                 fence_proxy_async_smem();
                 // the ring slot is free once the chain CTA has loaded chunk c - kRing
                 ok = true;
@@ -405,6 +419,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 stored = c + 1;
             }
+            if (f16x2_overflowed(ovf)) raise_error(kErrCheck);
             if (warp == 2 && stored > 0) {
                 bulk_wait_all();
                 fence_proxy_async_global();
@@ -434,6 +449,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             };
             if (gate_warp && j < n_chunks) load_gates(j);
             int n_sent[kRecv] = {};
+            uint32_t ovf = 0;                         // magnitude maximum of the fp16 operands sent
             for (int c = j; c < n_chunks; c += 2) {
                 if (gate_warp) {
                     float g_lo, g_hi;
@@ -516,7 +532,9 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         stsf4(Ls + t * LS_LD + s8, make_float4(v[0], v[1], v[2], v[3]));
                         stsf4(Ls + t * LS_LD + s8 + 4, make_float4(v[4], v[5], v[6], v[7]));
                     } else {
-                        sts128(send + 16384 + sw128_off(t, s8 >> 3), pack8_f16(v));
+                        const uint4 h = pack8_f16(v);
+                        ovf = f16x8_absmax(ovf, h);
+                        sts128(send + 16384 + sw128_off(t, s8 >> 3), h);
                     }
                 }
                 named_bar_sync(nb, 128);
@@ -635,7 +653,9 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const float4 c1 = r < 64 ? ldsf4(gam + s8 + 4) : make_float4(1.f, 1.f, 1.f, 1.f);
                     const float v[8] = {t0.x * b0.x * c0.x, t0.y * b0.y * c0.y, t0.z * b0.z * c0.z, t0.w * b0.w * c0.w,
                                         t1.x * b1.x * c1.x, t1.y * b1.y * c1.y, t1.z * b1.z * c1.z, t1.w * b1.w * c1.w};
-                    sts128(send + (r < 64 ? 0 : 8192) + sw128_off(t, s8 >> 3), pack8_f16(v));
+                    const uint4 h = pack8_f16(v);
+                    ovf = f16x8_absmax(ovf, h);
+                    sts128(send + (r < 64 ? 0 : 8192) + sw128_off(t, s8 >> 3), h);
                 }
                 fence_proxy_async_smem();
                 // then one copy into the chain CTA's slot c % kRecv, once it has finished the
@@ -652,6 +672,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 ++n_sent[slot];
             }
+            if (f16x2_overflowed(ovf)) raise_error(kErrCheck);
             // the chain CTA drains this group's copies before either CTA exits
             if (r == 0)
                 for (int sl = 0; sl < kRecv; ++sl)
@@ -815,6 +836,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 la1 = lane + 32 < nv ? log_alpha[(size_t)(tok0 + lane + 32) * H + head] : 0.f;
             };
             if (n_chunks > 0) load_la(0);
+            uint32_t ovf = 0;                     // magnitude maximum of the converted (scaled) Q, V values
             for (int c = 0; c < n_chunks; ++c) {
                 const int st = c % kQVStages;
                 float g_lo, g_hi;
@@ -825,23 +847,12 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (u == 0) ok = wait(B_QV_FULL + st, c / kQVStages);
                 if (!named_bar_and(3, 64, ok)) break;
                 uint8_t *qv = smem + OFF_QV + st * QV_STAGE;
-                // A whole 128-byte row is rewritten, so the swizzle does not matter; the
-                // rotated order keeps the eight threads of a row group on distinct banks.
-                // (Rolled over the four rows: this code shares the instruction cache with the
-                // epilogue.)
-#pragma unroll 1
-                for (int w4 = 0; w4 < 4; ++w4) {
-                    uint8_t *row = qv + w4 * 8192 + u * 128;
-                    const float f = w4 < 2 ? fq : 1.f;
-                    uint4 v[8];
-#pragma unroll
-                    for (int it = 0; it < 8; ++it) v[it] = lds128(row + (((it + u) & 7) << 4));
-#pragma unroll
-                    for (int it = 0; it < 8; ++it) sts128(row + (((it + u) & 7) << 4), bf16x8_to_f16x8(v[it], f));
-                }
+                // [Q d0..63 | Q d64.. | V d0..63 | V d64..]: Q scaled by gamma_u * scale
+                ovf = convert_rows_bf16_f16(qv, 4, 2, fq, u, ovf);
                 fence_proxy_async_smem();
                 mbar_arrive(&bar[B_CONV + st]);
             }
+            if (f16x2_overflowed(ovf)) raise_error(kErrCheck);
         } else {
             // ============================================================ epilogue warpgroups
             const int hh = (warp - 4) >> 2;           // column half of every accumulator
@@ -862,19 +873,26 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (r == 0) ok = wait(b, parity);
                 return named_bar_and(nb, 128, ok);
             };
+            // magnitude maxima of the values converted to fp16 operands here: -W^T and U~^T
+            // (packed fp16, f16x2_absmax) and the state copy (fp32, NaN-propagating)
+            uint32_t h16max = 0;
+            float fmax16 = 0.f;
             // -W^T of chunk c: this half's 32 columns t of W^T into rows k = r of the operand
+            // (off the recursion's critical path: rolled, eight columns at a time)
             auto do_wb = [&](int c) -> bool {
                 if (!group_wait(B_WFULL, c)) return false;
                 tc_fence_after();
-                uint32_t wv[32];
-                tmem_ld_x32(tmem + lane_base + TM_W + 32 * hh, wv);
-                tmem_wait_ld();
-#pragma unroll
+#pragma unroll 1
                 for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t wv[8];
+                    tmem_ld_x8(tmem + lane_base + TM_W + 32 * hh + 8 * c4, wv);
+                    tmem_wait_ld();
                     float v8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v8[e] = -__uint_as_float(wv[c4 * 8 + e]);
-                    sts128(smem + OFF_WB + sw128_off(r, 4 * hh + c4), pack8_f16(v8));
+                    for (int e = 0; e < 8; ++e) v8[e] = -__uint_as_float(wv[e]);
+                    const uint4 h = pack8_f16(v8);
+                    h16max = f16x8_absmax(h16max, h);
+                    sts128(smem + OFF_WB + sw128_off(r, 4 * hh + c4), h);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -909,8 +927,11 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             sv[i + 3] = __float_as_uint(f.w);
                         }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
+                        for (int i = 0; i < 16; ++i) {
+                            fmax16 = max_abs_nan(fmax16, __uint_as_float(sv[2 * i]));
+                            fmax16 = max_abs_nan(fmax16, __uint_as_float(sv[2 * i + 1]));
                             sp[i] = pack_f16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+                        }
                         tmem_st_x16(tmem + lane_base + TM_SB + 32 * hh + 16 * q2, sp);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gC);
@@ -964,10 +985,13 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     tmem_st_x16(tmem + lane_base + TM_UB + 16 * hh, pu);
                     tmem_st_x16(tmem + lane_base + TM_UD + 16 * hh, pd);
                     tmem_wait_st();
+                    tc_fence_before();
+                    named_bar_arrive(NB_S_TRIG, NB_TRIG_THREADS);   // S(c)
+                    ++n_strig;
+                    // range check of U~ (the decayed copy is no larger), after the trigger
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) h16max = f16x2_absmax(h16max, pu[i]);
                 }
-                tc_fence_before();
-                named_bar_arrive(NB_S_TRIG, NB_TRIG_THREADS);   // S(c)
-                ++n_strig;
                 // -W^T of the next chunk while S(c) runs
                 if (!last && !do_wb(c + 1)) break;
                 // E3: the fp16 state copy of S_{c+1} and the fp32 state rescaled by the next
@@ -1018,6 +1042,9 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         tc_fence_before();
                         named_bar_arrive(NB_X_TRIG, NB_TRIG_THREADS);   // X(c+1)
                         ++n_xtrig;
+                        // range check of the state copy, after the trigger
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) h16max = f16x2_absmax(f16x2_absmax(h16max, pa[i]), pb[i]);
                     }
                 }
                 // y: tokens [32 hh, 32 hh + 32) of Y^T (lane v of each warp). A full chunk goes
@@ -1086,30 +1113,39 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         }
                     }
                 } else {
-                    uint32_t ya[32];
-                    tmem_ld_x32(tmem + lane_base + TM_Y + (c & 1) * 64 + 32 * hh, ya);
-                    tmem_wait_ld();
-                    if (n_valid == kC) {
-                        // the previous chunk's store has read the staging tile (it had a whole
-                        // chunk to do so)
+                    // eight tokens at a time (off the critical path: rolled). A full chunk: the
+                    // staging tile, once the previous chunk's store has read it (it had a whole
+                    // chunk to do so), then one TMA store; a partial one: row by row.
+                    const bool full = n_valid == kC;
+                    if (full) {
                         if (r == 0) bulk_wait_read();
                         named_bar_sync(nb, 128);
-                        TY *ys = reinterpret_cast<TY *>(smem + OFF_YST + hh * YST_HALF);
+                    }
+                    const int nv = full ? 32 : n_valid - 32 * hh;
+                    TY *ys = reinterpret_cast<TY *>(smem + OFF_YST + hh * YST_HALF);
+                    TY *yp = y + ((size_t)(tok0 + 32 * hh) * H + head) * kD + r;
+                    const size_t ystride = (size_t)H * kD;
+#pragma unroll 1
+                    for (int j8 = 0; j8 < 32; j8 += 8) {
+                        uint32_t ya[8];
+                        tmem_ld_x8(tmem + lane_base + TM_Y + (c & 1) * 64 + 32 * hh + j8, ya);
+                        tmem_wait_ld();
 #pragma unroll
-                        for (int jt = 0; jt < 32; ++jt) ys[jt * kD + r] = from_f32<TY>(__uint_as_float(ya[jt]));
+                        for (int e = 0; e < 8; ++e) {
+                            const TY v = from_f32<TY>(__uint_as_float(ya[e]));
+                            if (full)
+                                ys[(j8 + e) * kD + r] = v;
+                            else if (j8 + e < nv)
+                                yp[(size_t)(j8 + e) * ystride] = v;
+                        }
+                    }
+                    if (full) {
                         fence_proxy_async_smem();
                         named_bar_sync(nb, 128);
                         if (r == 0) {
                             tma_store_3d(&tm_y, ys, 0, head, (int)(tok0 + 32 * hh));
                             bulk_commit();
                         }
-                    } else {
-                        const int nv = n_valid - 32 * hh;
-                        TY *yp = y + ((size_t)(tok0 + 32 * hh) * H + head) * kD + r;
-                        const size_t ystride = (size_t)H * kD;
-#pragma unroll
-                        for (int jt = 0; jt < 32; ++jt)
-                            if (jt < nv) yp[jt * ystride] = from_f32<TY>(__uint_as_float(ya[jt]));
                     }
                 }
                 g_lo = n_lo;
@@ -1119,6 +1155,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // waiting for
             if (n_strig < n_chunks) named_bar_arrive(NB_S_TRIG, NB_TRIG_THREADS);
             if (n_xtrig < n_chunks) named_bar_arrive(NB_X_TRIG, NB_TRIG_THREADS);
+            if (!(fmax16 < kF16Limit) || f16x2_overflowed(h16max)) raise_error(kErrCheck);
             if (r == 0) bulk_wait_all();          // y stores complete before the CTA exits
         }
     }

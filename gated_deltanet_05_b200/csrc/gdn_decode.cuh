@@ -21,11 +21,11 @@ namespace gdn {
 
 constexpr int kDecodeThreads = 256;
 
-template <int DK, typename T>
+template <int DK, typename T, typename TY>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                    const float *__restrict__ alpha, const float *__restrict__ beta,
-                   float *__restrict__ S, int dv, float scale, T *__restrict__ y)
+                   float *__restrict__ S, int dv, float scale, TY *__restrict__ y)
 {
     constexpr int LPR = DK / 4;              // lanes per row
     constexpr int RPW = 32 / LPR;            // rows per warp pass
@@ -45,7 +45,7 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
 
     float *Sc = S + (size_t)chain * dv * DK;
     const T *vc = v + (size_t)chain * dv;
-    T *yc = y + (size_t)chain * dv;
+    TY *yc = y + (size_t)chain * dv;
 
     const int rows_per_round = WARPS * RPW * ROWS_IN_FLIGHT;
     for (int base = 0; base < dv; base += rows_per_round) {
@@ -79,7 +79,7 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
                 sn.w = fmaf(a, s[i].w, be * kv.w);
                 store4(Sc + (size_t)row[i] * DK + 4 * part, sn);
                 if (part == 0)
-                    yc[row[i]] = from_f32<T>(fmaf(a, r, be * kq));
+                    yc[row[i]] = from_f32<TY>(fmaf(a, r, be * kq));
             }
         }
     }
@@ -100,11 +100,11 @@ namespace gdn {
 constexpr int kDecodeMaxTokens = 8;
 constexpr int kDecodeTokThreads = 256;
 
-template <int DK, typename T>
+template <int DK, typename T, typename TY>
 __global__ void __launch_bounds__(kDecodeTokThreads)
 decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                      const float *__restrict__ alpha, const float *__restrict__ beta,
-                     float *__restrict__ S, int n, int H, int dv, float scale, T *__restrict__ y)
+                     float *__restrict__ S, int n, int H, int dv, float scale, TY *__restrict__ y)
 {
     constexpr int LPR = DK / 16;             // lanes per row, 16 elements each
     constexpr int RPW = 32 / LPR;            // rows per warp pass
@@ -188,7 +188,7 @@ decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
                 const float be = b * ev;
 #pragma unroll
                 for (int e = 0; e < 16; ++e) s[f][e] = fmaf(a, s[f][e], be * kv[e]);
-                if (valid && part == 0) y[tok_row(i) * dv + row[f]] = from_f32<T>(fmaf(a, r, be * kq));
+                if (valid && part == 0) y[tok_row(i) * dv + row[f]] = from_f32<TY>(fmaf(a, r, be * kq));
             }
         }
 #pragma unroll

@@ -110,14 +110,40 @@ gdn_status launch_chunk_f32(const void *q, const void *k, const void *v, const f
     return launch_status();
 }
 
-// Number of SM ids of the current device (the tensor-core kernel's workspace has one
-// region per SM id); 0 if the device cannot be queried.
-int device_sm_count()
+// Number of SM ids of the current device. The tensor-core kernel's workspace has one
+// region per SM id, and SM ids (%smid) run up to %nsmid - 1, which may exceed the SM count
+// (ids need not be contiguous). %nsmid is read once per device by a one-thread kernel
+// (followed by a synchronous copy, so the first query on a device synchronises it and
+// must not happen inside a stream capture); the result is the larger of it and the SM
+// count. 0 if the device cannot be queried.
+__device__ unsigned int g_nsmid_word;
+
+__global__ void nsmid_kernel()
+{
+    unsigned int n;
+    asm volatile("mov.u32 %0, %%nsmid;" : "=r"(n));
+    g_nsmid_word = n;
+}
+
+constexpr int kMaxDevices = 64;
+int g_sm_ids[kMaxDevices] = {};
+std::mutex g_sm_ids_mutex;
+
+int device_sm_ids()
 {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    return n;
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    std::lock_guard<std::mutex> lock(g_sm_ids_mutex);
+    if (g_sm_ids[dev] > 0) return g_sm_ids[dev];
+    nsmid_kernel<<<1, 1>>>();
+    unsigned int ids = 0;
+    if (cudaGetLastError() != cudaSuccess ||
+        cudaMemcpyFromSymbol(&ids, g_nsmid_word, sizeof(ids)) != cudaSuccess)
+        return 0;
+    g_sm_ids[dev] = (int)ids > n ? (int)ids : n;
+    return g_sm_ids[dev];
 }
 
 // Device check of the kernels' bounded mbarrier wait (gdn_selftest_bounded_wait). Thread 0
@@ -163,10 +189,15 @@ gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const
                               size_t ws_bytes, cudaStream_t st, const void *z = nullptr,
                               const float *gn_w = nullptr, float gn_eps = 0.f)
 {
-    const int n_sm = device_sm_count();
-    if (n_sm <= 0) return GDN_ERR_CUDA;
-    if (!ws || !aligned(ws, 128) || ws_bytes < (size_t)n_sm * gdn::sm100::kWsBytesPerSm)
+    const int n_ids = device_sm_ids();
+    if (n_ids <= 0) return GDN_ERR_CUDA;
+    if (!ws || !aligned(ws, 128) || ws_bytes < (size_t)n_ids * gdn::sm100::kWsBytesPerSm)
         return GDN_ERR_INVALID_ARG;
+    if (2 * (int64_t)n_seq * H > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    // every region the workspace holds may serve an SM id (the kernel checks its own id
+    // against this count and records GDN_ERR_DEVICE_CHECK if it falls outside)
+    const size_t slots = ws_bytes / gdn::sm100::kWsBytesPerSm;
+    const int ws_slots = slots > 0x7fffffff ? 0x7fffffff : (int)slots;
     CUtensorMap mq, mk, mv, my;
     if (!make_map(&mq, q, n_tok, H) || !make_map(&mk, k, n_tok, H) || !make_map(&mv, v, n_tok, H) ||
         !make_y_map(&my, y, n_tok, H, sizeof(TY) == 4))
@@ -180,7 +211,7 @@ gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const
     const unsigned grid = (unsigned)(2 * (int64_t)n_seq * H);
     kern<<<grid, gdn::sm100::kThreads, smem, st>>>(mq, mk, mv, my, la, beta, S0, cu, n_seq, H, scale,
                                                    static_cast<TY *>(y), S_T,
-                                                   static_cast<uint8_t *>(ws), n_sm,
+                                                   static_cast<uint8_t *>(ws), ws_slots,
                                                    static_cast<const __nv_bfloat16 *>(z), gn_w, gn_eps);
     return launch_status();
 }
@@ -209,7 +240,7 @@ size_t gdn_chunk_fwd_workspace_bytes(int n_seq, int64_t total_tokens, int H, int
 {
     (void)n_seq; (void)total_tokens; (void)H;
     if (d_k != 128 || d_v != 128 || chunk != 64) return 0;
-    return (size_t)device_sm_count() * gdn::sm100::kWsBytesPerSm;
+    return (size_t)device_sm_ids() * gdn::sm100::kWsBytesPerSm;
 }
 
 gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
@@ -359,18 +390,19 @@ gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gd
                                  int n_seq, int H, int d_k, int d_v, int chunk, float scale, void *y,
                                  gdn_dtype y_dtype, float *S_T, void *stream)
 {
-    // the fixed array covers kNoAllocMaxSms SM ids of the current device
-    size_t need = 0;
+    // the fixed array covers kNoAllocMaxSms SM ids of the current device; all of it is
+    // offered to the kernel
+    size_t have = 0;
     if (d_k == 128 && d_v == 128 && chunk == 64) {
-        const int n_sm = device_sm_count();
-        if (n_sm <= 0) return GDN_ERR_CUDA;
-        if (n_sm > kNoAllocMaxSms) return GDN_ERR_UNSUPPORTED;
-        need = (size_t)n_sm * gdn::sm100::kWsBytesPerSm;
+        const int n_ids = device_sm_ids();
+        if (n_ids <= 0) return GDN_ERR_CUDA;
+        if (n_ids > kNoAllocMaxSms) return GDN_ERR_UNSUPPORTED;
+        have = sizeof(g_noalloc_ws);
     }
     void *ws = nullptr;
-    if (need > 0 && cudaGetSymbolAddress(&ws, g_noalloc_ws) != cudaSuccess) return GDN_ERR_CUDA;
+    if (have > 0 && cudaGetSymbolAddress(&ws, g_noalloc_ws) != cudaSuccess) return GDN_ERR_CUDA;
     return gdn_chunk_fwd(q, k, v, in_dtype, log_alpha, beta, S0, cu_seqlens_dev, cu_seqlens_host, n_seq, H,
-                         d_k, d_v, chunk, scale, y, y_dtype, S_T, ws, need, stream);
+                         d_k, d_v, chunk, scale, y, y_dtype, S_T, ws, have, stream);
 }
 
 gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *stream)
@@ -383,10 +415,11 @@ gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *strea
 
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
                            const float *alpha, const float *beta, float *S, int n_seq, int H,
-                           int d_k, int d_v, float scale, void *y, void *stream)
+                           int d_k, int d_v, float scale, void *y, gdn_dtype y_dtype, void *stream)
 {
     if (n_seq < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (y_dtype != GDN_F32 && y_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (!pow2_in(d_k, 16, 128) || !pow2_in(d_v, 16, 128)) return GDN_ERR_UNSUPPORTED;
     const int64_t n_chain = (int64_t)n_seq * H;
     if (n_chain == 0) return GDN_OK;
@@ -398,16 +431,18 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
         return GDN_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     const unsigned grid = (unsigned)n_chain;
+#define GDN_DECODE_LAUNCH(DK, T, TY)                                                               \
+    gdn::decode_step_kernel<DK, T, TY><<<grid, gdn::kDecodeThreads, 0, st>>>(                      \
+        (const T *)q, (const T *)k, (const T *)v, alpha, beta, S, d_v, scale, (TY *)y)
 #define GDN_DECODE_CASE(DK)                                                                        \
     case DK:                                                                                       \
-        if (in_dtype == GDN_F32)                                                                   \
-            gdn::decode_step_kernel<DK, float><<<grid, gdn::kDecodeThreads, 0, st>>>(              \
-                (const float *)q, (const float *)k, (const float *)v, alpha, beta, S, d_v, scale,  \
-                (float *)y);                                                                       \
-        else                                                                                       \
-            gdn::decode_step_kernel<DK, __nv_bfloat16><<<grid, gdn::kDecodeThreads, 0, st>>>(      \
-                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,      \
-                alpha, beta, S, d_v, scale, (__nv_bfloat16 *)y);                                   \
+        if (in_dtype == GDN_F32) {                                                                 \
+            if (y_dtype == GDN_F32) GDN_DECODE_LAUNCH(DK, float, float);                           \
+            else GDN_DECODE_LAUNCH(DK, float, __nv_bfloat16);                                      \
+        } else {                                                                                   \
+            if (y_dtype == GDN_F32) GDN_DECODE_LAUNCH(DK, __nv_bfloat16, float);                   \
+            else GDN_DECODE_LAUNCH(DK, __nv_bfloat16, __nv_bfloat16);                              \
+        }                                                                                          \
         break;
     switch (d_k) {
         GDN_DECODE_CASE(16)
@@ -417,17 +452,19 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
     default: return GDN_ERR_UNSUPPORTED;
     }
 #undef GDN_DECODE_CASE
+#undef GDN_DECODE_LAUNCH
     return launch_status();
 }
 
 gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
                              const float *alpha, const float *beta, float *S, int n_seq,
                              int n_tokens, int H, int d_k, int d_v, float scale, void *y,
-                             void *stream)
+                             gdn_dtype y_dtype, void *stream)
 {
     if (n_seq < 0 || H <= 0 || n_tokens < 1 || n_tokens > gdn::kDecodeMaxTokens)
         return GDN_ERR_INVALID_ARG;
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (y_dtype != GDN_F32 && y_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (!pow2_in(d_k, 16, 128) || !pow2_in(d_v, 16, 128)) return GDN_ERR_UNSUPPORTED;
     const int64_t n_chain = (int64_t)n_seq * H;
     if (n_chain == 0) return GDN_OK;
@@ -439,16 +476,18 @@ gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dt
         return GDN_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     const unsigned grid = (unsigned)n_chain;
+#define GDN_DECTOK_LAUNCH(DK, T, TY)                                                               \
+    gdn::decode_tokens_kernel<DK, T, TY><<<grid, gdn::kDecodeTokThreads, 0, st>>>(                 \
+        (const T *)q, (const T *)k, (const T *)v, alpha, beta, S, n_tokens, H, d_v, scale, (TY *)y)
 #define GDN_DECTOK_CASE(DK)                                                                        \
     case DK:                                                                                       \
-        if (in_dtype == GDN_F32)                                                                   \
-            gdn::decode_tokens_kernel<DK, float><<<grid, gdn::kDecodeTokThreads, 0, st>>>(         \
-                (const float *)q, (const float *)k, (const float *)v, alpha, beta, S, n_tokens, H, \
-                d_v, scale, (float *)y);                                                           \
-        else                                                                                       \
-            gdn::decode_tokens_kernel<DK, __nv_bfloat16><<<grid, gdn::kDecodeTokThreads, 0, st>>>( \
-                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,      \
-                alpha, beta, S, n_tokens, H, d_v, scale, (__nv_bfloat16 *)y);                      \
+        if (in_dtype == GDN_F32) {                                                                 \
+            if (y_dtype == GDN_F32) GDN_DECTOK_LAUNCH(DK, float, float);                           \
+            else GDN_DECTOK_LAUNCH(DK, float, __nv_bfloat16);                                      \
+        } else {                                                                                   \
+            if (y_dtype == GDN_F32) GDN_DECTOK_LAUNCH(DK, __nv_bfloat16, float);                   \
+            else GDN_DECTOK_LAUNCH(DK, __nv_bfloat16, __nv_bfloat16);                              \
+        }                                                                                          \
         break;
     switch (d_k) {
         GDN_DECTOK_CASE(16)
@@ -458,6 +497,7 @@ gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dt
     default: return GDN_ERR_UNSUPPORTED;
     }
 #undef GDN_DECTOK_CASE
+#undef GDN_DECTOK_LAUNCH
     return launch_status();
 }
 
@@ -476,7 +516,7 @@ gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dt
     cudaStream_t st = as_stream(stream);
     int dev = 0, n_sm = 148;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);   // grid sizing only
     // rows per CTA pass = 8 warps x rows-per-warp x 2 (unroll); at most 8 CTAs per SM
     const int64_t rows_per_cta = (int64_t)(gdn::kGateNormThreads / 32) * (32 / (d_v / 8)) * 2;
     int64_t blocks = (n_rows + rows_per_cta - 1) / rows_per_cta;

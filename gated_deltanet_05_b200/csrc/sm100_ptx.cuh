@@ -273,6 +273,19 @@ __device__ __noinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t p
     return true;
 }
 
+// The slow path of a kernel role's wait, out of line so that each call site stays a probe
+// and a call: a bounded wait with acquire at cluster scope (cluster != 0) or CTA scope; when
+// it gives up (a timeout, or the abort flag already raised) it also raises the other CTA's
+// abort flag (peer_abort, a shared::cluster address) so that both CTAs of the cluster stop.
+__device__ __noinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                uint32_t peer_abort, uint32_t cluster, long long limit_cycles)
+{
+    const bool ok = cluster ? mbar_wait_cluster_bounded(bar, parity, abort, limit_cycles)
+                            : mbar_wait_bounded(bar, parity, abort, limit_cycles);
+    if (!ok) asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1u) : "memory");
+    return ok;
+}
+
 // Bulk copy from this CTA's shared memory into another CTA's shared memory of the
 // cluster; completion is counted as transaction bytes on the destination's mbarrier.
 // No multicast. Addresses 16-byte aligned, size a multiple of 16.
@@ -498,6 +511,13 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16])
 {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -589,6 +609,28 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
 }
+
+// fp16 range checks. The tensor-core products take fp16 operands, which hold |x| < 65520
+// (larger values round to inf). f16x2_absmax keeps, per 16-bit half, the largest magnitude
+// bit pattern seen (sign cleared); a finite fp16 has a pattern below 0x7c00, inf and NaN do
+// not, so f16x2_overflowed tells whether any packed value converted so far overflowed.
+__device__ __forceinline__ uint32_t f16x2_absmax(uint32_t acc, uint32_t w) { return __vmaxu2(acc, w & 0x7fff7fffu); }
+__device__ __forceinline__ uint32_t f16x8_absmax(uint32_t acc, uint4 w)
+{
+    return f16x2_absmax(f16x2_absmax(acc, w.x), __vmaxu2(w.y & 0x7fff7fffu, __vmaxu2(w.z & 0x7fff7fffu, w.w & 0x7fff7fffu)));
+}
+__device__ __forceinline__ bool f16x2_overflowed(uint32_t acc)
+{
+    return (acc & 0xffffu) >= 0x7c00u || (acc >> 16) >= 0x7c00u;
+}
+// max(acc, |x|) that propagates NaN (so a NaN also fails the final range test).
+__device__ __forceinline__ float max_abs_nan(float acc, float x)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(acc), "f"(fabsf(x)));
+    return r;
+}
+constexpr float kF16Limit = 65520.f;   // fp16 round-to-nearest overflows at and above this
 
 }  // namespace sm100
 }  // namespace gdn

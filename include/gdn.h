@@ -87,20 +87,27 @@ typedef enum {
  *   S_T         [n_seq, H, d_v, d_k] fp32 out (final state per sequence), or NULL
  *   workspace   device scratch of workspace_bytes >= gdn_chunk_fwd_workspace_bytes(..),
  *               128-byte aligned (may be NULL when that is 0). The tensor-core path uses
- *               it as a ring of fp16 K tiles per SM id (SM count x 64 KB on the current
- *               device); no initial contents are needed and nothing is left in
- *               it. Calls on different streams may share one workspace (each SM id's
- *               region is used by at most one cluster at a time). Caller-owned.
+ *               it as a ring of fp16 K tiles per SM id (64 KB for each id the device's
+ *               SMs can report, %nsmid, at least the SM count); no initial contents are
+ *               needed and nothing is left in it. Calls on different streams may share one
+ *               workspace (each SM id's region is used by at most one cluster at a time).
+ *               Caller-owned. An SM id beyond the workspace's regions is recorded as
+ *               GDN_ERR_DEVICE_CHECK (gdn_device_error) and that chain is not computed.
  *
  * Paths: bf16 inputs with d_k = d_v = 128 and chunk = 64 run the sm_100a tensor-core
  * kernel (tcgen05 MMA with TMEM accumulators, TMA loads, fp32 state carry; bf16 inputs
  * feed the K K^T / Q K^T product, all other products use fp16 operands -- the inputs
- * convert exactly -- which requires |q|, |k|, |v| and the state entries below 65504);
- * every other supported case runs the CUDA-core fp32 chunk kernel.
+ * convert exactly -- which requires the scaled q, k, v, S0, the state and the derived
+ * operands to stay below 65520 in magnitude; the kernel checks every value it converts and
+ * records GDN_ERR_DEVICE_CHECK (gdn_device_error) when one does not, or is NaN: the
+ * outputs of that call are then unspecified); every other supported case runs the
+ * CUDA-core fp32 chunk kernel.
  */
-/* Scratch bytes gdn_chunk_fwd needs for these sizes on the current device: SM count x
- * 64 KB when d_k = d_v = 128 and chunk = 64 (the tensor-core path; sized for any input
- * dtype), else 0. Returns 0 when no device can be queried. */
+/* Scratch bytes gdn_chunk_fwd needs for these sizes on the current device: 64 KB per SM
+ * id when d_k = d_v = 128 and chunk = 64 (the tensor-core path; sized for any input
+ * dtype), else 0. Returns 0 when no device can be queried. The first call on a device reads
+ * its SM id range with a one-thread kernel and a synchronous copy (once per device and
+ * process): make it before any stream capture. */
 size_t gdn_chunk_fwd_workspace_bytes(int n_seq, int64_t total_tokens, int H, int d_k, int d_v,
                                      int chunk);
 
@@ -119,8 +126,9 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, gdn_dtype 
  * Same arguments, results and errors as gdn_chunk_fwd, minus workspace. The scratch of
  * the tensor-core path is a fixed file-scope device array of the library (one per
  * device, 160 SM ids x 64 KB = 10 MB, reached through cudaGetSymbolAddress); the call
- * allocates and frees nothing. A device with more than 160 SMs returns
- * GDN_ERR_UNSUPPORTED. The array is shared by every call in the process: overlapping
+ * allocates and frees nothing. A device whose SM ids (%nsmid) exceed 160 returns
+ * GDN_ERR_UNSUPPORTED. The first call on a device reads that range once (a one-thread
+ * kernel and a synchronous copy): make it before any stream capture. The array is shared by every call in the process: overlapping
  * calls on different streams do not race only because each SM id's region is used by at
  * most one cluster at a time (one cluster's solver CTA occupies an SM), the same
  * property that lets gdn_chunk_fwd callers share one workspace.
@@ -206,12 +214,14 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
  *   q, k   [n_seq, H, d_k] in in_dtype;  v [n_seq, H, d_v] in in_dtype
  *   alpha  [n_seq, H] fp32 in (0, 1];  beta [n_seq, H] fp32 in [0, 1]
  *   S      [n_seq, H, d_v, d_k] fp32, read and overwritten with the new state
- *   y      [n_seq, H, d_v] out, in in_dtype
+ *   y      [n_seq, H, d_v] out, in y_dtype (GDN_F32 or GDN_BF16, independent of
+ *          in_dtype; a bf16 y is the round-to-nearest-even of the fp32 result)
  *   d_k, d_v each in {16, 32, 64, 128}
  */
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
                            const float *alpha, const float *beta, float *S, int n_seq, int H,
-                           int d_k, int d_v, float scale, void *y, void *stream);
+                           int d_k, int d_v, float scale, void *y, gdn_dtype y_dtype,
+                           void *stream);
 
 /*
  * gdn_decode_tokens -- n_tokens consecutive tokens for each of n_seq * H chains, in place,
@@ -225,7 +235,8 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
  *   q, k   [n_seq * n_tokens, H, d_k] in in_dtype;  v [n_seq * n_tokens, H, d_v] in in_dtype
  *   alpha  [n_seq * n_tokens, H] fp32 in (0, 1];  beta [n_seq * n_tokens, H] fp32 in [0, 1]
  *   S      [n_seq, H, d_v, d_k] fp32, read and overwritten with the state after the last token
- *   y      [n_seq * n_tokens, H, d_v] out, in in_dtype
+ *   y      [n_seq * n_tokens, H, d_v] out, in y_dtype (GDN_F32 or GDN_BF16, independent
+ *          of in_dtype; a bf16 y is the round-to-nearest-even of the fp32 result)
  *   1 <= n_tokens <= 8; d_k, d_v each in {16, 32, 64, 128}
  * The pages run decode with several tokens per step (pwwt.cn translation, Figure 6
  * settings: next_n = 4) but give no kernel for it.
@@ -233,7 +244,7 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
 gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
                              const float *alpha, const float *beta, float *S, int n_seq,
                              int n_tokens, int H, int d_k, int d_v, float scale, void *y,
-                             void *stream);
+                             gdn_dtype y_dtype, void *stream);
 
 /*
  * gdn_gate_norm -- the output epilogue o = sigmoid(z) * RMSNorm(y) * (1 + w).

@@ -20,6 +20,15 @@ def rel_err(got, ref) -> float:
     return float(np.max(np.abs(got - ref)) / rms)
 
 
+def assert_is_rounding(lo: torch.Tensor, hi: torch.Tensor):
+    """lo (bf16) is the round-to-nearest-even of hi (fp32), to within one bf16 ulp where
+    two launches' fp32 values could differ in the last bit."""
+    want = hi.to(torch.bfloat16)
+    same = lo.view(torch.int16) == want.view(torch.int16)
+    ulp = (lo.float() - want.float()).abs() <= want.float().abs() * 2.0 ** -7 + 1e-30
+    assert bool(same.float().mean() > 0.999) and bool(ulp.all())
+
+
 def f64(t) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
@@ -59,3 +68,30 @@ def to_dev(inp: dict, device="cuda") -> dict:
     for key, val in inp.items():
         out[key] = val.to(device) if isinstance(val, torch.Tensor) else val
     return out
+
+
+def check_all_chains(inp: dict, y, S_T, tol: float, scale: float = 1.0, head_group: int = 8,
+                     out_fn=None):
+    """Every (sequence, head) chain of a full workload against the oracle, element by
+    element: y (or out_fn(y_ref, heads) when given, e.g. the gated output) and the final
+    states. Heads are taken head_group at a time to bound host memory. Returns the worst
+    (y error, state error)."""
+    H = inp["q"].shape[1]
+    seqs = list(range(inp["cu_seqlens"].numel() - 1))
+    worst_y = worst_s = 0.0
+    y = y.cpu()
+    S_T = None if S_T is None else S_T.cpu()
+    for h0 in range(0, H, head_group):
+        heads = list(range(h0, min(H, h0 + head_group)))
+        sub, _, hs = subset(inp, seqs, heads)
+        y_ref, S_ref = oracle_prefill(sub, scale)
+        if out_fn is not None:
+            y_ref = out_fn(y_ref, sub)
+        ey = rel_err(f64(y.index_select(1, hs)), y_ref)
+        worst_y = max(worst_y, ey)
+        assert ey <= tol, (heads, ey)
+        if S_T is not None:
+            es = rel_err(f64(S_T[:, heads]), S_ref)
+            worst_s = max(worst_s, es)
+            assert es <= tol, (heads, es)
+    return worst_y, worst_s

@@ -99,8 +99,11 @@ def test_selftest_rejects_bad_arguments(L):
 def test_decode_and_gate_norm_reject_bad_arguments(L):
     dec = lambda **kw: L.gdn_decode_step(kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 0), FAKE,
                                          FAKE, kw.get("S", FAKE), kw.get("n", 4), kw.get("H", 2),
-                                         kw.get("dk", 128), kw.get("dv", 128), 1.0, FAKE, None)
+                                         kw.get("dk", 128), kw.get("dv", 128), 1.0, FAKE,
+                                         kw.get("ydt", 0), None)
     assert dec(n=-1) == 1
+    assert dec(ydt=2) == 1
+    assert dec(dt=2) == 1
     assert dec(H=0) == 1
     assert dec(dk=48) == 2
     assert dec(dv=512) == 2
@@ -174,8 +177,9 @@ def test_decode_tokens_rejects_bad_arguments(L):
     dt = lambda **kw: L.gdn_decode_tokens(kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 0), FAKE, FAKE,
                                           kw.get("S", FAKE), kw.get("n", 4), kw.get("nt", 4),
                                           kw.get("H", 2), kw.get("dk", 128), kw.get("dv", 128), 1.0,
-                                          FAKE, None)
+                                          FAKE, kw.get("ydt", 1), None)
     assert dt(nt=0) == 1
+    assert dt(ydt=3) == 1
     assert dt(nt=9) == 1
     assert dt(n=-1) == 1
     assert dt(H=0) == 1

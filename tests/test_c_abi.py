@@ -21,7 +21,7 @@ int main(void)
     if (strcmp(gdn_status_string(GDN_ERR_TIMEOUT), "GDN_ERR_TIMEOUT") != 0) return 2;
     if (gdn_backward_workspace_bytes(cu, 2, 2, 16, 16) != (size_t)2 * 2 * (1 + 1 + 65) * 16 * 16 * 4) return 3;
     /* rejected before any launch: an unsupported head size, an unknown dtype */
-    if (gdn_decode_step(0, 0, 0, GDN_F32, 0, 0, 0, 1, 1, 48, 16, 1.f, 0, 0) != GDN_ERR_UNSUPPORTED) return 4;
+    if (gdn_decode_step(0, 0, 0, GDN_F32, 0, 0, 0, 1, 1, 48, 16, 1.f, 0, GDN_F32, 0) != GDN_ERR_UNSUPPORTED) return 4;
     if (gdn_gate_norm(0, (gdn_dtype)7, 0, GDN_F32, 0, 4, 16, 1e-6f, 0, GDN_F32, 0) != GDN_ERR_INVALID_ARG) return 5;
     printf("ok %d\n", gdn_version());
     return 0;

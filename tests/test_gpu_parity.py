@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import workloads as W
-from tests.helpers import TOL, f64, oracle_prefill, rel_err, to_dev
+from tests.helpers import TOL, assert_is_rounding, f64, oracle_prefill, rel_err, to_dev
 
 gdn = pytest.importorskip("gated_deltanet_05_b200")
 
@@ -35,15 +35,6 @@ def run_prefill(inp, scale=1.0, final_state=True, y_dtype=torch.float32):
                            y_dtype=y_dtype)
     torch.cuda.synchronize()
     return y.cpu(), (None if S_T is None else S_T.cpu())
-
-
-def assert_is_rounding(lo: torch.Tensor, hi: torch.Tensor):
-    """lo (bf16) is the round-to-nearest-even of hi (fp32), to within one bf16 ulp where
-    two launches' fp32 values could differ in the last bit."""
-    want = hi.to(torch.bfloat16)
-    same = lo.view(torch.int16) == want.view(torch.int16)
-    ulp = (lo.float() - want.float()).abs() <= want.float().abs() * 2.0 ** -7 + 1e-30
-    assert bool(same.float().mean() > 0.999) and bool(ulp.all())
 
 
 def check_prefill(inp, scale=1.0, tol=None):
@@ -98,10 +89,16 @@ def test_decode_small(d, dtype):
         x = W.make_decode_inputs(w, step, n_seq=n, H=H, d=d)
         cast = (lambda t: t.to(torch.bfloat16)) if dtype == "bf16" else (lambda t: t)
         q, k, v = cast(x["q"]), cast(x["k"]), cast(x["v"])
+        S_before = Sd.clone()
         y = gdn.decode_step(q.cuda(), k.cuda(), v.cuda(), x["alpha"].cuda(), x["beta"].cuda(),
                             Sd, scale=0.9)
+        y16 = gdn.decode_step(q.cuda(), k.cuda(), v.cuda(), x["alpha"].cuda(), x["beta"].cuda(),
+                              S_before, scale=0.9, y_dtype=torch.bfloat16)
         y_ref, S_ref = oracle.decode_step(q, k, v, x["alpha"], x["beta"], S_ref, scale=0.9)
+        assert y.dtype == torch.float32
         assert rel_err(f64(y.cpu()), y_ref) <= TOL[dtype]
+        assert_is_rounding(y16.cpu(), y.cpu())        # bf16 y: the rounding of the fp32 y
+        assert torch.equal(S_before, Sd)
     assert rel_err(f64(Sd.cpu()), oracle.state_to_lib(S_ref)) <= TOL[dtype]
 
 
