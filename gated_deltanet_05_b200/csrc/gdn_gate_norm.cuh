@@ -6,9 +6,9 @@
 // and y is not mean-subtracted. One row per (token, head), over its d_v elements;
 // fp32 arithmetic, one read of y and z and one write of o (HBM-bound).
 //
-// Mapping: each lane owns 8 consecutive elements of a row (y, z and o may each be fp32 or
-// bf16); LPR = d_v / 8 lanes cover one row, a warp takes RPW = 32 / LPR rows per pass
-// and UNROLL passes at once, in a grid-stride loop over rows.
+// Mapping: each lane owns 32 bytes of y of a row (8 fp32 or 16 bf16 elements; z and o may
+// each be fp32 or bf16); LPR lanes cover one row, a warp takes RPW = 32 / LPR rows per pass
+// and UNROLL passes at once (their loads all in flight), in a grid-stride loop over rows.
 #pragma once
 #include "gdn_common.cuh"
 
@@ -49,54 +49,79 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float *x)
     *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Raw 16-byte words <-> floats: element i of a lane's run, for fp32 or bf16 storage.
+__device__ __forceinline__ float raw_elem(const uint4 *w, int i, float)
+{
+    const uint4 v = w[i >> 2];
+    const uint32_t x = (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
+    return __uint_as_float(x);
+}
+__device__ __forceinline__ float raw_elem(const uint4 *w, int i, __nv_bfloat16)
+{
+    const uint4 v = w[i >> 3];
+    const int j = (i & 7) >> 1;
+    const uint32_t x = j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+    return __uint_as_float((i & 1) ? (x & 0xffff0000u) : (x << 16));
+}
+
+// sigmoid(z) with the SM's approximate exponential and division (a few ulp of fp32)
+__device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+
 template <typename TY, typename TZ, typename TO, int DV>
 __global__ void __launch_bounds__(kGateNormThreads)
 gate_norm_kernel(const TY *__restrict__ y, const TZ *__restrict__ z, const float *__restrict__ w,
                  int64_t n_rows, float eps, TO *__restrict__ o)
 {
-    constexpr int LPR = DV / 8;                     // lanes per row, 8 elements each
-    static_assert(LPR >= 1 && LPR <= 32, "d_v in 8..256");
+    // each lane reads 32 bytes of y per row (8 fp32 or 16 bf16 elements), kept as raw words
+    // until used, so that UNROLL rows per lane are in flight at a modest register cost
+    constexpr int EPL_W = 32 / (int)sizeof(TY);
+    constexpr int EPL = DV < EPL_W ? DV : EPL_W;    // elements per lane
+    constexpr int LPR = DV / EPL;                   // lanes per row
+    static_assert(LPR >= 1 && LPR <= 32, "d_v in 16..256");
     constexpr int RPW = 32 / LPR;                   // rows per warp pass
-    constexpr int UNROLL = 2;
+    constexpr int UNROLL = 4;
+    constexpr int NY = EPL * (int)sizeof(TY) / 16, NZ = EPL * (int)sizeof(TZ) / 16;
+    static_assert(NY >= 1 && NZ >= 1, "16-byte accesses");
 
     const int lane = threadIdx.x & 31;
     const int part = lane % LPR, sub = lane / LPR;
     const int64_t warp_global = ((int64_t)blockIdx.x * kGateNormThreads + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * kGateNormThreads) >> 5;
 
-    float wp[8];
+    float wp[EPL];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) wp[e] = 1.0f + w[part * 8 + e];
+    for (int e = 0; e < EPL; ++e) wp[e] = 1.0f + w[part * EPL + e];
 
     for (int64_t r0 = warp_global * RPW * UNROLL; r0 < n_rows; r0 += n_warps * RPW * UNROLL) {
-        float yv[UNROLL][8], zv[UNROLL][8];
+        uint4 yr[UNROLL][NY], zr[UNROLL][NZ];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
             const int64_t row = r0 + u * RPW + sub;
-            if (row < n_rows) {
-                load8(y + row * DV + part * 8, yv[u]);
-                load8(z + row * DV + part * 8, zv[u]);
-            } else {
+            const uint4 *yp = reinterpret_cast<const uint4 *>(y + row * DV + part * EPL);
+            const uint4 *zp = reinterpret_cast<const uint4 *>(z + row * DV + part * EPL);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) yv[u][e] = zv[u][e] = 0.f;
-            }
+            for (int i = 0; i < NY; ++i) yr[u][i] = row < n_rows ? yp[i] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int i = 0; i < NZ; ++i) zr[u][i] = row < n_rows ? zp[i] : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
             const int64_t row = r0 + u * RPW + sub;
             float ss = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(yv[u][e], yv[u][e], ss);
+            for (int e = 0; e < EPL; ++e) {
+                const float v = raw_elem(yr[u], e, TY());
+                ss = fmaf(v, v, ss);
+            }
             ss = group_sum<LPR>(ss);
             const float inv_rms = rsqrtf(ss * (1.0f / DV) + eps);
             if (row < n_rows) {
-                float ov[8];
+                float ov[EPL];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float gate = 1.0f / (1.0f + expf(-zv[u][e]));
-                    ov[e] = gate * (yv[u][e] * inv_rms) * wp[e];
-                }
-                store8(o + row * DV + part * 8, ov);
+                for (int e = 0; e < EPL; ++e)
+                    ov[e] = fast_sigmoid(raw_elem(zr[u], e, TZ())) * (raw_elem(yr[u], e, TY()) * inv_rms) * wp[e];
+#pragma unroll
+                for (int e = 0; e < EPL; e += 8) store8(o + row * DV + part * EPL + e, ov + e);
             }
         }
     }

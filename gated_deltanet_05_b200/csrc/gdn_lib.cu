@@ -15,6 +15,9 @@
 #include "gdn_decode.cuh"
 #include "gdn_featurize.cuh"
 #include "gdn_gate_norm.cuh"
+#include "gdn_qsa.cuh"
+
+#include <cmath>
 
 namespace {
 
@@ -213,6 +216,75 @@ gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const
                                                    static_cast<TY *>(y), S_T,
                                                    static_cast<uint8_t *>(ws), ws_slots,
                                                    static_cast<const __nv_bfloat16 *>(z), gn_w, gn_eps);
+    return launch_status();
+}
+
+// ---- QSA indexer: host-side sizes (the same formulas as qsa_setup_kernel)
+struct QsaSizes {
+    int64_t n_tok = 0, n_blocks = 0, nb_max = 0, n_tiles = 0, n_ctas = 0;
+};
+
+QsaSizes qsa_sizes(const int32_t *cu, int n_seq, int r)
+{
+    QsaSizes z;
+    z.n_tok = cu[n_seq];
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t len = (int64_t)cu[s + 1] - cu[s];
+        z.n_blocks += len / r;
+        if (len / r > z.nb_max) z.nb_max = len / r;
+        const int64_t nt = (len + gdn::qsa::kTileT - 1) / gdn::qsa::kTileT;
+        z.n_tiles += nt;
+        for (int64_t i = 0; i < nt; ++i)
+            z.n_ctas += (gdn::qsa::qsa_tile_steps(len, r, i) + gdn::qsa::kMaxSteps - 1) / gdn::qsa::kMaxSteps;
+    }
+    return z;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// workspace: blk0, tile0 [n_seq + 1], cta0 [n_tiles + 1] (int32), then the query and key
+// vectors (bf16 or fp32)
+size_t qsa_ws_layout(const QsaSizes &z, int n_seq, int Hq, size_t elem, size_t *off_q, size_t *off_k)
+{
+    const size_t ints = align256(sizeof(int32_t) * ((size_t)2 * (n_seq + 1) + (size_t)z.n_tiles + 1));
+    *off_q = ints;
+    *off_k = *off_q + align256((size_t)z.n_tok * Hq * gdn::qsa::kD * elem);
+    return *off_k + align256((size_t)z.n_blocks * gdn::qsa::kD * elem);
+}
+
+// q vectors [n_tok][Hq][128] bf16 as a 3-D map, box {64, 1, 128}; key vectors [n_blocks][128]
+// bf16 as a 2-D map, box {64, 128}; both 128-byte swizzled (the MMA operand layout)
+bool make_qsa_maps(CUtensorMap *mq, CUtensorMap *mk, void *qv, void *kv, int64_t n_tok, int Hq, int64_t n_blocks)
+{
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t qd[3] = {128, (cuuint64_t)Hq, (cuuint64_t)n_tok};
+    cuuint64_t qs[2] = {256, (cuuint64_t)Hq * 256};
+    cuuint32_t qb[3] = {64, 1, 128}, e3[3] = {1, 1, 1};
+    if (enc(mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, qv, qd, qs, qb, e3, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+        return false;
+    cuuint64_t kd[2] = {128, (cuuint64_t)n_blocks};
+    cuuint64_t ks[1] = {256};
+    cuuint32_t kbx[2] = {64, 128}, e2[2] = {1, 1};
+    return enc(mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, kd, ks, kbx, e2, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int HQ>
+gdn_status launch_qsa_scores_tc(const CUtensorMap &mq, const CUtensorMap &mk, const int32_t *cu, const int32_t *blk0,
+                                const int32_t *tile0, const int32_t *cta0, int n_seq, int r, int64_t nb_max,
+                                int64_t n_ctas, float *I, cudaStream_t st)
+{
+    const int smem = (int)gdn::qsa::tc::smem_bytes(HQ);
+    if (smem > smem_optin()) return GDN_ERR_UNSUPPORTED;
+    auto kern = gdn::qsa::qsa_scores_tc_kernel<HQ>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    kern<<<(unsigned)n_ctas, gdn::qsa::tc::kThreads, smem, st>>>(mq, mk, cu, blk0, tile0, cta0, n_seq, r,
+                                                                 (int)nb_max, I);
     return launch_status();
 }
 
@@ -517,8 +589,11 @@ gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dt
     int dev = 0, n_sm = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);   // grid sizing only
-    // rows per CTA pass = 8 warps x rows-per-warp x 2 (unroll); at most 8 CTAs per SM
-    const int64_t rows_per_cta = (int64_t)(gdn::kGateNormThreads / 32) * (32 / (d_v / 8)) * 2;
+    // rows per CTA pass = 8 warps x rows per warp pass (32 bytes of y per lane) x 4 (unroll);
+    // at most 8 CTAs per SM
+    const int epl = y_dtype == GDN_BF16 ? 16 : 8;
+    const int lpr = d_v / epl > 0 ? d_v / epl : 1;
+    const int64_t rows_per_cta = (int64_t)(gdn::kGateNormThreads / 32) * (32 / lpr) * 4;
     int64_t blocks = (n_rows + rows_per_cta - 1) / rows_per_cta;
     const int64_t cap = (int64_t)n_sm * 8;
     if (blocks > cap) blocks = cap;
@@ -607,6 +682,116 @@ gdn_status gdn_featurize(const void *xq, const void *xk, const void *xv, gdn_dty
     }
 #undef GDN_FT_D
 #undef GDN_FT
+    return launch_status();
+}
+
+size_t gdn_qsa_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, int Hq, int d, int r, gdn_dtype dtype)
+{
+    if (!cu_seqlens_host || n_seq < 1 || Hq < 1 || d != gdn::qsa::kD || r < 1) return 0;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return 0;
+    const QsaSizes z = qsa_sizes(cu_seqlens_host, n_seq, r);
+    size_t oq, ok;
+    return qsa_ws_layout(z, n_seq, Hq, dtype == GDN_BF16 ? 2 : 4, &oq, &ok);
+}
+
+gdn_status gdn_qsa_indexer(const void *qx, const void *kx, gdn_dtype dtype, const float *wq, const float *wk,
+                           const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int n_seq, int Hq,
+                           int d, int r, int K, int rot, float base, float eps, float *scores, int32_t *blocks,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    using namespace gdn::qsa;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens_host || !cu_seqlens_dev || n_seq < 1 || Hq < 1 || r < 1 || K < 1) return GDN_ERR_INVALID_ARG;
+    if (rot < 0 || rot > d || rot % 8 != 0 || !(base > 0.f) || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if (d != kD) return GDN_ERR_UNSUPPORTED;
+    if (dtype == GDN_BF16 ? (Hq != 1 && Hq != 2 && Hq != 4) : Hq > kMaxHeadsF32) return GDN_ERR_UNSUPPORTED;
+    const int kb = (K + r - 1) / r;
+    if (kb > kMaxKB) return GDN_ERR_UNSUPPORTED;
+    if (cu_seqlens_host[0] != 0) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < n_seq; ++i)
+        if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return GDN_ERR_INVALID_ARG;
+    const QsaSizes z = qsa_sizes(cu_seqlens_host, n_seq, r);
+    if (z.n_tok == 0) return GDN_OK;
+    if (!qx || !kx || !wq || !wk || !blocks || (z.nb_max > 0 && !scores)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(qx, 16) || !aligned(kx, 16) || !aligned(wq, 4) || !aligned(wk, 4) || !aligned(scores, 4) ||
+        !aligned(blocks, 4) || !aligned(cu_seqlens_dev, 4))
+        return GDN_ERR_INVALID_ARG;
+    if (z.n_tok * Hq > 0x3fffffffLL || z.n_tok * z.nb_max > ((int64_t)1 << 40) || z.n_ctas > 0x7fffffffLL)
+        return GDN_ERR_UNSUPPORTED;
+    const size_t elem = dtype == GDN_BF16 ? 2 : 4;
+    size_t off_q, off_k;
+    const size_t need = qsa_ws_layout(z, n_seq, Hq, elem, &off_q, &off_k);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int32_t *blk0 = reinterpret_cast<int32_t *>(ws);
+    int32_t *tile0 = blk0 + (n_seq + 1);
+    int32_t *cta0 = tile0 + (n_seq + 1);
+    RopeTable rope{};
+    for (int j = 0; j < rot / 2; ++j) rope.inv_freq[j] = std::pow((double)base, -2.0 * j / (double)rot);
+
+    qsa_setup_kernel<<<1, 32, 0, st>>>(cu_seqlens_dev, n_seq, r, blk0, tile0, cta0);
+    const int64_t n_vec = z.n_tok * Hq + z.n_blocks;
+    const unsigned vec_blocks = (unsigned)((n_vec * 32 + kVecThreads - 1) / kVecThreads);
+    if (dtype == GDN_BF16)
+        qsa_vectors_kernel<__nv_bfloat16, __nv_bfloat16><<<vec_blocks, kVecThreads, 0, st>>>(
+            (const __nv_bfloat16 *)qx, (const __nv_bfloat16 *)kx, wq, wk, cu_seqlens_dev, blk0, n_seq, z.n_tok, Hq, r,
+            rot, eps, rope, (__nv_bfloat16 *)(ws + off_q), (__nv_bfloat16 *)(ws + off_k));
+    else
+        qsa_vectors_kernel<float, float><<<vec_blocks, kVecThreads, 0, st>>>(
+            (const float *)qx, (const float *)kx, wq, wk, cu_seqlens_dev, blk0, n_seq, z.n_tok, Hq, r, rot, eps,
+            rope, (float *)(ws + off_q), (float *)(ws + off_k));
+    if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+    if (z.nb_max > 0) {
+        if (dtype == GDN_BF16) {
+            CUtensorMap mq, mk;
+            if (!make_qsa_maps(&mq, &mk, ws + off_q, ws + off_k, z.n_tok, Hq, z.n_blocks)) return GDN_ERR_CUDA;
+            gdn_status rc = Hq == 1 ? launch_qsa_scores_tc<1>(mq, mk, cu_seqlens_dev, blk0, tile0, cta0, n_seq, r,
+                                                              z.nb_max, z.n_ctas, scores, st)
+                          : Hq == 2 ? launch_qsa_scores_tc<2>(mq, mk, cu_seqlens_dev, blk0, tile0, cta0, n_seq, r,
+                                                              z.nb_max, z.n_ctas, scores, st)
+                                    : launch_qsa_scores_tc<4>(mq, mk, cu_seqlens_dev, blk0, tile0, cta0, n_seq, r,
+                                                              z.nb_max, z.n_ctas, scores, st);
+            if (rc != GDN_OK) return rc;
+        } else {
+            const int smem = kF32Tok * Hq * kD * (int)sizeof(float);
+            dim3 grid((unsigned)((z.nb_max + kF32Blk - 1) / kF32Blk), (unsigned)((z.n_tok + kF32Tok - 1) / kF32Tok));
+            if (cudaFuncSetAttribute(qsa_scores_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+                return GDN_ERR_CUDA;
+            qsa_scores_f32_kernel<<<grid, 256, smem, st>>>((const float *)(ws + off_q), (const float *)(ws + off_k),
+                                                           cu_seqlens_dev, blk0, n_seq, z.n_tok, Hq, (int)z.nb_max, r,
+                                                           scores);
+            if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+        }
+    }
+    int kb2 = 1;
+    while (kb2 < kb) kb2 <<= 1;
+    const int smem_sel = kb2 * (int)sizeof(unsigned long long);
+    if (cudaFuncSetAttribute(qsa_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_sel) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    qsa_topk_kernel<<<(unsigned)z.n_tok, kTopkThreads, smem_sel, st>>>(scores, cu_seqlens_dev, n_seq, (int)z.nb_max,
+                                                                       r, kb, blocks);
+    return launch_status();
+}
+
+gdn_status gdn_qsa_token_sets(const int32_t *blocks, const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                              int n_seq, int K_B, int r, int32_t *tokens, int32_t *count, void *stream)
+{
+    using namespace gdn::qsa;
+    if (!cu_seqlens_host || !cu_seqlens_dev || n_seq < 1 || K_B < 1 || r < 1) return GDN_ERR_INVALID_ARG;
+    if (K_B > kMaxKB) return GDN_ERR_UNSUPPORTED;
+    if (cu_seqlens_host[0] != 0) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < n_seq; ++i)
+        if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return GDN_ERR_INVALID_ARG;
+    const int64_t n_tok = cu_seqlens_host[n_seq];
+    if (n_tok == 0) return GDN_OK;
+    if (!blocks || !tokens || !count) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)K_B * r + r - 1 > 0x7fffffffLL || n_tok > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    int kb2 = 1;
+    while (kb2 < K_B) kb2 <<= 1;
+    qsa_token_sets_kernel<<<(unsigned)n_tok, kTopkThreads, kb2 * sizeof(uint32_t), as_stream(stream)>>>(
+        blocks, cu_seqlens_dev, n_seq, K_B, r, tokens, count);
     return launch_status();
 }
 
