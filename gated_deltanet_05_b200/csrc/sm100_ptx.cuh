@@ -434,6 +434,16 @@ __device__ __forceinline__ void tma_load_3d_lead(void *smem_dst, const void *des
         "l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(leader)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_2d_lead(void *smem_dst, const void *desc, uint64_t *bar, int c0, int c1,
+                                                 uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred l;\n\tsetp.ne.b32 l, %5, 0;\n\t"
+        "@l cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];\n\t}" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(leader)
+        : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx_lead(uint64_t *bar, uint32_t bytes, uint32_t leader)
 {
     asm volatile(

@@ -298,6 +298,61 @@ gdn_status gdn_featurize(const void *xq, const void *xk, const void *xv, gdn_dty
                          int d_v, float eps, void *q, void *k, void *v, float *beta,
                          float *log_alpha, void *stream);
 
+/*
+ * gdn_qsa_indexer -- the compressed lightweight indexer of Qwen Sparse Attention (QSA):
+ * per query token, scores of the compressed key blocks and the K_B best blocks.
+ *
+ * Defines: the indexer equations of the joezjh.github.io notes page "Qwen3.8-Flash-Next"
+ * (section on Qwen Sparse Attention, "压缩轻量级 Indexer": key compression, Partial RoPE,
+ * block-causal ReLU importance, Top-K blocks) with the sizes of the pwwt.cn translation
+ * (section on the QSA implementation: four indexer query heads sharing one key head,
+ * token budget K = 2048 at compression ratio r = 4). The projections W x are inputs. For
+ * each sequence of the packed batch (positions restart at its first token), with
+ * RMSNorm(x) = x / sqrt(mean(x^2) + eps) * (1 + w) (zero-centred weight) and PRoPE(x, p)
+ * rotating dimensions (j, j + rot/2), j < rot/2, by the angle p * base^(-2j/rot):
+ *     q_i^h = PRoPE(RMSNorm_wq(qx_i^h), i)
+ *     k_b   = PRoPE(RMSNorm_wk(mean_{j<r} kx_{b r + j}), b r)    b < n_b = floor(len / r)
+ *     I_ib  = sum_h ReLU(<q_i^h, k_b>)      for the visible blocks b < nvis_i =
+ *                                            min(n_b, floor((i + 1) / r))
+ *     B_i   = the K_B = ceil(K / r) visible blocks of largest I_ib, ordered by score
+ *             (descending) then block index (ascending, which also breaks ties); -1 padded
+ *
+ *   qx   [n_tok, Hq, d] and kx [n_tok, d] in dtype (GDN_BF16: tensor-core scores on bf16
+ *        copies of the normalised, rotated vectors, fp32 accumulation; GDN_F32: fp32
+ *        CUDA-core scores); wq, wk [d] fp32
+ *   cu_seqlens_dev / cu_seqlens_host [n_seq + 1] int32 as for gdn_chunk_fwd
+ *   Hq in {1, 2, 4} for GDN_BF16 (1..8 for GDN_F32); d = 128; r >= 1; K >= 1;
+ *   rot even, 0 <= rot <= d; base > 0; eps >= 0
+ *   scores  [n_tok, nb_max] fp32 out, nb_max = max over sequences of floor(len / r):
+ *           I_ib for b < nvis_i; the other entries of a row are not written
+ *   blocks  [n_tok, K_B] int32 out (B_i)
+ *   workspace >= gdn_qsa_workspace_bytes(...) bytes, 16-byte aligned: the normalised,
+ *           rotated queries and compressed keys
+ * Four launches on `stream` (vectors, scores, selection). The pages give no precision for
+ * the indexer; the selection is taken on the scores this call returns.
+ */
+size_t gdn_qsa_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, int Hq, int d, int r,
+                               gdn_dtype dtype);
+gdn_status gdn_qsa_indexer(const void *qx, const void *kx, gdn_dtype dtype, const float *wq,
+                           const float *wk, const int32_t *cu_seqlens_dev,
+                           const int32_t *cu_seqlens_host, int n_seq, int Hq, int d, int r, int K,
+                           int rot, float base, float eps, float *scores, int32_t *blocks,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_qsa_token_sets -- the token set S_i of each query token from its selected blocks:
+ * the r tokens of every selected block plus the tail r floor((i + 1) / r) .. i, in
+ * ascending order (positions within the token's sequence), -1 padded.
+ *
+ * Defines: the final token set of the QSA indexer (joezjh.github.io notes, section on
+ * Qwen Sparse Attention).
+ *   blocks  [n_tok, K_B] int32 (gdn_qsa_indexer's output; -1 entries are skipped)
+ *   tokens  [n_tok, K_B * r + r - 1] int32 out;  count [n_tok] int32 out (|S_i|)
+ */
+gdn_status gdn_qsa_token_sets(const int32_t *blocks, const int32_t *cu_seqlens_dev,
+                              const int32_t *cu_seqlens_host, int n_seq, int K_B, int r,
+                              int32_t *tokens, int32_t *count, void *stream);
+
 /* A static, human-readable name for a status code. */
 const char *gdn_status_string(gdn_status status);
 
