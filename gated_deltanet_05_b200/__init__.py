@@ -23,6 +23,7 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "chunk_fwd_gated", "chunk_fwd_noalloc", "backward", "selftest_bounded_wait", "decode_step", "decode_tokens", "gate_norm", "featurize",
+           "qsa_indexer", "qsa_token_sets",
            "device_error", "lib", "LIB_PATH",
            "GdnError", "EXPORTED_SYMBOLS", "STATUS"]
 
@@ -35,8 +36,8 @@ GDN_F32, GDN_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_fwd_gated",
                     "gdn_chunk_fwd_noalloc", "gdn_backward_workspace_bytes", "gdn_backward",
                     "gdn_selftest_bounded_wait", "gdn_decode_step", "gdn_decode_tokens",
-                    "gdn_gate_norm", "gdn_featurize", "gdn_status_string", "gdn_device_error",
-                    "gdn_version")
+                    "gdn_gate_norm", "gdn_featurize", "gdn_qsa_workspace_bytes", "gdn_qsa_indexer",
+                    "gdn_qsa_token_sets", "gdn_status_string", "gdn_device_error", "gdn_version")
 
 
 class GdnError(RuntimeError):
@@ -89,6 +90,13 @@ def lib():
         L.gdn_featurize.restype = i32
         L.gdn_featurize.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, i32, i64,
                                     i32, i32, i32, f32, vp, vp, vp, vp, vp, vp]
+        L.gdn_qsa_workspace_bytes.restype = ctypes.c_size_t
+        L.gdn_qsa_workspace_bytes.argtypes = [vp, i32, i32, i32, i32, i32]
+        L.gdn_qsa_indexer.restype = i32
+        L.gdn_qsa_indexer.argtypes = [vp, vp, i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32, vp, vp,
+                                      vp, ctypes.c_size_t, vp]
+        L.gdn_qsa_token_sets.restype = i32
+        L.gdn_qsa_token_sets.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_status_string.argtypes = [i32]
         L.gdn_device_error.restype = i32
@@ -379,6 +387,69 @@ def featurize(xq, xk, xv, conv_q, conv_k, conv_v, beta_logit, alpha_logit, A, b_
                              _ptr(log_alpha), _stream(xq.device))
     _check("gdn_featurize", rc)
     return q, k, v, beta, log_alpha
+
+
+def qsa_indexer(qx, kx, wq, wk, cu_seqlens, r=4, K=2048, rot=64, base=10000.0, eps=1e-6,
+                cu_seqlens_host=None, out=None):
+    """The QSA compressed indexer over packed sequences (see gdn_qsa_indexer in gdn.h).
+
+    qx [N, Hq, 128] and kx [N, 128] (one dtype: bfloat16 runs the tensor-core scores,
+    float32 the fp32 CUDA-core ones); wq, wk [128] fp32 (zero-centred RMSNorm weights);
+    cu_seqlens [n_seq + 1] int32 (device). Returns (scores [N, nb_max] fp32, valid only for
+    each token's visible blocks, blocks [N, ceil(K / r)] int32, -1 padded). `out` may
+    supply (scores, blocks)."""
+    for t, n in ((qx, "qx"), (kx, "kx"), (wq, "wq"), (wk, "wk"), (cu_seqlens, "cu_seqlens")):
+        _cuda(t, n)
+    if kx.dtype != qx.dtype:
+        raise TypeError("qx and kx must share one dtype")
+    if wq.dtype != torch.float32 or wk.dtype != torch.float32:
+        raise TypeError("wq and wk must be float32")
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    N, Hq, d = qx.shape
+    n_seq = cu_seqlens.numel() - 1
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.to("cpu")
+    cu_h = cu_seqlens_host.to(torch.int32).contiguous()
+    lens = (cu_h[1:] - cu_h[:-1]).tolist()
+    nb_max = max([ln // r for ln in lens] + [0])
+    kb = -(-K // r)
+    if out is None:
+        out = (torch.empty((N, max(nb_max, 1)), dtype=torch.float32, device=qx.device),
+               torch.empty((N, kb), dtype=torch.int32, device=qx.device))
+    scores, blocks = out
+    _cuda(scores, "scores")
+    _cuda(blocks, "blocks")
+    L = lib()
+    code = _dtype_code(qx)
+    ws_bytes = L.gdn_qsa_workspace_bytes(ctypes.c_void_p(cu_h.data_ptr()), n_seq, Hq, d, r, code)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=qx.device)
+    rc = L.gdn_qsa_indexer(_ptr(qx), _ptr(kx), code, _ptr(wq), _ptr(wk), _ptr(cu_seqlens),
+                           ctypes.c_void_p(cu_h.data_ptr()), n_seq, Hq, d, int(r), int(K), int(rot),
+                           float(base), float(eps), _ptr(scores), _ptr(blocks), _ptr(ws), ws_bytes,
+                           _stream(qx.device))
+    _check("gdn_qsa_indexer", rc)
+    return scores[:, :nb_max], blocks
+
+
+def qsa_token_sets(blocks, cu_seqlens, r=4, cu_seqlens_host=None):
+    """Token sets of the QSA indexer's selection: (tokens [N, K_B * r + r - 1] int32 in
+    ascending order, -1 padded, positions within each sequence; count [N] int32)."""
+    _cuda(blocks, "blocks")
+    _cuda(cu_seqlens, "cu_seqlens")
+    if blocks.dtype != torch.int32:
+        raise TypeError("blocks must be int32")
+    N, kb = blocks.shape
+    n_seq = cu_seqlens.numel() - 1
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.to("cpu")
+    cu_h = cu_seqlens_host.to(torch.int32).contiguous()
+    tokens = torch.empty((N, kb * r + r - 1), dtype=torch.int32, device=blocks.device)
+    count = torch.empty((N,), dtype=torch.int32, device=blocks.device)
+    rc = lib().gdn_qsa_token_sets(_ptr(blocks), _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), n_seq, kb,
+                                  int(r), _ptr(tokens), _ptr(count), _stream(blocks.device))
+    _check("gdn_qsa_token_sets", rc)
+    return tokens, count
 
 
 def selftest_bounded_wait(limit_cycles=2_000_000, mode=0, device=None):

@@ -19,6 +19,12 @@ benchmark workloads of this library:
 
 Draw order within one workload: q, k, v, beta logits, A, u, S0, z, w.
 
+The QSA compressed indexer (make_qsa_inputs) takes the indexer's projected query and key
+streams: qx ~ N(0, 1) [N_tok, Hq, 128] and kx ~ N(0, 1) [N_tok, 128] in the workload dtype
+and the zero-centred RMSNorm weights wq, wk ~ N(0, 0.02); draw order qx, kx, wq, wk. Its
+benchmark shape is one 16,384-token sequence with Hq = 4, r = 4, K = 2048 (a scaled-down
+stand-in for the pages' 1M-token context prefilled in 16K-token chunks).
+
 The featurisation step in front of the recurrence takes the projected streams instead
 (make_featurize_inputs): xq, xk, xv ~ N(0, 1) in the workload dtype, depthwise
 convolution weights ~ N(0, 1/W) fp32 with W = 4 taps, beta and alpha logits ~ N(0, 1),
@@ -34,7 +40,7 @@ import torch
 
 __all__ = [
     "Workload", "WORKLOADS", "make_prefill_inputs", "make_decode_inputs", "make_featurize_inputs",
-    "varlen_lengths", "to_f64",
+    "varlen_lengths", "to_f64", "QSA_WORKLOAD", "make_qsa_inputs",
 ]
 
 
@@ -212,3 +218,21 @@ def to_f64(t) -> np.ndarray:
 
 def ceil_div(a: int, b: int) -> int:
     return -(-a // b)
+
+
+QSA_WORKLOAD = {"lengths": (16384,), "Hq": 4, "r": 4, "K": 2048, "dtype": "bf16", "seed": 5}
+
+
+def make_qsa_inputs(lengths, Hq: int, dtype: str = "bf16", seed: int = 5, d: int = 128) -> dict:
+    """Inputs of the QSA compressed indexer for packed sequences of the given lengths."""
+    rng = np.random.default_rng(seed)
+    n = int(sum(lengths))
+    cast = (lambda a: torch.from_numpy(a).to(torch.bfloat16)) if dtype == "bf16" else \
+        (lambda a: torch.from_numpy(a.astype(np.float32)))
+    qx = cast(rng.standard_normal((n, Hq, d)))
+    kx = cast(rng.standard_normal((n, d)))
+    wq = torch.from_numpy(rng.normal(0.0, 0.02, d).astype(np.float32))
+    wk = torch.from_numpy(rng.normal(0.0, 0.02, d).astype(np.float32))
+    cu = torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32)
+    return {"qx": qx, "kx": kx, "wq": wq, "wk": wk, "cu_seqlens": cu, "lengths": tuple(lengths), "Hq": Hq,
+            "dtype": dtype}
