@@ -25,7 +25,7 @@ namespace gdn {
 
 constexpr int kFeatThreads = 128;
 constexpr int kFeatRun = 32;      // tokens per warp task
-constexpr int kFeatBatch = 4;     // rows loaded ahead
+constexpr int kFeatBatch = 2;     // rows loaded ahead
 constexpr int kFeatMaxWidth = 4;  // convolution taps
 
 // SiLU with the fast exponential and division intrinsics (relative error ~1e-6, well inside
@@ -36,25 +36,46 @@ __device__ __forceinline__ float softplus_f32(float x)
     return x > 0.f ? x + log1pf(expf(-x)) : log1pf(expf(x));
 }
 
-// Four consecutive elements as loaded: one float4 (fp32) or two packed bf16 pairs.
+// Eight consecutive elements as loaded: two float4 (fp32) or four packed bf16 pairs.
+struct F8 { float4 a, b; };
 template <typename T> struct RawRow;
-template <> struct RawRow<float> { using type = float4; };
-template <> struct RawRow<__nv_bfloat16> { using type = uint2; };
-__device__ __forceinline__ void raw_to_f32(const float4 &r, float (&x)[4])
+template <> struct RawRow<float> { using type = F8; };
+template <> struct RawRow<__nv_bfloat16> { using type = uint4; };
+__device__ __forceinline__ void raw_to_f32(const F8 &r, float (&x)[8])
 {
-    x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
+    x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+    x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
 }
-__device__ __forceinline__ void raw_to_f32(const uint2 &r, float (&x)[4])
+__device__ __forceinline__ void raw_to_f32(const uint4 &r, float (&x)[8])
 {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void store8f(float *p, const float (&x)[8])
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
+}
+__device__ __forceinline__ void store8f(__nv_bfloat16 *p, const float (&x)[8])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // One launch covers n_streams streams of width D (q and k with L2 = true; v with
 // L2 = false) and, when beta_logit is given, the gates.
 template <typename T, int D, bool L2>
-__global__ void __launch_bounds__(kFeatThreads, 6)
+__global__ void __launch_bounds__(kFeatThreads, 4)
 featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float *__restrict__ w0,
                  const float *__restrict__ w1, T *__restrict__ o0, T *__restrict__ o1, int n_streams,
                  int W, const int32_t *__restrict__ cu, int n_seq, int64_t n_tok, int H, float eps,
@@ -62,8 +83,9 @@ featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float
                  const float *__restrict__ A, const float *__restrict__ b_alpha, float *__restrict__ beta,
                  float *__restrict__ log_alpha)
 {
-    constexpr int LPR = D / 4;
-    static_assert(LPR >= 4 && LPR <= 32, "D in 16..128");
+    constexpr int CPL = 8;                  // channels per lane
+    constexpr int LPR = D / CPL;
+    static_assert(LPR >= 2 && LPR <= 16, "D in 16..128");
     constexpr int RPW = 32 / LPR;
     const int lane = threadIdx.x & 31;
     const int64_t task = ((int64_t)blockIdx.x * kFeatThreads + threadIdx.x) >> 5;
@@ -90,15 +112,15 @@ featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float
     const int64_t run = rem / n_hg;
     const int h = (int)(rem % n_hg) * RPW + lane / LPR;
     const bool active = h < H;
-    const int ch0 = (lane % LPR) * 4;
+    const int ch0 = (lane % LPR) * CPL;
     const T *x = s == 0 ? x0 : x1;
     const float *wt = s == 0 ? w0 : w1;
     T *o = s == 0 ? o0 : o1;
 
     // taps padded to four: tap kFeatMaxWidth - W + j multiplies the row W - 1 - j back
-    float w4[4][kFeatMaxWidth];
+    float w4[CPL][kFeatMaxWidth];
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < CPL; ++c)
 #pragma unroll
         for (int j = 0; j < kFeatMaxWidth; ++j) {
             const int jj = j - (kFeatMaxWidth - W);
@@ -129,14 +151,14 @@ featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float
     T *oh = o + (size_t)h * D + ch0;
 
     // window: rows t-3, t-2, t-1 (zero before the sequence's first token)
-    float win[3][4];
+    using Raw = typename RawRow<T>::type;
+    float win[3][CPL];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
         const int64_t tt = t0 - 3 + j;
-        const float4 f = (active && tt >= bos) ? load4(xh + tt * row_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
-        win[j][0] = f.x; win[j][1] = f.y; win[j][2] = f.z; win[j][3] = f.w;
+        const Raw rw = (active && tt >= bos) ? *reinterpret_cast<const Raw *>(xh + tt * row_stride) : Raw{};
+        raw_to_f32(rw, win[j]);
     }
-    using Raw = typename RawRow<T>::type;
     auto load_batch = [&](Raw (&raw)[kFeatBatch], int64_t tb) {
 #pragma unroll
         for (int u = 0; u < kFeatBatch; ++u) {
@@ -155,7 +177,7 @@ featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float
         for (int u = 0; u < kFeatBatch; ++u) {
             const int64_t tt = tb + u;
             if (tt >= t_end) break;                 // warp-uniform
-            float xr[4];
+            float xr[CPL];
             raw_to_f32(cur[u], xr);
             if (tt == next) {                       // a new sequence starts here
                 while (next <= tt && seq < n_seq - 1) {
@@ -169,12 +191,12 @@ featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float
 #pragma unroll
                 for (int j = 0; j < 3; ++j)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) win[j][c] = 0.f;
+                    for (int c = 0; c < CPL; ++c) win[j][c] = 0.f;
             }
-            float f[4];
+            float f[CPL];
             float ss = 0.f;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < CPL; ++c) {
                 float acc = w4[c][3] * xr[c];
                 acc = fmaf(w4[c][2], win[2][c], acc);
                 acc = fmaf(w4[c][1], win[1][c], acc);
@@ -186,11 +208,11 @@ featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float
                 ss = group_sum<LPR>(ss);
                 const float inv = rsqrtf(ss + eps);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) f[c] *= inv;
+                for (int c = 0; c < CPL; ++c) f[c] *= inv;
             }
-            if (active) store4(oh + tt * row_stride, make_float4(f[0], f[1], f[2], f[3]));
+            if (active) store8f(oh + tt * row_stride, f);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < CPL; ++c) {
                 win[0][c] = win[1][c];
                 win[1][c] = win[2][c];
                 win[2][c] = xr[c];
