@@ -8,7 +8,7 @@
 #include <mutex>
 
 #include "gdn.h"
-#include "gdn_backward.cuh"
+#include "gdn_backward_chunk.cuh"
 #include "gdn_chunk_f32.cuh"
 #include "gdn_chunk_sm100.cuh"
 #include "gdn_common.cuh"
@@ -109,7 +109,7 @@ gdn_status launch_chunk_f32(const void *q, const void *k, const void *v, const f
     const unsigned grid = (unsigned)((int64_t)n_seq * H * (dv / dvt));
     kern<<<grid, gdn::kChunkF32Threads, smem, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), la, beta, S0,
-        cu, H, dk, dv, C, dvt, scale, static_cast<TY *>(y), S_T);
+        cu, H, dk, dv, C, dvt, scale, static_cast<TY *>(y), S_T, nullptr, 0);
     return launch_status();
 }
 
@@ -404,7 +404,12 @@ size_t gdn_backward_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, i
         const int64_t l = (int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i];
         if (l > max_len) max_len = l;
     }
-    return (size_t)n_seq * H * gdn::bwd_ws_floats_per_chain(max_len, d_k, d_v) * sizeof(float);
+    const int64_t max_chunks = (max_len + gdn::bwdc::kC - 1) / gdn::bwdc::kC;
+    const int n_vt = d_v / (d_v < gdn::bwdc::kDVT ? d_v : gdn::bwdc::kDVT);
+    // per (chain, chunk): the start state and the end-state adjoint [d_k][d_v], and one block
+    // of sums over v per value slice
+    const size_t per_chunk = 2 * (size_t)d_k * d_v + (size_t)n_vt * gdn::bwdc::part_floats(d_k);
+    return (size_t)n_seq * H * (size_t)max_chunks * per_chunk * sizeof(float);
 }
 
 gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
@@ -414,6 +419,7 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
                         float *dq, float *dk, float *dv, float *dlog_alpha, float *dbeta, float *dS0,
                         void *workspace, size_t workspace_bytes, void *stream)
 {
+    using namespace gdn::bwdc;
     if (n_seq < 0 || H <= 0 || !cu_seqlens_host || (n_seq > 0 && !cu_seqlens_dev))
         return GDN_ERR_INVALID_ARG;
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
@@ -422,7 +428,6 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
     for (int i = 0; i < n_seq; ++i)
         if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return GDN_ERR_INVALID_ARG;
     if (n_seq == 0) return GDN_OK;
-    if ((int64_t)n_seq * H > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     const int64_t n_tok = cu_seqlens_host[n_seq];
     if (n_tok > 0 && (!q || !k || !v || !log_alpha || !beta || !dy || !dq || !dk || !dv ||
                       !dlog_alpha || !dbeta))
@@ -434,19 +439,56 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
     for (int i = 0; i < n_seq; ++i)
         if ((int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i] > max_len)
             max_len = (int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i];
+    const int64_t n_chain = (int64_t)n_seq * H;
+    const int64_t max_chunks = (max_len + kC - 1) / kC;
+    const int dvt = d_v < kDVT ? d_v : kDVT;
+    const int n_vt = d_v / dvt;
+    if (n_chain * n_vt > 0x7fffffffLL || max_chunks > 65535) return GDN_ERR_UNSUPPORTED;
+    if (max_chunks == 0) {
+        // no tokens: dS0 = dS_T (or 0)
+        if (dS0) {
+            cudaStream_t st0 = as_stream(stream);
+            const size_t bytes = (size_t)n_chain * d_k * d_v * sizeof(float);
+            const cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, bytes, cudaMemcpyDeviceToDevice, st0)
+                                       : cudaMemsetAsync(dS0, 0, bytes, st0);
+            if (e != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        return GDN_OK;
+    }
     cudaStream_t st = as_stream(stream);
-    const int smem = (int)(sizeof(float) * (2 * (size_t)d_v * (d_k + 1) + 2 * d_k + 4 * d_v + gdn::kBwdThreads / 32));
-    if (smem > smem_optin()) return GDN_ERR_UNSUPPORTED;
-    const unsigned grid = (unsigned)((int64_t)n_seq * H);
-#define GDN_BWD(T)                                                                                 \
-    {                                                                                              \
-        auto kern = gdn::gdn_backward_kernel<T>;                                                   \
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
-            return GDN_ERR_CUDA;                                                                   \
-        kern<<<grid, gdn::kBwdThreads, smem, st>>>((const T *)q, (const T *)k, (const T *)v, log_alpha, beta, \
-                                                   S0, cu_seqlens_dev, H, d_k, d_v, scale, (const T *)dy, dS_T, \
-                                                   dq, dk, dv, dlog_alpha, dbeta, dS0,             \
-                                                   static_cast<float *>(workspace), max_len);      \
+    float *S_chunks = static_cast<float *>(workspace);
+    float *dS_chunks = S_chunks + (size_t)n_chain * max_chunks * d_k * d_v;
+    float *parts = dS_chunks + (size_t)n_chain * max_chunks * d_k * d_v;
+    const int smem_f = (int)(chunk_f32_layout(kC, d_k, dvt).total * sizeof(float));
+    const int smem_s = (int)(state_layout(d_k).total * sizeof(float));
+    const int smem_v = (int)(vpart_layout(d_k).total * sizeof(float));
+    const int smem_k = (int)(kpart_layout(d_k).total * sizeof(float));
+    const int optin = smem_optin();
+    if (smem_f > optin || smem_s > optin || smem_v > optin || smem_k > optin) return GDN_ERR_UNSUPPORTED;
+    const dim3 grid_v((unsigned)(n_chain * n_vt), (unsigned)max_chunks);
+    const dim3 grid_k((unsigned)n_chain, (unsigned)max_chunks);
+#define GDN_BWD(T)                                                                                   \
+    {                                                                                                \
+        auto kf = gdn::chunk_fwd_f32_kernel<T, float>;                                               \
+        auto ks = chunk_bwd_state_kernel<T>;                                                         \
+        auto kv = chunk_bwd_vpart_kernel<T>;                                                         \
+        auto kk = chunk_bwd_kpart_kernel<T>;                                                         \
+        if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f) != cudaSuccess || \
+            cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_s) != cudaSuccess || \
+            cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_v) != cudaSuccess || \
+            cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)   \
+            return GDN_ERR_CUDA;                                                                     \
+        kf<<<(unsigned)(n_chain * n_vt), gdn::kChunkF32Threads, smem_f, st>>>(                       \
+            (const T *)q, (const T *)k, (const T *)v, log_alpha, beta, S0, cu_seqlens_dev, H, d_k, d_v, kC, dvt, \
+            scale, (float *)nullptr, (float *)nullptr, S_chunks, (int)max_chunks);                   \
+        ks<<<(unsigned)(n_chain * n_vt), kThreads, smem_s, st>>>(                                    \
+            (const T *)q, (const T *)k, (const T *)dy, log_alpha, beta, cu_seqlens_dev, H, d_k, d_v, scale, dS_T, \
+            dS_chunks, (int)max_chunks, dS0);                                                        \
+        kv<<<grid_v, kThreads, smem_v, st>>>((const T *)q, (const T *)k, (const T *)v, (const T *)dy, log_alpha, \
+                                             beta, cu_seqlens_dev, H, d_k, d_v, scale, S_chunks, dS_chunks,      \
+                                             (int)max_chunks, parts, dv);                              \
+        kk<<<grid_k, kThreads, smem_k, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
+                                             n_vt, scale, (int)max_chunks, parts, dq, dk, dbeta, dlog_alpha);    \
     }
     if (in_dtype == GDN_F32)
         GDN_BWD(float)
@@ -654,7 +696,7 @@ gdn_status gdn_featurize(const void *xq, const void *xk, const void *xv, gdn_dty
     const int64_t n_runs = (n_tok + gdn::kFeatRun - 1) / gdn::kFeatRun;
     const int warps_per_block = gdn::kFeatThreads / 32;
     auto blocks_for = [&](int d, int n_streams, bool gates) -> unsigned {
-        const int rpw = 32 / (d / 4);
+        const int rpw = 32 / (d / 8);
         const int64_t n_hg = (H + rpw - 1) / rpw;
         const int64_t tasks = n_streams * n_runs * n_hg + (gates ? n_runs : 0);
         return (unsigned)((tasks + warps_per_block - 1) / warps_per_block);
