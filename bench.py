@@ -359,6 +359,7 @@ def run_ours(args, rank, world, local, pg):
         "long": bench_prefill_shape(args, "long", device, peaks, peak_kind, pg, rank),
         "varlen": bench_prefill_shape(args, "varlen", device, peaks, peak_kind, pg, rank)}
     decode = None if args.no_decode else bench_decode(args, device, peaks, peak_kind, pg)
+    qsa = None if args.no_shapes else bench_qsa(args, device, peaks, pg, rank)
     featurize = bench_featurize(args, device, peaks, peak_kind, pg, rank)
     backward = bench_backward(args, inp, device, pg) if world == 1 else None
     e2e = bench_e2e(args, inp, device, pg, world)
@@ -379,6 +380,7 @@ def run_ours(args, rank, world, local, pg):
         "fused_step": fused,
         "decode": decode,
         "featurize": featurize,
+        "qsa_indexer": qsa,
         "backward": backward,
         "e2e": e2e,
         "gpu_launches": 2 * args.steps,
@@ -444,6 +446,54 @@ def bench_prefill_shape(args, name, device, peaks, peak_kind, pg, rank):
             "tensor": {"achieved": tflops, "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
                        "flops_per_launch": flops},
             "launches": reps, "l2": "inputs above the 126 MB L2"}
+
+
+def bench_qsa(args, device, peaks, pg, rank):
+    """The QSA compressed indexer (gdn_qsa_indexer: vectors, tensor-core scores, top-K) on
+    one 16,384-token sequence, Hq = 4, r = 4, K = 2048, bf16. The score FLOPs count every
+    visible (token, block) pair: 2 * 128 * Hq per pair."""
+    import torch
+
+    import gated_deltanet_05_b200 as gdn
+    import workloads as W
+    cfg = W.QSA_WORKLOAD
+    inp = W.make_qsa_inputs(cfg["lengths"], cfg["Hq"], cfg["dtype"], seed=cfg["seed"] + 1000 * rank)
+    d = {k: inp[k].to(device) for k in ("qx", "kx", "wq", "wk", "cu_seqlens")}
+    r, K, Hq = cfg["r"], cfg["K"], cfg["Hq"]
+    n = int(inp["cu_seqlens"][-1])
+    nb = n // r
+    kb = -(-K // r)
+    out = (torch.empty((n, nb), dtype=torch.float32, device=device),
+           torch.empty((n, kb), dtype=torch.int32, device=device))
+    stream = torch.cuda.current_stream(device)
+
+    def run():
+        gdn.qsa_indexer(d["qx"], d["kx"], d["wq"], d["wk"], d["cu_seqlens"], r=r, K=K,
+                        cu_seqlens_host=inp["cu_seqlens"], out=out)
+
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize(device)
+    reps = 20
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(pg, device)
+    a.record(stream)
+    for _ in range(reps):
+        run()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    status = gdn.device_error(device)
+    if status != "GDN_OK":
+        raise SystemExit(f"device error in the QSA leg: {status}")
+    ms = max_over_ranks(pg, a.elapsed_time(b), device) / reps
+    pairs = sum(min(nb, (i + 1) // r) for i in range(n))
+    flops = 2.0 * 128 * Hq * pairs
+    return {"workload": f"QSA indexer bf16: 1 seq x {n} tokens, Hq={Hq}, d=128, r={r}, K={K} (K_B={kb})",
+            "kernels": "qsa_setup, qsa_vectors, qsa_scores_tc (tcgen05), qsa_topk",
+            "ms_per_call": ms, "tokens_per_s": n / (ms * 1e-3), "visible_pairs": pairs,
+            "score_flops": flops, "score_tflops_over_call": flops / (ms * 1e-3) / 1e12,
+            "score_bytes_written": 4 * pairs, "launches": reps}
 
 
 def bench_decode(args, device, peaks, peak_kind, pg):
@@ -667,7 +717,8 @@ def run_case(args):
     --case decode:N        (N sequences x 32 heads, d=128, fp32 state)
     --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)
     --case featurize:S,T,H (bf16, d=128, conv width 4)
-    --case decode_tokens:N,T (N sequences x 32 heads, d=128, T tokens per call)"""
+    --case decode_tokens:N,T (N sequences x 32 heads, d=128, T tokens per call)
+    --case qsa:N           (the QSA indexer on one N-token sequence, Hq=4, r=4, K=2048, bf16)"""
     import torch
 
     import gated_deltanet_05_b200 as gdn
@@ -714,6 +765,13 @@ def run_case(args):
         wn = (torch.randn(128, generator=g) * 0.02).cuda()
         for _ in range(args.reps):
             gdn.gate_norm(y, z, wn, out_dtype=torch.bfloat16)
+    elif kind == "qsa":
+        (n,) = dims
+        inp = W.make_qsa_inputs((n,), 4, "bf16", seed=5)
+        d = {k: inp[k].cuda() for k in ("qx", "kx", "wq", "wk", "cu_seqlens")}
+        for _ in range(args.reps):
+            gdn.qsa_indexer(d["qx"], d["kx"], d["wq"], d["wk"], d["cu_seqlens"], r=4, K=2048,
+                            cu_seqlens_host=inp["cu_seqlens"])
     elif kind == "featurize":
         n_seq, T, H = dims
         w = W.Workload("case", "bf16", (T,) * n_seq, H, 128, 128, 64, seed=1)
