@@ -807,13 +807,12 @@ gdn_status gdn_qsa_indexer(const void *qx, const void *kx, gdn_dtype dtype, cons
             if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
         }
     }
-    int kb2 = 1;
-    while (kb2 < kb) kb2 <<= 1;
-    const int smem_sel = kb2 * (int)sizeof(unsigned long long);
+    const int smem_sel = (int)topk_smem_bytes(kb);
+    if (smem_sel > smem_optin()) return GDN_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(qsa_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_sel) != cudaSuccess)
         return GDN_ERR_CUDA;
-    qsa_topk_kernel<<<(unsigned)z.n_tok, kTopkThreads, smem_sel, st>>>(scores, cu_seqlens_dev, n_seq, (int)z.nb_max,
-                                                                       r, kb, blocks);
+    qsa_topk_kernel<<<(unsigned)((z.n_tok + kTopkWarps - 1) / kTopkWarps), kTopkWarps * 32, smem_sel, st>>>(
+        scores, cu_seqlens_dev, n_seq, z.n_tok, (int)z.nb_max, r, kb, blocks);
     return launch_status();
 }
 

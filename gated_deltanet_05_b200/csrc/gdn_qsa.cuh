@@ -20,7 +20,7 @@
 //   qsa_scores_tc_kernel  tcgen05: 128 query tokens x 128 key blocks per step, one M=128,
 //                       N=128 accumulator per query head in TMEM, ReLU-summed over heads
 //   qsa_scores_f32_kernel CUDA cores, fp32: one thread per (token, block)
-//   qsa_topk_kernel     one CTA per token: radix selection of the K_B largest scores, then
+//   qsa_topk_kernel     one warp per token: radix selection of the K_B largest scores, then
 //                       a bitonic sort of the selection by (score desc, block asc)
 //   qsa_token_sets_kernel one CTA per token: the selected blocks in ascending order,
 //                       expanded to tokens, plus the tail
@@ -229,9 +229,10 @@ constexpr uint32_t HEAD_BYTES = 32768;       // one head's 128 tokens x 128 dims
 constexpr uint32_t KT_BYTES = 32768;         // one key tile: 128 blocks x 128 dims bf16, two boxes
 constexpr int kKStages = 2;
 constexpr long long kWaitLimit = 2000000000LL;
+constexpr uint32_t STAGE_BYTES = 8 * 32 * 17 * 4;   // per epilogue warp: 32 rows x 16 columns (+1 pad)
 constexpr uint32_t smem_bytes(int hq)
 {
-    return (uint32_t)hq * HEAD_BYTES + kKStages * KT_BYTES + 256 + 1024;
+    return (uint32_t)hq * HEAD_BYTES + kKStages * KT_BYTES + STAGE_BYTES + 256 + 1024;
 }
 }  // namespace tc
 
@@ -254,7 +255,8 @@ qsa_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
     constexpr uint32_t OFF_K = HQ * tc::HEAD_BYTES;
-    constexpr uint32_t OFF_BAR = OFF_K + tc::kKStages * tc::KT_BYTES;
+    constexpr uint32_t OFF_STAGE = OFF_K + tc::kKStages * tc::KT_BYTES;
+    constexpr uint32_t OFF_BAR = OFF_STAGE + tc::STAGE_BYTES;
     enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + tc::kKStages, B_AFULL = B_KEMPTY + tc::kKStages,
            B_AEMPTY = B_AFULL + HQ, B_DRAIN = B_AEMPTY + HQ, N_BAR };
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
@@ -354,11 +356,6 @@ qsa_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ---------------------------------------------------------------- epilogue
         const int e = warp - 4, half = e >> 2;
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u << 16;
-        const int64_t pos = t_first + 32 * (warp & 3) + lane;    // this thread's query token
-        const bool row_ok = pos < len;
-        int64_t nvis = (pos + 1) / r;
-        if (nvis > len / r) nvis = len / r;
-        float *out = I + (size_t)(bos + pos) * nb_max;
         bool ok = true;
 #pragma unroll 1
         for (int j = 0; j < n_my && ok; ++j) {
@@ -383,11 +380,27 @@ qsa_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 mbar_arrive(&bar[B_AEMPTY + h]);
             }
             if (!ok) break;
+            // the warp's 32 rows x 64 scores go out through its staging slice, 16 columns at
+            // a time: each store instruction writes two rows' 16 consecutive scores (lanes
+            // 0..15 and 16..31), instead of 32 rows' single scores
             const int64_t b0 = (step0 + j) * kTileB + 64 * half;
-            if (row_ok) {
+            float *stg = reinterpret_cast<float *>(smem + OFF_STAGE) + e * 32 * 17;
+            const int64_t t_row0 = t_first + 32 * (warp & 3);      // sequence position of row 0
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (b0 + i < nvis) out[b0 + i] = acc[i];
+            for (int c16 = 0; c16 < 4; ++c16) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) stg[lane * 17 + i] = acc[16 * c16 + i];
+                __syncwarp();
+#pragma unroll 4
+                for (int rr = 0; rr < 32; rr += 2) {
+                    const int row = rr + (lane >> 4), col = lane & 15;
+                    const int64_t p_row = t_row0 + row;
+                    int64_t nv_row = (p_row + 1) / r;
+                    if (nv_row > len / r) nv_row = len / r;
+                    const int64_t b = b0 + 16 * c16 + col;
+                    if (p_row < len && b < nv_row) I[(size_t)(bos + p_row) * nb_max + b] = stg[row * 17 + col];
+                }
+                __syncwarp();
             }
         }
         // leaving early: release the issuer from any head it may still wait for
@@ -410,138 +423,121 @@ __device__ __forceinline__ uint32_t fkey(float x)
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive prefix sum of one int per thread (kTopkThreads threads); returns the
-// thread's prefix and writes the total to *total.
-__device__ __forceinline__ int block_exclusive_sum(int x, int *warp_sums, int *total)
+// One warp per token (kTopkWarps tokens per CTA): B_t = the kb largest scores of the visible
+// blocks, ordered by (score descending, block ascending); -1 padded. Radix selection on the
+// order-preserving keys (four 8-bit passes over the row, a 256-bin histogram per warp in
+// shared memory) finds the kb-th largest key T; the keys above T and the lowest-index keys
+// equal to T are gathered (ballots keep index order), then sorted by the warp (bitonic, in
+// its shared-memory slice). Rows with at most kb visible blocks take every block.
+constexpr int kTopkWarps = 4;
+
+__host__ __device__ inline int topk_pow2(int kb)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    __syncthreads();
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int v = lane < kTopkThreads / 32 ? warp_sums[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += n;
-        }
-        if (lane < kTopkThreads / 32) warp_sums[lane] = v;     // inclusive warp totals
-    }
-    __syncthreads();
-    const int before = warp > 0 ? warp_sums[warp - 1] : 0;
-    *total = warp_sums[kTopkThreads / 32 - 1];
-    return before + incl - x;
+    int p = 1;
+    while (p < kb) p <<= 1;
+    return p;
+}
+__host__ __device__ inline size_t topk_smem_bytes(int kb)
+{
+    return (size_t)kTopkWarps * ((size_t)topk_pow2(kb) * sizeof(unsigned long long) + 256 * sizeof(int));
 }
 
-// One CTA per token: B_t = the kb largest scores of the visible blocks, ordered by (score
-// descending, block ascending); -1 padded. Radix selection on the order-preserving keys
-// (four 8-bit passes over the row) finds the kb-th largest key T; the keys above T and the
-// lowest-index keys equal to T are gathered, then sorted (bitonic, in shared memory).
-__global__ void __launch_bounds__(kTopkThreads)
-qsa_topk_kernel(const float *__restrict__ I, const int32_t *__restrict__ cu, int n_seq, int nb_max, int r, int kb,
-                int32_t *__restrict__ B)
+__global__ void __launch_bounds__(kTopkWarps * 32)
+qsa_topk_kernel(const float *__restrict__ I, const int32_t *__restrict__ cu, int n_seq, int64_t n_tok, int nb_max,
+                int r, int kb, int32_t *__restrict__ B)
 {
-    extern __shared__ unsigned long long sel[];        // [kb_pow2] composite keys
-    __shared__ int hist[256];
-    __shared__ int warp_sums[kTopkThreads / 32];
-    __shared__ int s_digit, s_above, s_count;
-    const int64_t t = blockIdx.x;
+    extern __shared__ unsigned long long topk_sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kb2 = topk_pow2(kb);
+    unsigned long long *sel = topk_sm + (size_t)warp * kb2;
+    int *hist = reinterpret_cast<int *>(topk_sm + (size_t)kTopkWarps * kb2) + warp * 256;
+    const int64_t t = (int64_t)blockIdx.x * kTopkWarps + warp;
+    if (t >= n_tok) return;
     const int s = upper_index(cu, n_seq + 1, t);
     const int64_t pos = t - cu[s], len = (int64_t)cu[s + 1] - cu[s];
     int64_t nv64 = (pos + 1) / r;
     if (nv64 > len / r) nv64 = len / r;
     const int nvis = (int)nv64;
     const float *row = I + (size_t)t * nb_max;
-    int kb2 = 1;
-    while (kb2 < kb) kb2 <<= 1;
     const int take = nvis < kb ? nvis : kb;
 
     uint32_t prefix = 0, mask = 0;
-    int need = take;                                   // keys still to take at or below the prefix
+    int need = take;                               // keys still to take at or below the prefix
     if (nvis > kb) {
         for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int i = threadIdx.x; i < 256; i += kTopkThreads) hist[i] = 0;
-            __syncthreads();
-            for (int b = threadIdx.x; b < nvis; b += kTopkThreads) {
+            for (int i = lane; i < 256; i += 32) hist[i] = 0;
+            __syncwarp();
+            for (int b = lane; b < nvis; b += 32) {
                 const uint32_t key = fkey(row[b]);
                 if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
             }
-            __syncthreads();
-            if (threadIdx.x < 32) {
-                // the digit d with (keys above d) < need <= (keys at or above d), scanning down
-                const int lane = threadIdx.x;
-                int above = 0, found = -1, found_above = 0;
-                for (int base = 255; base >= 0 && found < 0; base -= 32) {
-                    const int d = base - lane;
-                    const int c = hist[d];
-                    int incl = c;               // inclusive sum over lanes <= lane (digits >= d)
+            __syncwarp();
+            // the digit d with (keys above d) < need <= (keys at or above d): lane l holds the
+            // digits 255 - 8l .. 248 - 8l
+            int cnt[8], tot = 0;
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += n;
+            for (int j = 0; j < 8; ++j) {
+                cnt[j] = hist[255 - 8 * lane - j];
+                tot += cnt[j];
+            }
+            int incl = tot;                       // keys at or above this lane's lowest digit
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += nb;
+            }
+            const int above_lane = incl - tot;     // keys above this lane's digits
+            const bool hit = above_lane < need && incl >= need;
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            const int src = __ffs(m) - 1;
+            int digit = 0, above = 0;
+            if (lane == src) {
+                int acc = above_lane;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (acc + cnt[j] >= need) {
+                        digit = 255 - 8 * lane - j;
+                        above = acc;
+                        break;
                     }
-                    const bool hit = above + incl >= need && above + incl - c < need;
-                    const unsigned m = __ballot_sync(0xffffffffu, hit);
-                    if (m) {
-                        const int src = __ffs(m) - 1;
-                        found = base - src;
-                        found_above = above + __shfl_sync(0xffffffffu, incl - c, src);
-                    }
-                    above += __shfl_sync(0xffffffffu, incl, 31);
-                }
-                if (lane == 0) {
-                    s_digit = found;
-                    s_above = found_above;
+                    acc += cnt[j];
                 }
             }
-            __syncthreads();
-            prefix |= (uint32_t)s_digit << shift;
+            digit = __shfl_sync(0xffffffffu, digit, src);
+            above = __shfl_sync(0xffffffffu, above, src);
+            prefix |= (uint32_t)digit << shift;
             mask |= 255u << shift;
-            need -= s_above;
-            __syncthreads();
+            need -= above;
+            __syncwarp();
         }
     }
-    // gather: every key above the threshold (or every visible key when nvis <= kb), then the
-    // `need` lowest-index keys equal to it
-    if (threadIdx.x == 0) s_count = 0;
-    __syncthreads();
+    // gather in index order: the keys above T (every visible key when nvis <= kb), then the
+    // `need` lowest-index keys equal to T
     const uint32_t T = prefix;
     const bool all = nvis <= kb;
-    for (int b = threadIdx.x; b < nvis; b += kTopkThreads) {
-        const uint32_t key = fkey(row[b]);
-        if (all || key > T) {
-            const int at = atomicAdd(&s_count, 1);
-            sel[at] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)b);
+    int n_gt = 0, n_eq = 0;
+    for (int b0 = 0; b0 < nvis; b0 += 32) {
+        const int b = b0 + lane;
+        const uint32_t key = b < nvis ? fkey(row[b]) : 0u;
+        const bool gt = b < nvis && (all || key > T);
+        const bool eq = b < nvis && !all && key == T;
+        const unsigned mg = __ballot_sync(0xffffffffu, gt), me = __ballot_sync(0xffffffffu, eq);
+        const unsigned below = (1u << lane) - 1u;
+        if (gt) sel[n_gt + __popc(mg & below)] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)b);
+        if (eq) {
+            const int at = n_eq + __popc(me & below);
+            if (at < need) sel[kb - need + at] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)b);
         }
+        n_gt += __popc(mg);
+        n_eq += __popc(me);
     }
-    __syncthreads();
-    if (!all) {
-        const int base_n = s_count;
-        int taken = 0;
-        for (int b0 = 0; b0 < nvis && taken < need; b0 += kTopkThreads) {
-            const int b = b0 + threadIdx.x;
-            const bool eq = b < nvis && fkey(row[b]) == T;
-            int total;
-            const int rank = block_exclusive_sum(eq ? 1 : 0, warp_sums, &total);
-            if (eq && taken + rank < need)
-                sel[base_n + taken + rank] = ((unsigned long long)T << 32) | (0xffffffffu - (uint32_t)b);
-            taken += total;
-            __syncthreads();
-        }
-    }
-    __syncthreads();
-    for (int i = take + threadIdx.x; i < kb2; i += kTopkThreads) sel[i] = 0ull;
-    __syncthreads();
+    __syncwarp();
+    for (int i = take + lane; i < kb2; i += 32) sel[i] = 0ull;
+    __syncwarp();
     // bitonic sort, descending
     for (int k = 2; k <= kb2; k <<= 1)
         for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            for (int i = threadIdx.x; i < kb2; i += kTopkThreads) {
+            for (int i = lane; i < kb2; i += 32) {
                 const int ixj = i ^ jj;
                 if (ixj > i) {
                     const bool desc = (i & k) == 0;
@@ -552,10 +548,10 @@ qsa_topk_kernel(const float *__restrict__ I, const int32_t *__restrict__ cu, int
                     }
                 }
             }
-            __syncthreads();
+            __syncwarp();
         }
     int32_t *out = B + (size_t)t * kb;
-    for (int i = threadIdx.x; i < kb; i += kTopkThreads)
+    for (int i = lane; i < kb; i += 32)
         out[i] = i < take ? (int32_t)(0xffffffffu - (uint32_t)(sel[i] & 0xffffffffull)) : -1;
 }
 
