@@ -643,9 +643,22 @@ def bench_backward(args, inp, device, pg):
         ms = max_over_ranks(pg, a.elapsed_time(b), device) / reps
         status = gdn.device_error(device)
         n_tok = inp["q"].shape[0]
-        return {"kernel": "gdn::gdn_backward_kernel (fp32, one CTA per chain)", "ms_per_launch": ms,
-                "tokens_per_s": n_tok / (ms * 1e-3), "launches": reps, "status": status,
-                "workload": "prefill shape: 4 x 4096 tokens, H=16, d=128, bf16 inputs"}
+        # products of the chunked backward per (chain, 64-token chunk), full C x C tiles:
+        # 28 C^2 d + 20 C d^2 + 4 C^3 FLOP (prep 6 C^2 d; state chain forward 2 C^2 d + 4 C d^2;
+        # state adjoints 2 C^2 d + 6 C d^2; per-slice sums 10 C^2 d + 10 C d^2; dq/dk 8 C^2 d + 4 C^3)
+        C, d, H = 64, inp["q"].shape[2], inp["q"].shape[1]
+        lens = (inp["cu_seqlens"][1:] - inp["cu_seqlens"][:-1]).tolist()
+        n_cc = H * sum(-(-L // C) for L in lens)
+        flops = n_cc * (28 * C * C * d + 20 * C * d * d + 4 * C ** 3)
+        # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the maximum SM clock)
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        tf = flops / (ms * 1e-3) / 1e12
+        return {"kernel": "gdn::bwdc chunked backward (prep, fwd, state, vpart, kpart; fp32 CUDA cores)",
+                "ms_per_launch": ms, "tokens_per_s": n_tok / (ms * 1e-3), "launches": reps, "status": status,
+                "workload": "prefill shape: 4 x 4096 tokens, H=16, d=128, bf16 inputs",
+                "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                             "peak_source": "fp32 FMA rate from 148 SMs x 128 lanes at 1965 MHz",
+                             "flops_per_launch": flops}}
     except Exception as exc:                      # reported, not raised
         return {"error": f"{type(exc).__name__}: {exc}"[:300]}
 

@@ -49,16 +49,13 @@ __host__ __device__ inline ChunkF32Smem chunk_f32_layout(int C, int DK, int DVT)
     return L;
 }
 
-// S_chunks (optional, for the chunked backward): the state at the start of every chunk,
-// [chain][max_chunks][DK][DV] fp32 in the pages' orientation (key index first). y may be
-// NULL (no output rows are computed then).
 template <typename T, typename TY>
 __global__ void __launch_bounds__(kChunkF32Threads)
 chunk_fwd_f32_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                      const float *__restrict__ log_alpha, const float *__restrict__ beta,
                      const float *__restrict__ S0, const int32_t *__restrict__ cu_seqlens,
                      int H, int DK, int DV, int C, int DVT, float scale, TY *__restrict__ y,
-                     float *__restrict__ S_T, float *__restrict__ S_chunks, int max_chunks)
+                     float *__restrict__ S_T)
 {
     extern __shared__ float sm[];
     const ChunkF32Smem L = chunk_f32_layout(C, DK, DVT);
@@ -85,13 +82,6 @@ chunk_fwd_f32_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
     for (int64_t c0 = bos; c0 < eos; c0 += C) {
         const int n = (int)((eos - c0) < C ? (eos - c0) : C);
         __syncthreads();
-        if (S_chunks) {
-            float *dst = S_chunks + ((size_t)chain * max_chunks + (size_t)((c0 - bos) / C)) * DK * DV + v0;
-            for (int i = tid; i < DK * DVT; i += blockDim.x) {
-                const int a = i / DVT, b = i % DVT;
-                dst[(size_t)a * DV + b] = Ss[a * vp + b];
-            }
-        }
         // 1. load the chunk (rows past the sequence end are zero, with beta = log alpha = 0)
         for (int i = tid; i < C * DK; i += blockDim.x) {
             const int t = i / DK, a = i % DK;
@@ -189,7 +179,7 @@ chunk_fwd_f32_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
         // 7. Y = diag(gamma) Q S + P U~  (rows past the end are not stored)
         for (int i = tid; i < C * DVT; i += blockDim.x) {
             const int t = i / DVT, b = i % DVT;
-            if (t >= n || !y) continue;
+            if (t >= n) continue;
             float qs = 0.f;
             for (int a = 0; a < DK; ++a) qs = fmaf(Qs[t * kp + a], Ss[a * vp + b], qs);
             float acc = gam[t] * qs;

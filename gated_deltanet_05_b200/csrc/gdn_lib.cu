@@ -109,7 +109,7 @@ gdn_status launch_chunk_f32(const void *q, const void *k, const void *v, const f
     const unsigned grid = (unsigned)((int64_t)n_seq * H * (dv / dvt));
     kern<<<grid, gdn::kChunkF32Threads, smem, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), la, beta, S0,
-        cu, H, dk, dv, C, dvt, scale, static_cast<TY *>(y), S_T, nullptr, 0);
+        cu, H, dk, dv, C, dvt, scale, static_cast<TY *>(y), S_T);
     return launch_status();
 }
 
@@ -405,10 +405,11 @@ size_t gdn_backward_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, i
         if (l > max_len) max_len = l;
     }
     const int64_t max_chunks = (max_len + gdn::bwdc::kC - 1) / gdn::bwdc::kC;
-    const int n_vt = d_v / (d_v < gdn::bwdc::kDVT ? d_v : gdn::bwdc::kDVT);
-    // per (chain, chunk): the start state and the end-state adjoint [d_k][d_v], and one block
-    // of sums over v per value slice
-    const size_t per_chunk = 2 * (size_t)d_k * d_v + (size_t)n_vt * gdn::bwdc::part_floats(d_k);
+    const int n_vt = d_v / gdn::bwdc::slice_cols(d_v);
+    // per (chain, chunk): the start state and the end-state adjoint [d_k][d_v], the chunk's
+    // cache (T, A o Gamma, P, W), and one block of sums over v per value slice
+    const size_t per_chunk = 2 * (size_t)d_k * d_v + gdn::bwdc::cache_floats(d_k) +
+                             (size_t)n_vt * gdn::bwdc::part_floats(d_k);
     return (size_t)n_seq * H * (size_t)max_chunks * per_chunk * sizeof(float);
 }
 
@@ -441,7 +442,7 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
             max_len = (int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i];
     const int64_t n_chain = (int64_t)n_seq * H;
     const int64_t max_chunks = (max_len + kC - 1) / kC;
-    const int dvt = d_v < kDVT ? d_v : kDVT;
+    const int dvt = slice_cols(d_v);
     const int n_vt = d_v / dvt;
     if (n_chain * n_vt > 0x7fffffffLL || max_chunks > 65535) return GDN_ERR_UNSUPPORTED;
     if (max_chunks == 0) {
@@ -456,39 +457,48 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
         return GDN_OK;
     }
     cudaStream_t st = as_stream(stream);
+    const size_t n_cc = (size_t)n_chain * max_chunks;
     float *S_chunks = static_cast<float *>(workspace);
-    float *dS_chunks = S_chunks + (size_t)n_chain * max_chunks * d_k * d_v;
-    float *parts = dS_chunks + (size_t)n_chain * max_chunks * d_k * d_v;
-    const int smem_f = (int)(chunk_f32_layout(kC, d_k, dvt).total * sizeof(float));
-    const int smem_s = (int)(state_layout(d_k).total * sizeof(float));
-    const int smem_v = (int)(vpart_layout(d_k).total * sizeof(float));
+    float *dS_chunks = S_chunks + n_cc * d_k * d_v;
+    float *cache = dS_chunks + n_cc * d_k * d_v;
+    float *parts = cache + n_cc * cache_floats(d_k);
+    const int smem_p = (int)(prep_layout(d_k).total * sizeof(float));
+    const int smem_f = (int)(fwd_layout(d_k, dvt).total * sizeof(float));
+    const int smem_s = (int)(state_layout(d_k, dvt).total * sizeof(float));
+    const int smem_v = (int)(vpart_layout(d_k, dvt).total * sizeof(float));
     const int smem_k = (int)(kpart_layout(d_k).total * sizeof(float));
     const int optin = smem_optin();
-    if (smem_f > optin || smem_s > optin || smem_v > optin || smem_k > optin) return GDN_ERR_UNSUPPORTED;
+    if (smem_p > optin || smem_f > optin || smem_s > optin || smem_v > optin || smem_k > optin)
+        return GDN_ERR_UNSUPPORTED;
+    const dim3 grid_c((unsigned)n_chain, (unsigned)max_chunks);
     const dim3 grid_v((unsigned)(n_chain * n_vt), (unsigned)max_chunks);
-    const dim3 grid_k((unsigned)n_chain, (unsigned)max_chunks);
+    const unsigned grid_s = (unsigned)(n_chain * n_vt);
 #define GDN_BWD(T)                                                                                   \
     {                                                                                                \
-        auto kf = gdn::chunk_fwd_f32_kernel<T, float>;                                               \
+        auto kp = chunk_bwd_prep_kernel<T>;                                                          \
+        auto kf = chunk_bwd_fwd_kernel<T>;                                                           \
         auto ks = chunk_bwd_state_kernel<T>;                                                         \
         auto kv = chunk_bwd_vpart_kernel<T>;                                                         \
         auto kk = chunk_bwd_kpart_kernel<T>;                                                         \
-        if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f) != cudaSuccess || \
+        if (cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_p) != cudaSuccess || \
+            cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f) != cudaSuccess || \
             cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_s) != cudaSuccess || \
             cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_v) != cudaSuccess || \
             cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)   \
             return GDN_ERR_CUDA;                                                                     \
-        kf<<<(unsigned)(n_chain * n_vt), gdn::kChunkF32Threads, smem_f, st>>>(                       \
-            (const T *)q, (const T *)k, (const T *)v, log_alpha, beta, S0, cu_seqlens_dev, H, d_k, d_v, kC, dvt, \
-            scale, (float *)nullptr, (float *)nullptr, S_chunks, (int)max_chunks);                   \
-        ks<<<(unsigned)(n_chain * n_vt), kThreads, smem_s, st>>>(                                    \
-            (const T *)q, (const T *)k, (const T *)dy, log_alpha, beta, cu_seqlens_dev, H, d_k, d_v, scale, dS_T, \
-            dS_chunks, (int)max_chunks, dS0);                                                        \
-        kv<<<grid_v, kThreads, smem_v, st>>>((const T *)q, (const T *)k, (const T *)v, (const T *)dy, log_alpha, \
-                                             beta, cu_seqlens_dev, H, d_k, d_v, scale, S_chunks, dS_chunks,      \
-                                             (int)max_chunks, parts, dv);                              \
-        kk<<<grid_k, kThreads, smem_k, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
-                                             n_vt, scale, (int)max_chunks, parts, dq, dk, dbeta, dlog_alpha);    \
+        kp<<<grid_c, kThreads, smem_p, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
+                                             scale, (int)max_chunks, cache);                        \
+        kf<<<grid_s, kThreadsWide, smem_f, st>>>((const T *)k, (const T *)v, log_alpha, beta, S0, cu_seqlens_dev, \
+                                                 H, d_k, d_v, (int)max_chunks, cache, S_chunks);    \
+        ks<<<grid_s, kThreadsWide, smem_s, st>>>((const T *)q, (const T *)k, (const T *)dy, log_alpha, beta,     \
+                                                 cu_seqlens_dev, H, d_k, d_v, scale, dS_T, (int)max_chunks,     \
+                                                 cache, dS_chunks, dS0);                            \
+        kv<<<grid_v, kThreadsWide, smem_v, st>>>((const T *)k, (const T *)v, (const T *)dy, log_alpha, beta,     \
+                                                 cu_seqlens_dev, H, d_k, d_v, (int)max_chunks, cache, S_chunks, \
+                                                 dS_chunks, parts, dv);                             \
+        kk<<<grid_c, kThreads, smem_k, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
+                                             n_vt, scale, (int)max_chunks, cache, parts, dq, dk, dbeta,  \
+                                             dlog_alpha);                                           \
     }
     if (in_dtype == GDN_F32)
         GDN_BWD(float)
