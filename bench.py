@@ -731,7 +731,8 @@ def run_case(args):
     --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)
     --case featurize:S,T,H (bf16, d=128, conv width 4)
     --case decode_tokens:N,T (N sequences x 32 heads, d=128, T tokens per call)
-    --case qsa:N           (the QSA indexer on one N-token sequence, Hq=4, r=4, K=2048, bf16)"""
+    --case qsa:N           (the QSA indexer on one N-token sequence, Hq=4, r=4, K=2048, bf16)
+    --case backward:S,T,H  (gdn_backward, bf16 inputs, d=128, a bf16 cotangent of y)"""
     import torch
 
     import gated_deltanet_05_b200 as gdn
@@ -794,6 +795,14 @@ def run_case(args):
         dev = [inp[k].cuda() for k in keys]
         for _ in range(args.reps):
             gdn.featurize(*dev, cu_seqlens_host=inp["cu_seqlens"])
+    elif kind == "backward":
+        n_seq, T, H = dims
+        w = W.Workload("case", "bf16", (T,) * n_seq, H, 128, 128, 64, seed=1)
+        inp = W.make_prefill_inputs(w)
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        for _ in range(args.reps):
+            gdn.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"], d["z"],
+                         cu_seqlens_host=inp["cu_seqlens"])
     else:
         raise SystemExit(f"unknown case {args.case}")
     torch.cuda.synchronize()

@@ -32,9 +32,10 @@
 //                           sums over v that the rest needs (dP, dT, dW, dK~, dY S^T, ...), each
 //                           slice into its own block (no atomics: the result is deterministic)
 //   chunk_bwd_kpart_kernel  per (chain, chunk), all at once: dQ, dK, dbeta, dlog_alpha
-// Every matrix product runs from shared memory with a register tile per thread (rows and
-// columns interleaved across threads; odd row strides keep the lanes of a warp on distinct
-// banks).
+// Every matrix product runs from shared memory: a thread owns a 4 x 4 (or 4 x 2) tile of the
+// result and loads both operands as float4 along their contiguous dimension, four k-steps at
+// a time (8 vector loads per 64 FMAs); rows are padded to a multiple of 4 plus 4 floats so
+// that the lanes of a warp read distinct banks.
 #pragma once
 #include "gdn_common.cuh"
 
@@ -43,13 +44,19 @@ namespace bwdc {
 
 constexpr int kC = 64;               // chunk length
 constexpr int kDVT = 64;             // value columns per CTA in the sliced steps
-constexpr int kThreads = 256;        // prep and kpart
-constexpr int kThreadsWide = 512;    // fwd, state and vpart
+constexpr int kThreads = 256;        // prep
+constexpr int kThreadsWide = 512;    // fwd, state, vpart and kpart
 
 __host__ __device__ inline int slice_cols(int DV) { return DV < kDVT ? DV : kDVT; }
+// shared-memory row stride for rows of D floats (D a multiple of 8): 16-byte aligned rows
+// whose float4 slots fall on distinct banks for 8 consecutive rows
+__host__ __device__ inline int ldp(int D) { return D + 4; }
 // floats of the per-chunk sums block of one value slice: dP, dT [C][C]; dW, dK~, dY S^T
-// [C][DK]; the row sums of V o T^T dU~ [C]; <dS', S> [1]
-__host__ __device__ inline size_t part_floats(int DK) { return (size_t)kC * (2 * kC + 3 * DK + 1) + 1; }
+// [C][DK]; the row sums of V o T^T dU~ [C]; <dS', S> [1]; rounded up to a multiple of 4
+__host__ __device__ inline size_t part_floats(int DK)
+{
+    return ((size_t)kC * (2 * kC + 3 * DK + 1) + 1 + 3) & ~(size_t)3;
+}
 // floats of the per-chunk cache: T, A o Gamma, P [C][C] and W [C][DK]
 __host__ __device__ inline size_t cache_floats(int DK) { return (size_t)kC * (3 * kC + DK); }
 constexpr int kCacheT = 0, kCacheAG = kC * kC, kCacheP = 2 * kC * kC, kCacheW = 3 * kC * kC;
@@ -81,60 +88,140 @@ __device__ __forceinline__ void chunk_decays(const float *__restrict__ log_alpha
     for (int t = lane; t < kC; t += 32) Dd[t] = expf(gC - g[t]);
 }
 
-// Rows of a chunk into shared memory [kC][ld] (zero past n), optionally scaled.
+__device__ __forceinline__ float4 f4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ void st4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ float4 scale4(float4 v, float f) { return make_float4(v.x * f, v.y * f, v.z * f, v.w * f); }
+__device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+
+// Columns [col0, col0 + ncol) of a chunk's rows of a token-major [.., H, D] tensor into shared
+// memory [kC][ld] (zero past n), times f. ncol, col0 and D multiples of 4.
 template <typename T>
 __device__ __forceinline__ void load_rows(float *dst, int ld, const T *__restrict__ src, int64_t c0, int n, int H,
                                           int h, int D, int col0, int ncol, float f)
 {
-    for (int i = threadIdx.x; i < kC * ncol; i += blockDim.x) {
-        const int t = i / ncol, a = i % ncol;
-        dst[t * ld + a] = t < n ? f * to_f32(src[((size_t)(c0 + t) * H + h) * D + col0 + a]) : 0.f;
-    }
-}
-
-// A row-major block of the cache into shared memory with a padded stride.
-__device__ __forceinline__ void load_block(float *dst, int ld, const float *__restrict__ src, int rows, int cols)
-{
-    for (int i = threadIdx.x; i < rows * cols; i += blockDim.x) dst[(i / cols) * ld + i % cols] = src[i];
-}
-
-// acc[i][j] += sum_k a(m_i, k) b(k, n_j) over k < K, for one thread's tile: rows
-// m_i = tm + i ntm, columns n_j = tn + j ntn.
-template <int TM, int TN, class FA, class FB>
-__device__ __forceinline__ void mm_acc(float (&acc)[TM][TN], int tm, int tn, int ntm, int ntn, int K, FA a, FB b)
-{
+    const int nq = ncol >> 2;
 #pragma unroll 4
-    for (int kk = 0; kk < K; ++kk) {
-        float av[TM], bv[TN];
-#pragma unroll
-        for (int i = 0; i < TM; ++i) av[i] = a(tm + i * ntm, kk);
-#pragma unroll
-        for (int j = 0; j < TN; ++j) bv[j] = b(kk, tn + j * ntn);
-#pragma unroll
-        for (int i = 0; i < TM; ++i)
-#pragma unroll
-            for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    for (int i = threadIdx.x; i < kC * nq; i += blockDim.x) {
+        const int t = i / nq, a = (i % nq) * 4;
+        const float4 x = t < n ? scale4(load4(src + ((size_t)(c0 + t) * H + h) * D + col0 + a), f)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        st4(dst + t * ld + a, x);
     }
 }
 
-template <int TM, int TN>
-__device__ __forceinline__ void zero(float (&acc)[TM][TN])
+// The same rows stored transposed: dst[a][t] = src[t][a], [ncol][ld].
+template <typename T>
+__device__ __forceinline__ void load_rows_t(float *dst, int ld, const T *__restrict__ src, int64_t c0, int n, int H,
+                                            int h, int D, int ncol)
+{
+    const int nq = ncol >> 2;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < kC * nq; i += blockDim.x) {
+        const int t = i / nq, a = (i % nq) * 4;
+        const float4 x = t < n ? load4(src + ((size_t)(c0 + t) * H + h) * D + a) : make_float4(0.f, 0.f, 0.f, 0.f);
+        dst[(a + 0) * ld + t] = x.x;
+        dst[(a + 1) * ld + t] = x.y;
+        dst[(a + 2) * ld + t] = x.z;
+        dst[(a + 3) * ld + t] = x.w;
+    }
+}
+
+// A row-major [rows][cols] fp32 block (global, 16-byte aligned) into shared memory [rows][ld],
+// times f.
+__device__ __forceinline__ void load_block(float *dst, int ld, const float *__restrict__ src, int rows, int cols,
+                                           float f)
+{
+    const int nq = cols >> 2;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < rows * nq; i += blockDim.x) {
+        const int r = i / nq, c = (i % nq) * 4;
+        st4(dst + r * ld + c, scale4(f4(src + (size_t)r * cols + c), f));
+    }
+}
+
+// ---- register-tiled products from shared memory ------------------------------------------
+// C[M][N] += A[M][K] B[K][N]. A thread owns 4 rows x TN columns (TN = 4 or 2). A is stored
+// either [m][k] (AMK: rows interleave across threads, m_i = tm + i ntm, each row read as
+// float4 along k) or [k][m] (rows contiguous, m_i = 4 tm + i, read as float4 along m); B is
+// stored [k][n] (BKN: columns contiguous, n_j = TN tn + j) or [n][k] (columns interleave,
+// n_j = tn + j ntn, each read as float4 along k). Within a warp 8 row groups x 4 column
+// groups where the sizes allow, so each vector load covers at most 128 distinct bytes.
+// M, N, K multiples of 16 (K of 4); strides ldp(...); bases 16-byte aligned.
+template <int TN, bool AMK, bool BKN>
+struct Tile {
+    int tm, tn, ntm, ntn;
+    __device__ __forceinline__ Tile(int gi, int M, int N)
+    {
+        ntm = M >> 2;
+        ntn = N / TN;
+        if ((ntm & 7) == 0 && (ntn & 3) == 0) {
+            const int lane = gi & 31, w = gi >> 5, wm = ntm >> 3;
+            tm = (w % wm) * 8 + (lane & 7);
+            tn = (w / wm) * 4 + (lane >> 3);
+        } else {
+            tm = gi % ntm;
+            tn = gi / ntm;
+        }
+    }
+    __device__ __forceinline__ int row(int i) const { return AMK ? tm + i * ntm : 4 * tm + i; }
+    __device__ __forceinline__ int col(int j) const { return BKN ? TN * tn + j : tn + j * ntn; }
+    __device__ __forceinline__ void run(float (&acc)[4][TN], int K, const float *__restrict__ A, int lda,
+                                        const float *__restrict__ B, int ldb) const
+    {
+#pragma unroll 2
+        for (int k = 0; k < K; k += 4) {
+            float a[4][4], b[4][TN];             // a[i][kk], b[kk][j]
+            if (AMK) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 v = f4(A + row(i) * lda + k);
+                    a[i][0] = v.x; a[i][1] = v.y; a[i][2] = v.z; a[i][3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float4 v = f4(A + (k + kk) * lda + 4 * tm);
+                    a[0][kk] = v.x; a[1][kk] = v.y; a[2][kk] = v.z; a[3][kk] = v.w;
+                }
+            }
+            if (BKN) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    if constexpr (TN == 4) {
+                        const float4 v = f4(B + (k + kk) * ldb + 4 * tn);
+                        b[kk][0] = v.x; b[kk][1] = v.y; b[kk][2] = v.z; b[kk][3] = v.w;
+                    } else {
+                        const float2 v = *reinterpret_cast<const float2 *>(B + (k + kk) * ldb + 2 * tn);
+                        b[kk][0] = v.x; b[kk][1] = v.y;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < TN; ++j) {
+                    const float4 v = f4(B + col(j) * ldb + k);
+                    b[0][j] = v.x; b[1][j] = v.y; b[2][j] = v.z; b[3][j] = v.w;
+                }
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i][kk], b[kk][j], acc[i][j]);
+        }
+    }
+};
+
+template <int TN>
+__device__ __forceinline__ void zero(float (&acc)[4][TN])
 {
 #pragma unroll
-    for (int i = 0; i < TM; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
 }
 
-// Sum over the `width` consecutive lanes that share a tile row (width a power of two <= 32;
-// every lane of the warp takes part).
-__device__ __forceinline__ float row_group_sum(float x, int width)
-{
-    for (int off = width >> 1; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-    return x;
-}
-
-// Chunk geometry of (chain, chunk c): first token, valid rows; false past the sequence end.
+// Chunk geometry of (sequence seq, chunk c): first token and valid rows; false past the end.
 __device__ __forceinline__ bool chunk_of(const int32_t *__restrict__ cu_seqlens, int seq, int c, int64_t &c0, int &n)
 {
     const int64_t bos = cu_seqlens[seq], len = (int64_t)cu_seqlens[seq + 1] - bos;
@@ -152,8 +239,8 @@ __host__ __device__ inline PrepSmem prep_layout(int DK)
 {
     PrepSmem L;
     int o = 0;
-    const int kp = DK + 1, cp = kC + 1;
-    L.KQ = o; o += 2 * kC * kp;
+    const int kq = ldp(DK), cp = ldp(kC);
+    L.KQ = o; o += 2 * kC * kq;
     L.Ls = o; o += kC * cp;
     L.Ts = o; o += kC * cp;
     L.g = o; o += kC;
@@ -172,11 +259,11 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
                       const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int H, int DK,
                       float scale, int max_chunks, float *__restrict__ cache)
 {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     const PrepSmem Y = prep_layout(DK);
     float *KQ = sm + Y.KQ, *Ls = sm + Y.Ls, *Ts = sm + Y.Ts;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd;
-    const int kp = DK + 1, cp = kC + 1;
+    const int kq = ldp(DK), cp = ldp(kC);
     const int c = blockIdx.y, chain = blockIdx.x;
     const int seq = chain / H, h = chain % H;
     const int tid = threadIdx.x;
@@ -184,33 +271,29 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
     int n;
     if (!chunk_of(cu_seqlens, seq, c, c0, n)) return;
     float *cb = cache + ((size_t)chain * max_chunks + c) * cache_floats(DK);
-    load_rows(KQ, kp, k, c0, n, H, h, DK, 0, DK, 1.f);
-    load_rows(KQ + kC * kp, kp, q, c0, n, H, h, DK, 0, DK, scale);
+    load_rows(KQ, kq, k, c0, n, H, h, DK, 0, DK, 1.f);
+    load_rows(KQ + kC * kq, kq, q, c0, n, H, h, DK, 0, DK, scale);
     if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
     for (int i = tid; i < kC * kC; i += blockDim.x) Ts[(i / kC) * cp + i % kC] = (i / kC == i % kC) ? 1.f : 0.f;
     __syncthreads();
-    {
-        constexpr int TM = 8, TN = 4;
-        const int ntm = 2 * kC / TM, ntn = kC / TN;
-        for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-            const int tm = gi / ntn, tn = gi % ntn;
-            float acc[TM][TN];
-            zero(acc);
-            mm_acc(acc, tm, tn, ntm, ntn, DK, [&](int m, int a) { return KQ[m * kp + a]; },
-                   [&](int a, int s) { return KQ[s * kp + a]; });
+    // [K; Q] K^T: A = KQ [m][a], B(a, s) = K[s][a] stored [n][k]
+    for (int gi = tid; gi < (2 * kC / 4) * (kC / 4); gi += blockDim.x) {
+        const Tile<4, true, false> tl(gi, 2 * kC, kC);
+        float acc[4][4];
+        zero(acc);
+        tl.run(acc, DK, KQ, kq, KQ, kq);
 #pragma unroll
-            for (int i = 0; i < TM; ++i) {
-                const int m = tm + i * ntm, t = m & (kC - 1);
+        for (int i = 0; i < 4; ++i) {
+            const int m = tl.row(i), t = m & (kC - 1);
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const int s = tn + j * ntn;
-                    const float x = s <= t ? acc[i][j] * expf(g[t] - g[s]) : 0.f;
-                    if (m < kC) {
-                        cb[kCacheAG + t * kC + s] = x;
-                        Ls[t * cp + s] = s < t ? bet[t] * x : 0.f;
-                    } else {
-                        cb[kCacheP + t * kC + s] = x;
-                    }
+            for (int j = 0; j < 4; ++j) {
+                const int s = tl.col(j);
+                const float x = s <= t ? acc[i][j] * expf(g[t] - g[s]) : 0.f;
+                if (m < kC) {
+                    cb[kCacheAG + t * kC + s] = x;
+                    Ls[t * cp + s] = s < t ? bet[t] * x : 0.f;
+                } else {
+                    cb[kCacheP + t * kC + s] = x;
                 }
             }
         }
@@ -229,44 +312,42 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
             __syncthreads();
         }
     }
-    for (int i = tid; i < kC * kC; i += blockDim.x) cb[kCacheT + i] = Ts[(i / kC) * cp + i % kC];
-    for (int i = tid; i < kC * DK; i += blockDim.x) {
-        const int s = i / DK;
-        KQ[s * kp + i % DK] *= bet[s] * gam[s];
+    for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
+        const int r = i / (kC / 4), c4 = (i % (kC / 4)) * 4;
+        st4(cb + kCacheT + r * kC + c4, f4(Ts + r * cp + c4));
+    }
+    for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
+        const int s = i / (DK / 4), a = (i % (DK / 4)) * 4;
+        st4(KQ + s * kq + a, scale4(f4(KQ + s * kq + a), bet[s] * gam[s]));
     }
     __syncthreads();
-    {
-        constexpr int TM = 8, TN = 4;
-        const int ntm = kC / TM, ntn = DK / TN;
-        for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-            const int tm = gi / ntn, tn = gi % ntn;
-            float acc[TM][TN];
-            zero(acc);
-            mm_acc(acc, tm, tn, ntm, ntn, kC, [&](int t, int s) { return Ts[t * cp + s]; },
-                   [&](int s, int a) { return KQ[s * kp + a]; });
+    // W = T (diag(beta gamma) K): A = T [t][s], B = K scaled [s][a]
+    for (int gi = tid; gi < (kC / 4) * (DK / 4); gi += blockDim.x) {
+        const Tile<4, true, true> tl(gi, kC, DK);
+        float acc[4][4];
+        zero(acc);
+        tl.run(acc, kC, Ts, cp, KQ, kq);
 #pragma unroll
-            for (int i = 0; i < TM; ++i)
-#pragma unroll
-                for (int j = 0; j < TN; ++j) cb[kCacheW + (tm + i * ntm) * DK + tn + j * ntn] = acc[i][j];
-        }
+        for (int i = 0; i < 4; ++i)
+            st4(cb + kCacheW + tl.row(i) * DK + 4 * tl.tn, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
     }
 }
 
 // --------------------------------------------------------------------------- fwd
 struct FwdSmem {
-    int Kd, Ws, Ts, Vb, Us, Ss, g, gam, bet, Dd, total;
+    int Kd, Wn, Ts, Vb, Us, Ss, g, gam, bet, Dd, total;
 };
 __host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT)
 {
     FwdSmem L;
     int o = 0;
-    const int kp = DK + 1, vp = DVT + 1, cp = kC + 1;
-    L.Kd = o; o += kC * kp;
-    L.Ws = o; o += kC * kp;
+    const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
+    L.Kd = o; o += kC * kq;
+    L.Wn = o; o += kC * kq;
     L.Ts = o; o += kC * cp;
-    L.Vb = o; o += kC * vp;
-    L.Us = o; o += kC * vp;
-    L.Ss = o; o += DK * vp;
+    L.Vb = o; o += kC * vq;
+    L.Us = o; o += kC * vq;
+    L.Ss = o; o += DK * vq;
     L.g = o; o += kC;
     L.gam = o; o += kC;
     L.bet = o; o += kC;
@@ -285,12 +366,12 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
                      const int32_t *__restrict__ cu_seqlens, int H, int DK, int DV, int max_chunks,
                      const float *__restrict__ cache, float *__restrict__ S_chunks)
 {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
     const FwdSmem Y = fwd_layout(DK, DVT);
-    float *Kd = sm + Y.Kd, *Ws = sm + Y.Ws, *Ts = sm + Y.Ts, *Vb = sm + Y.Vb, *Us = sm + Y.Us, *Ss = sm + Y.Ss;
+    float *Kd = sm + Y.Kd, *Wn = sm + Y.Wn, *Ts = sm + Y.Ts, *Vb = sm + Y.Vb, *Us = sm + Y.Us, *Ss = sm + Y.Ss;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd;
-    const int kp = DK + 1, vp = DVT + 1, cp = kC + 1;
+    const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
     const int n_vt = DV / DVT;
     const int chain = blockIdx.x / n_vt, v0 = (blockIdx.x % n_vt) * DVT;
     const int seq = chain / H, h = chain % H;
@@ -299,9 +380,10 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
     const size_t st_off = (size_t)chain * DV * DK;
     for (int i = tid; i < DK * DVT; i += blockDim.x) {
         const int a = i % DK, b = i / DK;
-        Ss[a * vp + b] = S0 ? S0[st_off + (size_t)(v0 + b) * DK + a] : 0.f;
+        Ss[a * vq + b] = S0 ? S0[st_off + (size_t)(v0 + b) * DK + a] : 0.f;
     }
     const int n_chunks = (int)((len + kC - 1) / kC);
+    const int nvq = DVT / 4;
     for (int c = 0; c < n_chunks; ++c) {
         int64_t c0;
         int n;
@@ -310,78 +392,73 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
         __syncthreads();
         {
             float *dst = S_chunks + ((size_t)chain * max_chunks + c) * DK * DV + v0;
-            for (int i = tid; i < DK * DVT; i += blockDim.x) {
-                const int a = i / DVT, b = i % DVT;
-                dst[(size_t)a * DV + b] = Ss[a * vp + b];
+            for (int i = tid; i < DK * nvq; i += blockDim.x) {
+                const int a = i / nvq, b = (i % nvq) * 4;
+                st4(dst + (size_t)a * DV + b, f4(Ss + a * vq + b));
             }
         }
-        load_rows(Kd, kp, k, c0, n, H, h, DK, 0, DK, 1.f);
-        load_rows(Vb, vp, v, c0, n, H, h, DV, v0, DVT, 1.f);
-        load_block(Ts, cp, cb + kCacheT, kC, kC);
-        load_block(Ws, kp, cb + kCacheW, kC, DK);
+        load_rows(Kd, kq, k, c0, n, H, h, DK, 0, DK, 1.f);
+        load_rows(Vb, vq, v, c0, n, H, h, DV, v0, DVT, 1.f);
+        load_block(Ts, cp, cb + kCacheT, kC, kC, 1.f);
+        load_block(Wn, kq, cb + kCacheW, kC, DK, -1.f);
         if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
         __syncthreads();
-        for (int i = tid; i < kC * DK; i += blockDim.x) Kd[(i / DK) * kp + i % DK] *= Dd[i / DK];
-        for (int i = tid; i < kC * DVT; i += blockDim.x) Vb[(i / DVT) * vp + i % DVT] *= bet[i / DVT];
-        __syncthreads();
-        // U~ = T diag(beta) V - W S
-        {
-            constexpr int TM = 4, TN = 2;
-            const int ntm = kC / TM, ntn = DVT / TN;
-            for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-                const int tm = gi / ntn, tn = gi % ntn;
-                float acc[TM][TN];
-                zero(acc);
-                mm_acc(acc, tm, tn, ntm, ntn, kC, [&](int t, int s) { return Ts[t * cp + s]; },
-                       [&](int s, int b) { return Vb[s * vp + b]; });
-                mm_acc(acc, tm, tn, ntm, ntn, DK, [&](int t, int a) { return -Ws[t * kp + a]; },
-                       [&](int a, int b) { return Ss[a * vp + b]; });
-#pragma unroll
-                for (int i = 0; i < TM; ++i)
-#pragma unroll
-                    for (int j = 0; j < TN; ++j) Us[(tm + i * ntm) * vp + tn + j * ntn] = acc[i][j];
-            }
+        for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
+            const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
+            st4(Kd + t * kq + a, scale4(f4(Kd + t * kq + a), Dd[t]));
+        }
+        for (int i = tid; i < kC * nvq; i += blockDim.x) {
+            const int t = i / nvq, b = (i % nvq) * 4;
+            st4(Vb + t * vq + b, scale4(f4(Vb + t * vq + b), bet[t]));
         }
         __syncthreads();
-        // S <- gamma_C S + (diag(D) K)^T U~ (each thread reads and writes only its own entries of S)
-        {
-            constexpr int TM = 4, TN = 4;
-            const int ntm = DK / TM, ntn = DVT / TN;
-            const float gamC = gam[kC - 1];
-            for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-                const int tm = gi / ntn, tn = gi % ntn;
-                float acc[TM][TN];
+        // U~ = T diag(beta) V - W S
+        for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
+            const Tile<2, true, true> tl(gi, kC, DVT);
+            float acc[4][2];
+            zero(acc);
+            tl.run(acc, kC, Ts, cp, Vb, vq);
+            tl.run(acc, DK, Wn, kq, Ss, vq);
 #pragma unroll
-                for (int i = 0; i < TM; ++i)
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float2 *>(Us + tl.row(i) * vq + 2 * tl.tn) = make_float2(acc[i][0], acc[i][1]);
+        }
+        __syncthreads();
+        // S <- gamma_C S + (diag(D) K)^T U~: A(a, s) = Kd[s][a] stored [k][m]; each thread reads
+        // and writes only its own entries of S
+        const float gamC = gam[kC - 1];
+        for (int gi = tid; gi < (DK / 4) * (DVT / 4); gi += blockDim.x) {
+            const Tile<4, false, true> tl(gi, DK, DVT);
+            float acc[4][4];
 #pragma unroll
-                    for (int j = 0; j < TN; ++j) acc[i][j] = gamC * Ss[(tm + i * ntm) * vp + tn + j * ntn];
-                mm_acc(acc, tm, tn, ntm, ntn, kC, [&](int a, int s) { return Kd[s * kp + a]; },
-                       [&](int s, int b) { return Us[s * vp + b]; });
-#pragma unroll
-                for (int i = 0; i < TM; ++i)
-#pragma unroll
-                    for (int j = 0; j < TN; ++j) Ss[(tm + i * ntm) * vp + tn + j * ntn] = acc[i][j];
+            for (int i = 0; i < 4; ++i) {
+                const float4 x = f4(Ss + tl.row(i) * vq + 4 * tl.tn);
+                acc[i][0] = gamC * x.x; acc[i][1] = gamC * x.y; acc[i][2] = gamC * x.z; acc[i][3] = gamC * x.w;
             }
+            tl.run(acc, kC, Kd, kq, Us, vq);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                st4(Ss + tl.row(i) * vq + 4 * tl.tn, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
         }
     }
 }
 
 // --------------------------------------------------------------------------- state
 struct StateSmem {
-    int Kd, Qg, Ws, Ps, dYs, dUs, dSs, g, gam, bet, Dd, total;
+    int Kt, Qg, Wn, Ps, dYs, dUs, dSs, g, gam, bet, Dd, total;
 };
 __host__ __device__ inline StateSmem state_layout(int DK, int DVT)
 {
     StateSmem L;
     int o = 0;
-    const int kp = DK + 1, vp = DVT + 1, cp = kC + 1;
-    L.Kd = o; o += kC * kp;
-    L.Qg = o; o += kC * kp;
-    L.Ws = o; o += kC * kp;
+    const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
+    L.Kt = o; o += DK * cp;
+    L.Qg = o; o += kC * kq;
+    L.Wn = o; o += kC * kq;
     L.Ps = o; o += kC * cp;
-    L.dYs = o; o += kC * vp;
-    L.dUs = o; o += kC * vp;
-    L.dSs = o; o += DK * vp;
+    L.dYs = o; o += kC * vq;
+    L.dUs = o; o += kC * vq;
+    L.dSs = o; o += DK * vq;
     L.g = o; o += kC;
     L.gam = o; o += kC;
     L.bet = o; o += kC;
@@ -401,13 +478,13 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                        const float *__restrict__ dS_T, int max_chunks, const float *__restrict__ cache,
                        float *__restrict__ dS_chunks, float *__restrict__ dS0)
 {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
     const StateSmem Y = state_layout(DK, DVT);
-    float *Kd = sm + Y.Kd, *Qg = sm + Y.Qg, *Ws = sm + Y.Ws, *Ps = sm + Y.Ps;
+    float *Kt = sm + Y.Kt, *Qg = sm + Y.Qg, *Wn = sm + Y.Wn, *Ps = sm + Y.Ps;
     float *dYs = sm + Y.dYs, *dUs = sm + Y.dUs, *dSs = sm + Y.dSs;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd;
-    const int kp = DK + 1, vp = DVT + 1, cp = kC + 1;
+    const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
     const int n_vt = DV / DVT;
     const int chain = blockIdx.x / n_vt, v0 = (blockIdx.x % n_vt) * DVT;
     const int seq = chain / H, h = chain % H;
@@ -416,9 +493,10 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     const size_t st_off = (size_t)chain * DV * DK;
     for (int i = tid; i < DK * DVT; i += blockDim.x) {
         const int a = i % DK, b = i / DK;
-        dSs[a * vp + b] = dS_T ? dS_T[st_off + (size_t)(v0 + b) * DK + a] : 0.f;
+        dSs[a * vq + b] = dS_T ? dS_T[st_off + (size_t)(v0 + b) * DK + a] : 0.f;
     }
     const int n_chunks = (int)((len + kC - 1) / kC);
+    const int nvq = DVT / 4;
     for (int c = n_chunks - 1; c >= 0; --c) {
         int64_t c0;
         int n;
@@ -427,93 +505,84 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         __syncthreads();
         {
             float *dst = dS_chunks + ((size_t)chain * max_chunks + c) * DK * DV + v0;
-            for (int i = tid; i < DK * DVT; i += blockDim.x) {
-                const int a = i / DVT, b = i % DVT;
-                dst[(size_t)a * DV + b] = dSs[a * vp + b];
+            for (int i = tid; i < DK * nvq; i += blockDim.x) {
+                const int a = i / nvq, b = (i % nvq) * 4;
+                st4(dst + (size_t)a * DV + b, f4(dSs + a * vq + b));
             }
         }
-        load_rows(Kd, kp, k, c0, n, H, h, DK, 0, DK, 1.f);
-        load_rows(Qg, kp, q, c0, n, H, h, DK, 0, DK, scale);
-        load_rows(dYs, vp, dy, c0, n, H, h, DV, v0, DVT, 1.f);
-        load_block(Ws, kp, cb + kCacheW, kC, DK);
-        load_block(Ps, cp, cb + kCacheP, kC, kC);
+        load_rows_t(Kt, cp, k, c0, n, H, h, DK, DK);
+        load_rows(Qg, kq, q, c0, n, H, h, DK, 0, DK, scale);
+        load_rows(dYs, vq, dy, c0, n, H, h, DV, v0, DVT, 1.f);
+        load_block(Wn, kq, cb + kCacheW, kC, DK, -1.f);
+        load_block(Ps, cp, cb + kCacheP, kC, kC, 1.f);
         if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
         __syncthreads();
-        for (int i = tid; i < kC * DK; i += blockDim.x) {
-            const int t = i / DK, a = i % DK;
-            Kd[t * kp + a] *= Dd[t];
-            Qg[t * kp + a] *= gam[t];
+        for (int i = tid; i < DK * kC / 4; i += blockDim.x) {
+            const int a = i / (kC / 4), t = (i % (kC / 4)) * 4;
+            const float4 x = f4(Kt + a * cp + t);
+            st4(Kt + a * cp + t, make_float4(x.x * Dd[t], x.y * Dd[t + 1], x.z * Dd[t + 2], x.w * Dd[t + 3]));
+        }
+        for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
+            const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
+            st4(Qg + t * kq + a, scale4(f4(Qg + t * kq + a), gam[t]));
         }
         __syncthreads();
-        // dU~ = P^T dY + diag(D) K dS'
-        {
-            constexpr int TM = 4, TN = 2;
-            const int ntm = kC / TM, ntn = DVT / TN;
-            for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-                const int tm = gi / ntn, tn = gi % ntn;
-                float acc[TM][TN];
-                zero(acc);
-                mm_acc(acc, tm, tn, ntm, ntn, kC, [&](int s, int t) { return Ps[t * cp + s]; },
-                       [&](int t, int b) { return dYs[t * vp + b]; });
-                mm_acc(acc, tm, tn, ntm, ntn, DK, [&](int s, int a) { return Kd[s * kp + a]; },
-                       [&](int a, int b) { return dSs[a * vp + b]; });
+        // dU~ = P^T dY + diag(D) K dS': A(s, t) = P[t][s] and A(s, a) = Kd^T[a][s], both [k][m]
+        for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
+            const Tile<2, false, true> tl(gi, kC, DVT);
+            float acc[4][2];
+            zero(acc);
+            tl.run(acc, kC, Ps, cp, dYs, vq);
+            tl.run(acc, DK, Kt, cp, dSs, vq);
 #pragma unroll
-                for (int i = 0; i < TM; ++i)
-#pragma unroll
-                    for (int j = 0; j < TN; ++j) dUs[(tm + i * ntm) * vp + tn + j * ntn] = acc[i][j];
-            }
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float2 *>(dUs + tl.row(i) * vq + 2 * tl.tn) = make_float2(acc[i][0], acc[i][1]);
         }
         __syncthreads();
         // dS = gamma_C dS' + (diag(gamma) Q)^T dY - W^T dU~ (own entries of dS only)
-        {
-            constexpr int TM = 4, TN = 4;
-            const int ntm = DK / TM, ntn = DVT / TN;
-            const float gamC = gam[kC - 1];
-            for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-                const int tm = gi / ntn, tn = gi % ntn;
-                float acc[TM][TN];
+        const float gamC = gam[kC - 1];
+        for (int gi = tid; gi < (DK / 4) * (DVT / 4); gi += blockDim.x) {
+            const Tile<4, false, true> tl(gi, DK, DVT);
+            float acc[4][4];
 #pragma unroll
-                for (int i = 0; i < TM; ++i)
-#pragma unroll
-                    for (int j = 0; j < TN; ++j) acc[i][j] = gamC * dSs[(tm + i * ntm) * vp + tn + j * ntn];
-                mm_acc(acc, tm, tn, ntm, ntn, kC, [&](int a, int t) { return Qg[t * kp + a]; },
-                       [&](int t, int b) { return dYs[t * vp + b]; });
-                mm_acc(acc, tm, tn, ntm, ntn, kC, [&](int a, int t) { return -Ws[t * kp + a]; },
-                       [&](int t, int b) { return dUs[t * vp + b]; });
-#pragma unroll
-                for (int i = 0; i < TM; ++i)
-#pragma unroll
-                    for (int j = 0; j < TN; ++j) dSs[(tm + i * ntm) * vp + tn + j * ntn] = acc[i][j];
+            for (int i = 0; i < 4; ++i) {
+                const float4 x = f4(dSs + tl.row(i) * vq + 4 * tl.tn);
+                acc[i][0] = gamC * x.x; acc[i][1] = gamC * x.y; acc[i][2] = gamC * x.z; acc[i][3] = gamC * x.w;
             }
+            tl.run(acc, kC, Qg, kq, dYs, vq);
+            tl.run(acc, kC, Wn, kq, dUs, vq);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                st4(dSs + tl.row(i) * vq + 4 * tl.tn, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
         }
     }
     __syncthreads();
     if (dS0)
         for (int i = tid; i < DK * DVT; i += blockDim.x) {
             const int a = i % DK, b = i / DK;
-            dS0[st_off + (size_t)(v0 + b) * DK + a] = dSs[a * vp + b];
+            dS0[st_off + (size_t)(v0 + b) * DK + a] = dSs[a * vq + b];
         }
 }
 
 // --------------------------------------------------------------------------- vpart
 struct VpartSmem {
-    int Ks, Ts, Ps, Ss, dSs, Vs, dYs, Uts, dUs, Zs, g, gam, bet, Dd, red, total;
+    int Kt, Ts, Ps, Ss, dSs, Vs, dYs, Uts, dUs, Zs, g, gam, bet, Dd, red, total;
 };
 __host__ __device__ inline VpartSmem vpart_layout(int DK, int DVT)
 {
     VpartSmem L;
     int o = 0;
-    const int kp = DK + 1, vp = DVT + 1, cp = kC + 1;
-    L.Ks = o; o += kC * kp;
+    const int vq = ldp(DVT), cp = ldp(kC);
+    L.Kt = o; o += DK * cp;
     L.Ts = o; o += kC * cp;
     L.Ps = o; o += kC * cp;
-    L.Ss = o; o += DK * vp;
-    L.dSs = o; o += DK * vp;
-    L.Vs = o; o += kC * vp;
-    L.dYs = o; o += kC * vp;
-    L.Uts = o; o += kC * vp;
-    L.dUs = o; o += kC * vp;
-    L.Zs = o; o += kC * vp;
+    L.Ss = o; o += DK * vq;
+    L.dSs = o; o += DK * vq;
+    L.Vs = o; o += kC * vq;
+    L.dYs = o; o += kC * vq;
+    L.Uts = o; o += kC * vq;
+    L.dUs = o; o += kC * vq;
+    L.Zs = o; o += kC * vq;
     L.g = o; o += kC;
     L.gam = o; o += kC;
     L.bet = o; o += kC;
@@ -534,13 +603,13 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
                        const float *__restrict__ cache, const float *__restrict__ S_chunks,
                        const float *__restrict__ dS_chunks, float *__restrict__ parts, float *__restrict__ dv_out)
 {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
     const VpartSmem Y = vpart_layout(DK, DVT);
-    float *Ks = sm + Y.Ks, *Ts = sm + Y.Ts, *Ps = sm + Y.Ps, *Ss = sm + Y.Ss, *dSs = sm + Y.dSs;
+    float *Kt = sm + Y.Kt, *Ts = sm + Y.Ts, *Ps = sm + Y.Ps, *Ss = sm + Y.Ss, *dSs = sm + Y.dSs;
     float *Vs = sm + Y.Vs, *dYs = sm + Y.dYs, *Uts = sm + Y.Uts, *dUs = sm + Y.dUs, *Zs = sm + Y.Zs;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd, *red = sm + Y.red;
-    const int kp = DK + 1, vp = DVT + 1, cp = kC + 1;
+    const int vq = ldp(DVT), cp = ldp(kC);
     const int n_vt = DV / DVT;
     const int c = blockIdx.y;
     const int chain = blockIdx.x / n_vt, vt = blockIdx.x % n_vt, v0 = vt * DVT;
@@ -552,170 +621,127 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
     const size_t cidx = (size_t)chain * max_chunks + c;
     const float *cb = cache + cidx * cache_floats(DK);
     const float *Sg = S_chunks + cidx * DK * DV + v0, *dSg = dS_chunks + cidx * DK * DV + v0;
-    for (int i = tid; i < DK * DVT; i += blockDim.x) {
-        const int a = i / DVT, b = i % DVT;
-        Ss[a * vp + b] = Sg[(size_t)a * DV + b];
-        dSs[a * vp + b] = dSg[(size_t)a * DV + b];
+    const int nvq = DVT / 4;
+#pragma unroll 4
+    for (int i = tid; i < DK * nvq; i += blockDim.x) {
+        const int a = i / nvq, b = (i % nvq) * 4;
+        st4(Ss + a * vq + b, f4(Sg + (size_t)a * DV + b));
+        st4(dSs + a * vq + b, f4(dSg + (size_t)a * DV + b));
     }
-    load_rows(Ks, kp, k, c0, n, H, h, DK, 0, DK, 1.f);
-    load_rows(Vs, vp, v, c0, n, H, h, DV, v0, DVT, 1.f);
-    load_rows(dYs, vp, dy, c0, n, H, h, DV, v0, DVT, 1.f);
-    load_block(Ts, cp, cb + kCacheT, kC, kC);
-    load_block(Ps, cp, cb + kCacheP, kC, kC);
+    load_rows_t(Kt, cp, k, c0, n, H, h, DK, DK);
+    load_rows(Vs, vq, v, c0, n, H, h, DV, v0, DVT, 1.f);
+    load_rows(dYs, vq, dy, c0, n, H, h, DV, v0, DVT, 1.f);
+    load_block(Ts, cp, cb + kCacheT, kC, kC, 1.f);
+    load_block(Ps, cp, cb + kCacheP, kC, kC, 1.f);
     if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
     __syncthreads();
     float *P = parts + (cidx * n_vt + vt) * part_floats(DK);
     float *PdP = P, *PdT = P + kC * kC, *PdW = P + 2 * kC * kC, *PdKd = PdW + kC * DK, *PdYS = PdKd + kC * DK;
     float *Pvs = PdYS + kC * DK, *PdgC = Pvs + kC;
     // Z = diag(beta) (V - diag(gamma) K S);  dU~ = P^T dY + diag(D) K dS'
-    {
-        constexpr int TM = 4, TN = 2;
-        const int ntm = kC / TM, ntn = DVT / TN;
-        for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-            const int tm = gi / ntn, tn = gi % ntn;
-            float ks[TM][TN], kd[TM][TN], pd[TM][TN];
-            zero(ks);
-            zero(kd);
-            zero(pd);
-#pragma unroll 4
-            for (int a = 0; a < DK; ++a) {
-                float av[TM], bs[TN], bd[TN];
+    // (A(t, a) = K[t][a] = Kt[a][t] and A(s, t) = P[t][s], both stored [k][m])
+    for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
+        const Tile<2, false, true> tl(gi, kC, DVT);
+        float ks[4][2], kd[4][2], pd[4][2];
+        zero(ks);
+        zero(kd);
+        zero(pd);
+        tl.run(ks, DK, Kt, cp, Ss, vq);
+        tl.run(kd, DK, Kt, cp, dSs, vq);
+        tl.run(pd, kC, Ps, cp, dYs, vq);
 #pragma unroll
-                for (int i = 0; i < TM; ++i) av[i] = Ks[(tm + i * ntm) * kp + a];
+        for (int i = 0; i < 4; ++i) {
+            const int t = tl.row(i);
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    bs[j] = Ss[a * vp + tn + j * ntn];
-                    bd[j] = dSs[a * vp + tn + j * ntn];
-                }
-#pragma unroll
-                for (int i = 0; i < TM; ++i)
-#pragma unroll
-                    for (int j = 0; j < TN; ++j) {
-                        ks[i][j] = fmaf(av[i], bs[j], ks[i][j]);
-                        kd[i][j] = fmaf(av[i], bd[j], kd[i][j]);
-                    }
-            }
-            mm_acc(pd, tm, tn, ntm, ntn, kC, [&](int s, int t) { return Ps[t * cp + s]; },
-                   [&](int t, int b) { return dYs[t * vp + b]; });
-#pragma unroll
-            for (int i = 0; i < TM; ++i) {
-                const int t = tm + i * ntm;
-#pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const int b = tn + j * ntn;
-                    Zs[t * vp + b] = bet[t] * (Vs[t * vp + b] - gam[t] * ks[i][j]);
-                    dUs[t * vp + b] = fmaf(Dd[t], kd[i][j], pd[i][j]);
-                }
+            for (int j = 0; j < 2; ++j) {
+                const int b = tl.col(j);
+                Zs[t * vq + b] = bet[t] * (Vs[t * vq + b] - gam[t] * ks[i][j]);
+                dUs[t * vq + b] = fmaf(Dd[t], kd[i][j], pd[i][j]);
             }
         }
     }
     __syncthreads();
-    // U~ = T Z;  T^T dU~ -> dV = diag(beta) T^T dU~ and the row sums of V o T^T dU~.
-    // ntm * ntn is a multiple of 32 and at most the block, so every lane of a warp that
-    // enters has a tile and the row sums can use shuffles.
-    {
-        constexpr int TM = 4, TN = 2;
-        const int ntm = kC / TM, ntn = DVT / TN;
-        if (tid < ntm * ntn) {
-            const int tm = tid / ntn, tn = tid % ntn;
-            float u[TM][TN], w[TM][TN];
-            zero(u);
-            zero(w);
-            mm_acc(u, tm, tn, ntm, ntn, kC, [&](int t, int s) { return Ts[t * cp + s]; },
-                   [&](int s, int b) { return Zs[s * vp + b]; });
-            mm_acc(w, tm, tn, ntm, ntn, kC, [&](int t, int s) { return Ts[s * cp + t]; },
-                   [&](int s, int b) { return dUs[s * vp + b]; });
+    // U~ = T Z
+    for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
+        const Tile<2, true, true> tl(gi, kC, DVT);
+        float u[4][2];
+        zero(u);
+        tl.run(u, kC, Ts, cp, Zs, vq);
 #pragma unroll
-            for (int i = 0; i < TM; ++i) {
-                const int t = tm + i * ntm;
-                float rs = 0.f;
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float2 *>(Uts + tl.row(i) * vq + 2 * tl.tn) = make_float2(u[i][0], u[i][1]);
+    }
+    // T^T dU~ (A(t, s) = T[s][t], stored [k][m]): dV = diag(beta) T^T dU~, and V o T^T dU~
+    // into Ps (P is no longer needed) for its row sums
+    for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
+        const Tile<2, false, true> tl(gi, kC, DVT);
+        float w[4][2];
+        zero(w);
+        tl.run(w, kC, Ts, cp, dUs, vq);
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const int b = tn + j * ntn;
-                    Uts[t * vp + b] = u[i][j];
-                    if (t < n) dv_out[((size_t)(c0 + t) * H + h) * DV + v0 + b] = bet[t] * w[i][j];
-                    rs = fmaf(Vs[t * vp + b], w[i][j], rs);
-                }
-                rs = row_group_sum(rs, ntn);
-                if (tn == 0) Pvs[t] = rs;
-            }
+        for (int i = 0; i < 4; ++i) {
+            const int t = tl.row(i), b = 2 * tl.tn;
+            if (t < n)
+                *reinterpret_cast<float2 *>(dv_out + ((size_t)(c0 + t) * H + h) * DV + v0 + b) =
+                    make_float2(bet[t] * w[i][0], bet[t] * w[i][1]);
+            Ps[t * cp + b] = Vs[t * vq + b] * w[i][0];
+            Ps[t * cp + b + 1] = Vs[t * vq + b + 1] * w[i][1];
         }
     }
     __syncthreads();
-    // this slice's dY U~^T and dU~ Z^T [C][C]
-    {
-        constexpr int TM = 4, TN = 2;
-        const int ntm = kC / TM, ntn = kC / TN;
-        for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-            const int tm = gi / ntn, tn = gi % ntn;
-            float p[TM][TN], tt[TM][TN];
-            zero(p);
-            zero(tt);
-            mm_acc(p, tm, tn, ntm, ntn, DVT, [&](int t, int b) { return dYs[t * vp + b]; },
-                   [&](int b, int s) { return Uts[s * vp + b]; });
-            mm_acc(tt, tm, tn, ntm, ntn, DVT, [&](int t, int b) { return dUs[t * vp + b]; },
-                   [&](int b, int s) { return Zs[s * vp + b]; });
-#pragma unroll
-            for (int i = 0; i < TM; ++i)
-#pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const int e = (tm + i * ntm) * kC + tn + j * ntn;
-                    PdP[e] = p[i][j];
-                    PdT[e] = tt[i][j];
-                }
-        }
+    // row sums of V o T^T dU~: eight lanes per row
+    for (int r = tid; r < kC * 8; r += blockDim.x) {
+        const int t = r >> 3, part = r & 7;
+        float acc = 0.f;
+        for (int b = part; b < DVT; b += 8) acc += Ps[t * cp + b];
+        acc = group_sum<8>(acc);
+        if (part == 0) Pvs[t] = acc;
     }
-    // this slice's -dU~ S^T, U~ dS'^T and dY S^T [C][DK]
-    {
-        constexpr int TM = 4, TN = 4;
-        const int ntm = kC / TM, ntn = DK / TN;
-        for (int gi = tid; gi < ntm * ntn; gi += blockDim.x) {
-            const int tm = gi / ntn, tn = gi % ntn;
-            float w[TM][TN], kd[TM][TN], ys[TM][TN];
-            zero(w);
-            zero(kd);
-            zero(ys);
-#pragma unroll 2
-            for (int b = 0; b < DVT; ++b) {
-                float au[TM], at[TM], ay[TM], bs[TN], bd[TN];
+    // this slice's dY U~^T and dU~ Z^T [C][C] (B(b, s) = U~[s][b], Z[s][b]: stored [n][k])
+    for (int gi = tid; gi < (kC / 4) * (kC / 2); gi += blockDim.x) {
+        const Tile<2, true, false> tl(gi, kC, kC);
+        float p[4][2], tt[4][2];
+        zero(p);
+        zero(tt);
+        tl.run(p, DVT, dYs, vq, Uts, vq);
+        tl.run(tt, DVT, dUs, vq, Zs, vq);
 #pragma unroll
-                for (int i = 0; i < TM; ++i) {
-                    const int t = tm + i * ntm;
-                    au[i] = dUs[t * vp + b];
-                    at[i] = Uts[t * vp + b];
-                    ay[i] = dYs[t * vp + b];
-                }
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const int a = tn + j * ntn;
-                    bs[j] = Ss[a * vp + b];
-                    bd[j] = dSs[a * vp + b];
-                }
-#pragma unroll
-                for (int i = 0; i < TM; ++i)
-#pragma unroll
-                    for (int j = 0; j < TN; ++j) {
-                        w[i][j] = fmaf(au[i], bs[j], w[i][j]);
-                        kd[i][j] = fmaf(at[i], bd[j], kd[i][j]);
-                        ys[i][j] = fmaf(ay[i], bs[j], ys[i][j]);
-                    }
+            for (int j = 0; j < 2; ++j) {
+                const int e = tl.row(i) * kC + tl.col(j);
+                PdP[e] = p[i][j];
+                PdT[e] = tt[i][j];
             }
+    }
+    // this slice's -dU~ S^T, U~ dS'^T and dY S^T [C][DK] (B(b, a) = S[a][b]: stored [n][k])
+    for (int gi = tid; gi < (kC / 4) * (DK / 4); gi += blockDim.x) {
+        const Tile<4, true, false> tl(gi, kC, DK);
+        float acc[4][4];
+        zero(acc);
+        tl.run(acc, DVT, dUs, vq, Ss, vq);
 #pragma unroll
-            for (int i = 0; i < TM; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const int e = (tm + i * ntm) * DK + tn + j * ntn;
-                    PdW[e] = -w[i][j];
-                    PdKd[e] = kd[i][j];
-                    PdYS[e] = ys[i][j];
-                }
-        }
+            for (int j = 0; j < 4; ++j) PdW[tl.row(i) * DK + tl.col(j)] = -acc[i][j];
+        zero(acc);
+        tl.run(acc, DVT, Uts, vq, dSs, vq);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) PdKd[tl.row(i) * DK + tl.col(j)] = acc[i][j];
+        zero(acc);
+        tl.run(acc, DVT, dYs, vq, Ss, vq);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) PdYS[tl.row(i) * DK + tl.col(j)] = acc[i][j];
     }
     // <dS', S> over this slice
     float sd = 0.f;
     for (int i = tid; i < DK * DVT; i += blockDim.x) {
         const int a = i / DVT, b = i % DVT;
-        sd = fmaf(dSs[a * vp + b], Ss[a * vp + b], sd);
+        sd = fmaf(dSs[a * vq + b], Ss[a * vq + b], sd);
     }
     sd = group_sum<32>(sd);
     if ((tid & 31) == 0) red[tid >> 5] = sd;
@@ -729,18 +755,20 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
 
 // --------------------------------------------------------------------------- kpart
 struct KpartSmem {
-    int Ks, Qs, PdWs, Ts, G1, Asym, dGs, Es, g, gam, bet, Dd, red, total;
+    int Ks, Qs, PdWs, Ts, G1, G1T, Asym, dGs, Es, g, gam, bet, Dd, red, total;
 };
 __host__ __device__ inline KpartSmem kpart_layout(int DK)
 {
     KpartSmem L;
     int o = 0;
-    const int kp = DK + 1, cp = kC + 1;
-    L.Ks = o; o += kC * kp;
-    L.Qs = o; o += kC * kp;
-    L.PdWs = o; o += kC * kp;
+    const int kq = ldp(DK), cp = ldp(kC);
+    L.Ks = o; o += kC * kq;
+    L.Qs = o; o += kC * kq;
+    L.PdWs = o; o += kC * kq;
+    // Ts .. Es are contiguous: after the last products they hold dQ's and dK's sums
     L.Ts = o; o += kC * cp;
     L.G1 = o; o += kC * cp;
+    L.G1T = o; o += kC * cp;
     L.Asym = o; o += kC * cp;
     L.dGs = o; o += kC * cp;
     L.Es = o; o += kC * cp;
@@ -753,22 +781,22 @@ __host__ __device__ inline KpartSmem kpart_layout(int DK)
     return L;
 }
 
-// One CTA (kThreads) per (chain, chunk): dQ, dK, dbeta and dlog_alpha of the chunk from its
-// cache block and its sums buffer (the value slices' blocks added here, in slice order).
+// One CTA (kThreadsWide) per (chain, chunk): dQ, dK, dbeta and dlog_alpha of the chunk from
+// its cache block and its sums buffer (the value slices' blocks added here, in slice order).
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreadsWide)
 chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ log_alpha,
                        const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int H, int DK,
                        int n_vt, float scale, int max_chunks, const float *__restrict__ cache,
                        const float *__restrict__ parts, float *__restrict__ dq, float *__restrict__ dk,
                        float *__restrict__ dbeta, float *__restrict__ dlog_alpha)
 {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     const KpartSmem Y = kpart_layout(DK);
     float *Ks = sm + Y.Ks, *Qs = sm + Y.Qs, *PdWs = sm + Y.PdWs, *Ts = sm + Y.Ts, *G1 = sm + Y.G1;
-    float *Asym = sm + Y.Asym, *dGs = sm + Y.dGs, *Es = sm + Y.Es, *g = sm + Y.g;
+    float *G1T = sm + Y.G1T, *Asym = sm + Y.Asym, *dGs = sm + Y.dGs, *Es = sm + Y.Es, *g = sm + Y.g;
     float *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd, *red = sm + Y.red;
-    const int kp = DK + 1, cp = kC + 1;
+    const int kq = ldp(DK), cp = ldp(kC);
     const int c = blockIdx.y, chain = blockIdx.x;
     const int seq = chain / H, h = chain % H;
     const int tid = threadIdx.x;
@@ -787,83 +815,109 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         for (int j = 0; j < n_vt; ++j) acc += P0[j * pf + off];
         return acc;
     };
+    auto sum_slices4 = [&](size_t off) -> float4 {
+        float4 acc = f4(P0 + off);
+        for (int j = 1; j < n_vt; ++j) acc = add4(acc, f4(P0 + j * pf + off));
+        return acc;
+    };
 
-    load_rows(Ks, kp, k, c0, n, H, h, DK, 0, DK, 1.f);
-    load_rows(Qs, kp, q, c0, n, H, h, DK, 0, DK, scale);
-    load_block(Ts, cp, cb + kCacheT, kC, kC);
+    load_rows(Ks, kq, k, c0, n, H, h, DK, 0, DK, 1.f);
+    load_rows(Qs, kq, q, c0, n, H, h, DK, 0, DK, scale);
+    load_block(Ts, cp, cb + kCacheT, kC, kC, 1.f);
     if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-    for (int i = tid; i < kC * DK; i += blockDim.x) PdWs[(i / DK) * kp + i % DK] = sum_slices(oW + i);
+#pragma unroll 4
+    for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
+        const int r = i / (DK / 4), a = (i % (DK / 4)) * 4;
+        st4(PdWs + r * kq + a, sum_slices4(oW + (size_t)r * DK + a));
+    }
     // dT into dGs and dP into G1, summed over the slices
-    for (int i = tid; i < kC * kC; i += blockDim.x) {
-        const int t = i / kC, s = i % kC;
-        dGs[t * cp + s] = sum_slices(oT + i);
-        G1[t * cp + s] = sum_slices(oP + i);
+#pragma unroll 4
+    for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
+        const int t = i / (kC / 4), s = (i % (kC / 4)) * 4;
+        st4(dGs + t * cp + s, sum_slices4(oT + (size_t)t * kC + s));
+        st4(G1 + t * cp + s, sum_slices4(oP + (size_t)t * kC + s));
     }
     __syncthreads();
-    constexpr int SM = 4, SN = 4;            // tiles of the C x C products
-    const int sntm = kC / SM, sntn = kC / SN;
-    // M = dT T^T (into Asym)
-    for (int gi = tid; gi < sntm * sntn; gi += blockDim.x) {
-        const int tm = gi / sntn, tn = gi % sntn;
-        float acc[SM][SN];
+    // M = dT T^T into Asym (B(r, s) = T[s][r]: stored [n][k])
+    for (int gi = tid; gi < (kC / 4) * (kC / 4); gi += blockDim.x) {
+        const Tile<4, true, false> tl(gi, kC, kC);
+        float acc[4][4];
         zero(acc);
-        mm_acc(acc, tm, tn, sntm, sntn, kC, [&](int t, int r) { return dGs[t * cp + r]; },
-               [&](int r, int s) { return Ts[s * cp + r]; });
+        tl.run(acc, kC, dGs, cp, Ts, cp);
 #pragma unroll
-        for (int i = 0; i < SM; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < SN; ++j) Asym[(tm + i * sntm) * cp + tn + j * sntn] = acc[i][j];
+            for (int j = 0; j < 4; ++j) Asym[tl.row(i) * cp + tl.col(j)] = acc[i][j];
     }
     __syncthreads();
-    // dL = strict_tril(-T^T M), into dGs
-    for (int gi = tid; gi < sntm * sntn; gi += blockDim.x) {
-        const int tm = gi / sntn, tn = gi % sntn;
-        float acc[SM][SN];
+    // dL = strict_tril(-T^T M) into dGs (A(t, r) = T[r][t]: stored [k][m])
+    for (int gi = tid; gi < (kC / 4) * (kC / 4); gi += blockDim.x) {
+        const Tile<4, false, true> tl(gi, kC, kC);
+        float acc[4][4];
         zero(acc);
-        mm_acc(acc, tm, tn, sntm, sntn, kC, [&](int t, int r) { return Ts[r * cp + t]; },
-               [&](int r, int s) { return Asym[r * cp + s]; });
+        tl.run(acc, kC, Ts, cp, Asym, cp);
 #pragma unroll
-        for (int i = 0; i < SM; ++i)
+        for (int i = 0; i < 4; ++i) {
+            const int t = tl.row(i);
 #pragma unroll
-            for (int j = 0; j < SN; ++j) {
-                const int t = tm + i * sntm, s = tn + j * sntn;
+            for (int j = 0; j < 4; ++j) {
+                const int s = tl.col(j);
                 dGs[t * cp + s] = s < t ? -acc[i][j] : 0.f;
             }
+        }
     }
     __syncthreads();
-    // dA + dA^T with dA = diag(beta) (dL o Gamma), into Asym
+    // dA + dA^T with dA = diag(beta) (dL o Gamma), into Asym (symmetric)
     for (int i = tid; i < kC * kC; i += blockDim.x) {
         const int t = i / kC, s = i % kC;
         const float da_ts = s < t ? bet[t] * dGs[t * cp + s] * expf(g[t] - g[s]) : 0.f;
         const float da_st = t < s ? bet[s] * dGs[s * cp + t] * expf(g[s] - g[t]) : 0.f;
         Asym[t * cp + s] = da_ts + da_st;
     }
-    // T^T dW, kept in registers until PdWs may be overwritten (one tile per thread)
-    constexpr int TM = 8, TN = 4;
-    const int ntm = kC / TM, ntn = DK / TN;
-    const bool has_tile = tid < ntm * ntn;
-    const int tm = tid / ntn, tn = tid % ntn;
-    float tdw[TM][TN];
-    zero(tdw);
-    if (has_tile)
-        mm_acc(tdw, tm, tn, ntm, ntn, kC, [&](int t, int s) { return Ts[s * cp + t]; },
-               [&](int s, int a) { return PdWs[s * kp + a]; });
+    // T^T dW (A(t, s) = T[s][t]), kept in registers until PdWs may be overwritten
+    constexpr int kMaxTiles = (kC / 4) * (128 / 4) / kThreadsWide;   // 1 at DK = 128
+    const int n_tiles = (kC / 4) * (DK / 4);
+    float tdw[kMaxTiles][4][4];
+#pragma unroll
+    for (int r = 0; r < kMaxTiles; ++r) {
+        zero(tdw[r]);
+        const int gi = tid + r * kThreadsWide;
+        if (gi < n_tiles) Tile<4, false, true>(gi, kC, DK).run(tdw[r], kC, Ts, cp, PdWs, kq);
+    }
     __syncthreads();
     // per entry (same thread reads and writes it): dGamma o Gamma into dGs, dL o A o Gamma into
-    // Es, dP o Gamma into G1
-    for (int i = tid; i < kC * kC; i += blockDim.x) {
-        const int t = i / kC, s = i % kC;
-        const float gts = s <= t ? expf(g[t] - g[s]) : 0.f;
-        const float dl = dGs[t * cp + s], ag = cb[kCacheAG + i], dp = G1[t * cp + s];
-        dGs[t * cp + s] = dp * cb[kCacheP + i] + bet[t] * dl * ag;
-        Es[t * cp + s] = dl * ag;
-        G1[t * cp + s] = dp * gts;
+    // Es, dP o Gamma into G1 and its transpose into G1T
+#pragma unroll 2
+    for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
+        const int t = i / (kC / 4), s0 = (i % (kC / 4)) * 4;
+        const float4 ag4 = f4(cb + kCacheAG + t * kC + s0), p4 = f4(cb + kCacheP + t * kC + s0);
+        const float4 dl4 = f4(dGs + t * cp + s0), dp4 = f4(G1 + t * cp + s0);
+        const float ag[4] = {ag4.x, ag4.y, ag4.z, ag4.w}, pp[4] = {p4.x, p4.y, p4.z, p4.w};
+        const float dl[4] = {dl4.x, dl4.y, dl4.z, dl4.w}, dp[4] = {dp4.x, dp4.y, dp4.z, dp4.w};
+        float dgm[4], e[4], g1[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = s0 + u;
+            const float gts = s <= t ? expf(g[t] - g[s]) : 0.f;
+            dgm[u] = dp[u] * pp[u] + bet[t] * dl[u] * ag[u];
+            e[u] = dl[u] * ag[u];
+            g1[u] = dp[u] * gts;
+            G1T[s * cp + t] = g1[u];
+        }
+        st4(dGs + t * cp + s0, make_float4(dgm[0], dgm[1], dgm[2], dgm[3]));
+        st4(Es + t * cp + s0, make_float4(e[0], e[1], e[2], e[3]));
+        st4(G1 + t * cp + s0, make_float4(g1[0], g1[1], g1[2], g1[3]));
     }
-    if (has_tile)
 #pragma unroll
-        for (int i = 0; i < TM; ++i)
+    for (int r = 0; r < kMaxTiles; ++r) {
+        const int gi = tid + r * kThreadsWide;
+        if (gi < n_tiles) {
+            const Tile<4, false, true> tl(gi, kC, DK);
 #pragma unroll
-            for (int j = 0; j < TN; ++j) PdWs[(tm + i * ntm) * kp + tn + j * ntn] = tdw[i][j];
+            for (int i = 0; i < 4; ++i)
+                st4(PdWs + tl.row(i) * kq + 4 * tl.tn, make_float4(tdw[r][i][0], tdw[r][i][1], tdw[r][i][2], tdw[r][i][3]));
+        }
+    }
     __syncthreads();
     if (tid < kC) {
         float rs = 0.f, cs = 0.f, ab = 0.f;
@@ -875,63 +929,70 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         red[tid] = rs - cs;          // row sum - column sum of dGamma o Gamma
         red[kC + tid] = ab;          // row sum of dL o A o Gamma
     }
-    // dQ = diag(gamma) dY S^T + (dP o Gamma) K;
-    // dK = (dP o Gamma)^T Q + (dA + dA^T) K + diag(beta gamma) T^T dW + diag(D) dK~.
-    // ntm * ntn = 2 DK is a multiple of 32 and at most the block: shuffles are safe.
-    if (has_tile) {
-        float aq[TM][TN], ak[TM][TN];
-        zero(aq);
-        zero(ak);
-#pragma unroll 2
-        for (int s = 0; s < kC; ++s) {
-            float g1[TM], g1t[TM], as[TM], bk[TN], bq[TN];
+    // (dP o Gamma) K and (dP o Gamma)^T Q + (dA + dA^T) K, in registers until the region
+    // Ts .. Es is free (A(t, s) = G1[t][s] = G1T[s][t], G1[s][t] and Asym[s][t]: all [k][m])
+    float aq[kMaxTiles][4][4], ak[kMaxTiles][4][4];
 #pragma unroll
-            for (int i = 0; i < TM; ++i) {
-                const int t = tm + i * ntm;
-                g1[i] = G1[t * cp + s];
-                g1t[i] = G1[s * cp + t];
-                as[i] = Asym[t * cp + s];
-            }
-#pragma unroll
-            for (int j = 0; j < TN; ++j) {
-                bk[j] = Ks[s * kp + tn + j * ntn];
-                bq[j] = Qs[s * kp + tn + j * ntn];
-            }
-#pragma unroll
-            for (int i = 0; i < TM; ++i)
-#pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    aq[i][j] = fmaf(g1[i], bk[j], aq[i][j]);
-                    ak[i][j] = fmaf(g1t[i], bq[j], fmaf(as[i], bk[j], ak[i][j]));
-                }
+    for (int r = 0; r < kMaxTiles; ++r) {
+        zero(aq[r]);
+        zero(ak[r]);
+        const int gi = tid + r * kThreadsWide;
+        if (gi < n_tiles) {
+            const Tile<4, false, true> tl(gi, kC, DK);
+            tl.run(aq[r], kC, G1T, cp, Ks, kq);
+            tl.run(ak[r], kC, G1, cp, Qs, kq);
+            tl.run(ak[r], kC, Asym, cp, Ks, kq);
         }
+    }
+    __syncthreads();
+    float *GQ = Ts, *GK = Ts + kC * kq;
 #pragma unroll
-        for (int i = 0; i < TM; ++i) {
-            const int t = tm + i * ntm;
-            float rg = 0.f, rb = 0.f, rd = 0.f;
+    for (int r = 0; r < kMaxTiles; ++r) {
+        const int gi = tid + r * kThreadsWide;
+        if (gi < n_tiles) {
+            const Tile<4, false, true> tl(gi, kC, DK);
 #pragma unroll
-            for (int j = 0; j < TN; ++j) {
-                const int a = tn + j * ntn;
-                const size_t ta = (size_t)t * DK + a;
-                const float pys = sum_slices(oYS + ta), pkd = sum_slices(oKd + ta);
-                const float tw = PdWs[t * kp + a];
-                const float kta = Ks[t * kp + a];
-                rg = fmaf(Qs[t * kp + a], pys, rg);
-                rb = fmaf(kta, tw, rb);
-                rd = fmaf(kta, pkd, rd);
-                if (t < n) {
-                    dq[((size_t)(c0 + t) * H + h) * DK + a] = scale * (gam[t] * pys + aq[i][j]);
-                    dk[((size_t)(c0 + t) * H + h) * DK + a] = ak[i][j] + bet[t] * gam[t] * tw + Dd[t] * pkd;
-                }
+            for (int i = 0; i < 4; ++i) {
+                const int o = tl.row(i) * kq + 4 * tl.tn;
+                st4(GQ + o, make_float4(aq[r][i][0], aq[r][i][1], aq[r][i][2], aq[r][i][3]));
+                st4(GK + o, make_float4(ak[r][i][0], ak[r][i][1], ak[r][i][2], ak[r][i][3]));
             }
-            rg = row_group_sum(rg, ntn);
-            rb = row_group_sum(rb, ntn);
-            rd = row_group_sum(rd, ntn);
-            if (tn == 0) {
-                red[2 * kC + t] = rg + bet[t] * rb;     // dgamma_t
-                red[3 * kC + t] = rb;                   // sum_a K o T^T dW
-                red[4 * kC + t] = rd;                   // dD_t
+        }
+    }
+    __syncthreads();
+    // dQ = diag(gamma) dY S^T + (dP o Gamma) K;
+    // dK = (dP o Gamma)^T Q + (dA + dA^T) K + diag(beta gamma) T^T dW + diag(D) dK~;
+    // a warp per row t, four consecutive a per lane, with the row sums for dbeta and
+    // dlog_alpha; two rows at a time so that their loads are in flight together
+    const int warp = tid >> 5, lane = tid & 31, n_warps = blockDim.x >> 5;
+#pragma unroll 2
+    for (int t = warp; t < kC; t += n_warps) {
+        float rg = 0.f, rb = 0.f, rd = 0.f;
+        for (int a = 4 * lane; a < DK; a += 128) {
+            const size_t ta = (size_t)t * DK + a;
+            const float4 pys = sum_slices4(oYS + ta), pkd = sum_slices4(oKd + ta);
+            const float4 tw = f4(PdWs + t * kq + a), kt = f4(Ks + t * kq + a), qt = f4(Qs + t * kq + a);
+            const float4 gq = f4(GQ + t * kq + a), gk = f4(GK + t * kq + a);
+            rg += qt.x * pys.x + qt.y * pys.y + qt.z * pys.z + qt.w * pys.w;
+            rb += kt.x * tw.x + kt.y * tw.y + kt.z * tw.z + kt.w * tw.w;
+            rd += kt.x * pkd.x + kt.y * pkd.y + kt.z * pkd.z + kt.w * pkd.w;
+            if (t < n) {
+                const float gt = gam[t], bg = bet[t] * gam[t], dt = Dd[t];
+                st4(dq + ((size_t)(c0 + t) * H + h) * DK + a,
+                    make_float4(scale * (gt * pys.x + gq.x), scale * (gt * pys.y + gq.y),
+                                scale * (gt * pys.z + gq.z), scale * (gt * pys.w + gq.w)));
+                st4(dk + ((size_t)(c0 + t) * H + h) * DK + a,
+                    make_float4(gk.x + bg * tw.x + dt * pkd.x, gk.y + bg * tw.y + dt * pkd.y,
+                                gk.z + bg * tw.z + dt * pkd.z, gk.w + bg * tw.w + dt * pkd.w));
             }
+        }
+        rg = group_sum<32>(rg);
+        rb = group_sum<32>(rb);
+        rd = group_sum<32>(rd);
+        if (lane == 0) {
+            red[2 * kC + t] = rg + bet[t] * rb;     // dgamma_t
+            red[3 * kC + t] = rb;                   // sum_a K o T^T dW
+            red[4 * kC + t] = rd;                   // dD_t
         }
     }
     __syncthreads();

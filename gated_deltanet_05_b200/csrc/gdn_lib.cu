@@ -436,6 +436,9 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
     const size_t need = gdn_backward_workspace_bytes(cu_seqlens_host, n_seq, H, d_k, d_v);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return GDN_ERR_INVALID_ARG;
     if (!aligned(S0, 4) || !aligned(dS_T, 4) || !aligned(dS0, 4)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dy, 16) || !aligned(dq, 16) ||
+        !aligned(dk, 16) || !aligned(dv, 16))
+        return GDN_ERR_INVALID_ARG;
     int64_t max_len = 0;
     for (int i = 0; i < n_seq; ++i)
         if ((int64_t)cu_seqlens_host[i + 1] - cu_seqlens_host[i] > max_len)
@@ -496,7 +499,7 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
         kv<<<grid_v, kThreadsWide, smem_v, st>>>((const T *)k, (const T *)v, (const T *)dy, log_alpha, beta,     \
                                                  cu_seqlens_dev, H, d_k, d_v, (int)max_chunks, cache, S_chunks, \
                                                  dS_chunks, parts, dv);                             \
-        kk<<<grid_c, kThreads, smem_k, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
+        kk<<<grid_c, kThreadsWide, smem_k, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
                                              n_vt, scale, (int)max_chunks, cache, parts, dq, dk, dbeta,  \
                                              dlog_alpha);                                           \
     }

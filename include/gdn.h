@@ -187,12 +187,14 @@ gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_
  *          gdn_chunk_fwd (S0 may be NULL: zeros)
  *   dy     [n_tok, H, d_v] in in_dtype;  dS_T [n_seq, H, d_v, d_k] fp32 or NULL (zero)
  *   dq, dk [n_tok, H, d_k], dv [n_tok, H, d_v], dlog_alpha, dbeta [n_tok, H] fp32 out
+ *          (dy, dq, dk, dv 16-byte aligned, like q, k, v)
  *   dS0    [n_seq, H, d_v, d_k] fp32 out, or NULL
  *   workspace: gdn_backward_workspace_bytes(...) bytes, 16-byte aligned: per (chain, chunk
  *          of 64 tokens) the chunk's start state and the adjoint of its end state
  *          (d_k x d_v each), the chunk's cache of state-free matrices (3 x 64 x 64 + 64 x d_k
  *          floats: T, A o Gamma, P, W) and, per slice of min(d_v, 64) value columns, one
- *          block of the chunk's sums over v (2 x 64 x 64 + 3 x 64 x d_k + 64 + 1 floats);
+ *          block of the chunk's sums over v (2 x 64 x 64 + 3 x 64 x d_k + 64 + 1 floats,
+ *          rounded up to a multiple of 4);
  *          n_seq * H * ceil(max_len / 64) chunks are provided for
  *   d_k, d_v in {16, 32, 64, 128}
  * The chain rule through the chunked form, fp32 on CUDA cores, five launches: the

@@ -128,7 +128,7 @@ def test_backward_rejects_bad_arguments(L):
     # per (chain, 64-token chunk): two 128 x 128 states, the chunk's cache (3 x 64 x 64 +
     # 64 x 128 floats), and two 64-column value slices' blocks of per-chunk sums
     # (2 x 64 x 64 + 3 x 64 x 128 + 64 + 1 floats each)
-    part = 64 * (2 * 64 + 3 * 128 + 1) + 1
+    part = (64 * (2 * 64 + 3 * 128 + 1) + 1 + 3) // 4 * 4      # rounded up to a multiple of 4
     assert L.gdn_backward_workspace_bytes(ctypes.cast(cu, ctypes.c_void_p), 2, 2, 128, 128) == \
         2 * 2 * 1 * (2 * 128 * 128 + 64 * (3 * 64 + 128) + 2 * part) * 4
     assert L.gdn_backward_workspace_bytes(None, 2, 2, 128, 128) == 0
@@ -146,6 +146,7 @@ def test_backward_rejects_bad_arguments(L):
     assert bw(cu=None) == 1
     assert bw(cu=(ctypes.c_int32 * 3)(0, 64, 10)) == 1
     assert bw(dy=None) == 1
+    assert bw(dy=ctypes.c_void_p(0x10008)) == 1     # dy must be 16-byte aligned
     assert bw(wsb=1000) == 1
     assert bw(ws=None) == 1
     assert bw(n_seq=0) == 0

@@ -68,3 +68,31 @@ def test_backward_matches_oracle(lens, H, dk, dv, dtype, with_state):
             r = oracle.state_to_lib(r)
         err = rel_err(f64(g), r)
         assert err <= 1e-4, f"{name}: {err:.3e}"
+
+
+def test_backward_full_size_sampled_chains():
+    """The prefill workload's shape (4 x 4096 tokens, H = 16, d = 128, bf16), as `bench.py`
+    times it: every gradient finite, and the gradients of sampled (sequence, head) chains
+    against the oracle run on those chains alone (a chain's gradients depend on its own
+    inputs only)."""
+    import workloads as W
+    inp = W.make_prefill_inputs(W.WORKLOADS["prefill"])
+    d = {k: inp[k].cuda() for k in ("q", "k", "v", "log_alpha", "beta", "cu_seqlens", "z")}
+    got = gdn.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["cu_seqlens"], d["z"],
+                       cu_seqlens_host=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    got = [g.cpu() for g in got]
+    for g in got:
+        assert torch.isfinite(g).all()
+    cu = inp["cu_seqlens"].tolist()
+    for s, h in ((0, 0), (2, 9), (3, 15)):
+        a, b = cu[s], cu[s + 1]
+        one = lambda t: t[a:b, h:h + 1].contiguous()
+        ref = oracle.backward(one(inp["q"]), one(inp["k"]), one(inp["v"]), one(inp["log_alpha"]),
+                              one(inp["beta"]), np.array([0, b - a]), one(inp["z"]))
+        names = ("dq", "dk", "dv", "dlog_alpha", "dbeta")
+        for name, g, r in zip(names, got[:5], ref[:5]):
+            err = rel_err(f64(g[a:b, h:h + 1]), r)
+            assert err <= 1e-4, f"chain ({s}, {h}) {name}: {err:.3e}"
+        err = rel_err(f64(got[5][s:s + 1, h:h + 1]), oracle.state_to_lib(ref[5]))
+        assert err <= 1e-4, f"chain ({s}, {h}) dS0: {err:.3e}"
