@@ -32,12 +32,13 @@
 //                           sums over v that the rest needs (dP, dT, dW, dK~, dY S^T, ...), each
 //                           slice into its own block (no atomics: the result is deterministic)
 //   chunk_bwd_kpart_kernel  per (chain, chunk), all at once: dQ, dK, dbeta, dlog_alpha
-// Every matrix product runs from shared memory: a thread owns a 4 x 4 (or 4 x 2) tile of the
-// result and loads both operands as float4 along their contiguous dimension, four k-steps at
-// a time (8 vector loads per 64 FMAs); rows are padded to a multiple of 4 plus 4 floats so
-// that the lanes of a warp read distinct banks.
+// Every matrix product runs from shared memory on the tensor cores (mma.sync m16n8k8, tf32)
+// with each operand split into two tf32 parts, which keeps fp32 accuracy; a warp owns a
+// 16 x 16 block of the result. Rows in shared memory are padded to a multiple of 4 plus 4
+// floats (16-byte aligned rows; distinct banks for the fragment loads).
 #pragma once
 #include "gdn_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gdn {
 namespace bwdc {
@@ -48,8 +49,8 @@ constexpr int kThreads = 256;        // prep
 constexpr int kThreadsWide = 512;    // fwd, state, vpart and kpart
 
 __host__ __device__ inline int slice_cols(int DV) { return DV < kDVT ? DV : kDVT; }
-// shared-memory row stride for rows of D floats (D a multiple of 8): 16-byte aligned rows
-// whose float4 slots fall on distinct banks for 8 consecutive rows
+// shared-memory row stride for rows of D floats (D a multiple of 16): 16-byte aligned rows,
+// and rows g = 0..7 of a fragment load start on distinct banks
 __host__ __device__ inline int ldp(int D) { return D + 4; }
 // floats of the per-chunk sums block of one value slice: dP, dT [C][C]; dW, dK~, dY S^T
 // [C][DK]; the row sums of V o T^T dU~ [C]; <dS', S> [1]; rounded up to a multiple of 4
@@ -90,6 +91,7 @@ __device__ __forceinline__ void chunk_decays(const float *__restrict__ log_alpha
 
 __device__ __forceinline__ float4 f4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ void st4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void st2(float *p, float a, float b) { *reinterpret_cast<float2 *>(p) = make_float2(a, b); }
 __device__ __forceinline__ float4 scale4(float4 v, float f) { return make_float4(v.x * f, v.y * f, v.z * f, v.w * f); }
 __device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
 
@@ -109,7 +111,9 @@ __device__ __forceinline__ void load_rows(float *dst, int ld, const T *__restric
     }
 }
 
-// The same rows stored transposed: dst[a][t] = src[t][a], [ncol][ld].
+// The first ncol columns of the same rows stored transposed, dst[a][t] = src[t][a] ([ncol][ld]).
+// A warp covers 8 rows x 16 columns, so its global loads fill whole sectors and its
+// shared-memory stores meet at most two to a bank.
 template <typename T>
 __device__ __forceinline__ void load_rows_t(float *dst, int ld, const T *__restrict__ src, int64_t c0, int n, int H,
                                             int h, int D, int ncol)
@@ -117,7 +121,7 @@ __device__ __forceinline__ void load_rows_t(float *dst, int ld, const T *__restr
     const int nq = ncol >> 2;
 #pragma unroll 4
     for (int i = threadIdx.x; i < kC * nq; i += blockDim.x) {
-        const int t = i / nq, a = (i % nq) * 4;
+        const int rest = i >> 3, a = (rest % nq) * 4, t = (rest / nq) * 8 + (i & 7);
         const float4 x = t < n ? load4(src + ((size_t)(c0 + t) * H + h) * D + a) : make_float4(0.f, 0.f, 0.f, 0.f);
         dst[(a + 0) * ld + t] = x.x;
         dst[(a + 1) * ld + t] = x.y;
@@ -139,87 +143,96 @@ __device__ __forceinline__ void load_block(float *dst, int ld, const float *__re
     }
 }
 
-// ---- register-tiled products from shared memory ------------------------------------------
-// C[M][N] += A[M][K] B[K][N]. A thread owns 4 rows x TN columns (TN = 4 or 2). A is stored
-// either [m][k] (AMK: rows interleave across threads, m_i = tm + i ntm, each row read as
-// float4 along k) or [k][m] (rows contiguous, m_i = 4 tm + i, read as float4 along m); B is
-// stored [k][n] (BKN: columns contiguous, n_j = TN tn + j) or [n][k] (columns interleave,
-// n_j = tn + j ntn, each read as float4 along k). Within a warp 8 row groups x 4 column
-// groups where the sizes allow, so each vector load covers at most 128 distinct bytes.
-// M, N, K multiples of 16 (K of 4); strides ldp(...); bases 16-byte aligned.
-template <int TN, bool AMK, bool BKN>
-struct Tile {
-    int tm, tn, ntm, ntn;
-    __device__ __forceinline__ Tile(int gi, int M, int N)
+// ---- tensor-core products from shared memory --------------------------------------------
+// C[M][N] += A[M][K] B[K][N] on mma.sync m16n8k8 tiles in tf32. Each operand is split as
+// x = hi + lo with hi = tf32(x) and lo = tf32(x - hi), and A B is taken as
+// lo_A hi_B + hi_A lo_B + hi_A hi_B: the dropped lo_A lo_B and the rounding of lo leave an
+// error of order 2^-21 |A| |B|, that of an fp32 product; accumulation is fp32.
+// A(m, k) = AMK ? A[m lda + k] : A[k lda + m];  B(k, n) = BKN ? B[k ldb + n] : B[n ldb + k].
+// A warp owns the 16 x 16 block `tile` of C (tiles numbered row-major over N / 16 columns):
+// with g = lane / 4, q = lane % 4, its elements (f, e) (fragment f = 0, 1; e = 0..3) sit at
+// row m0 + g + 8 (e / 2), column n0 + 8 f + 2 q + e % 2. M, N multiples of 16, K of 8.
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+{
+    hi = sm100::to_tf32(x);
+    lo = sm100::to_tf32(x - __uint_as_float(hi));
+}
+
+__device__ __forceinline__ void mma8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <bool AMK, bool BKN>
+struct WTile {
+    int m0, n0, g, q;
+    float c[2][4];
+    __device__ __forceinline__ WTile(int tile, int N)
     {
-        ntm = M >> 2;
-        ntn = N / TN;
-        if ((ntm & 7) == 0 && (ntn & 3) == 0) {
-            const int lane = gi & 31, w = gi >> 5, wm = ntm >> 3;
-            tm = (w % wm) * 8 + (lane & 7);
-            tn = (w / wm) * 4 + (lane >> 3);
-        } else {
-            tm = gi % ntm;
-            tn = gi / ntm;
-        }
+        const int lane = threadIdx.x & 31, ntn = N >> 4;
+        m0 = (tile / ntn) << 4;
+        n0 = (tile % ntn) << 4;
+        g = lane >> 2;
+        q = lane & 3;
+#pragma unroll
+        for (int f = 0; f < 2; ++f)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[f][e] = 0.f;
     }
-    __device__ __forceinline__ int row(int i) const { return AMK ? tm + i * ntm : 4 * tm + i; }
-    __device__ __forceinline__ int col(int j) const { return BKN ? TN * tn + j : tn + j * ntn; }
-    __device__ __forceinline__ void run(float (&acc)[4][TN], int K, const float *__restrict__ A, int lda,
-                                        const float *__restrict__ B, int ldb) const
+    __device__ __forceinline__ int row(int h) const { return m0 + g + 8 * h; }          // h = e / 2
+    __device__ __forceinline__ int col(int f) const { return n0 + 8 * f + 2 * q; }      // e % 2 = 0
+    // fn(row, col, C[row][col], C[row][col + 1]) for the four pairs of this lane
+    template <class F>
+    __device__ __forceinline__ void each(F fn) const
+    {
+#pragma unroll
+        for (int f = 0; f < 2; ++f)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) fn(row(h), col(f), c[f][2 * h], c[f][2 * h + 1]);
+    }
+    // C[row][col], C[row][col + 1] = fn(row, col) (a float2)
+    template <class F>
+    __device__ __forceinline__ void init(F fn)
+    {
+#pragma unroll
+        for (int f = 0; f < 2; ++f)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 v = fn(row(h), col(f));
+                c[f][2 * h] = v.x;
+                c[f][2 * h + 1] = v.y;
+            }
+    }
+    __device__ __forceinline__ void run(int K, const float *__restrict__ A, int lda, const float *__restrict__ B,
+                                        int ldb)
     {
 #pragma unroll 2
-        for (int k = 0; k < K; k += 4) {
-            float a[4][4], b[4][TN];             // a[i][kk], b[kk][j]
-            if (AMK) {
+        for (int k = 0; k < K; k += 8) {
+            uint32_t ah[4], al[4], bh[2][2], bl[2][2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 v = f4(A + row(i) * lda + k);
-                    a[i][0] = v.x; a[i][1] = v.y; a[i][2] = v.z; a[i][3] = v.w;
-                }
-            } else {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const float4 v = f4(A + (k + kk) * lda + 4 * tm);
-                    a[0][kk] = v.x; a[1][kk] = v.y; a[2][kk] = v.z; a[3][kk] = v.w;
-                }
-            }
-            if (BKN) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    if constexpr (TN == 4) {
-                        const float4 v = f4(B + (k + kk) * ldb + 4 * tn);
-                        b[kk][0] = v.x; b[kk][1] = v.y; b[kk][2] = v.z; b[kk][3] = v.w;
-                    } else {
-                        const float2 v = *reinterpret_cast<const float2 *>(B + (k + kk) * ldb + 2 * tn);
-                        b[kk][0] = v.x; b[kk][1] = v.y;
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const float4 v = f4(B + col(j) * ldb + k);
-                    b[0][j] = v.x; b[1][j] = v.y; b[2][j] = v.z; b[3][j] = v.w;
-                }
+            for (int e = 0; e < 4; ++e) {
+                const int m = m0 + g + 8 * (e & 1), kk = k + q + 4 * (e >> 1);
+                split_tf32(AMK ? A[m * lda + kk] : A[kk * lda + m], ah[e], al[e]);
             }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
+            for (int f = 0; f < 2; ++f)
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                for (int e = 0; e < 2; ++e) {
+                    const int kk = k + q + 4 * e, nn = n0 + 8 * f + g;
+                    split_tf32(BKN ? B[kk * ldb + nn] : B[nn * ldb + kk], bh[f][e], bl[f][e]);
+                }
 #pragma unroll
-                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i][kk], b[kk][j], acc[i][j]);
+            for (int f = 0; f < 2; ++f) {
+                mma8(c[f], al, bh[f][0], bh[f][1]);
+                mma8(c[f], ah, bl[f][0], bl[f][1]);
+                mma8(c[f], ah, bh[f][0], bh[f][1]);
+            }
         }
     }
 };
-
-template <int TN>
-__device__ __forceinline__ void zero(float (&acc)[4][TN])
-{
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
-}
 
 // Chunk geometry of (sequence seq, chunk c): first token and valid rows; false past the end.
 __device__ __forceinline__ bool chunk_of(const int32_t *__restrict__ cu_seqlens, int seq, int c, int64_t &c0, int &n)
@@ -266,7 +279,7 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
     const int kq = ldp(DK), cp = ldp(kC);
     const int c = blockIdx.y, chain = blockIdx.x;
     const int seq = chain / H, h = chain % H;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, n_warps = blockDim.x >> 5;
     int64_t c0;
     int n;
     if (!chunk_of(cu_seqlens, seq, c, c0, n)) return;
@@ -277,26 +290,21 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
     for (int i = tid; i < kC * kC; i += blockDim.x) Ts[(i / kC) * cp + i % kC] = (i / kC == i % kC) ? 1.f : 0.f;
     __syncthreads();
     // [K; Q] K^T: A = KQ [m][a], B(a, s) = K[s][a] stored [n][k]
-    for (int gi = tid; gi < (2 * kC / 4) * (kC / 4); gi += blockDim.x) {
-        const Tile<4, true, false> tl(gi, 2 * kC, kC);
-        float acc[4][4];
-        zero(acc);
-        tl.run(acc, DK, KQ, kq, KQ, kq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int m = tl.row(i), t = m & (kC - 1);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int s = tl.col(j);
-                const float x = s <= t ? acc[i][j] * expf(g[t] - g[s]) : 0.f;
-                if (m < kC) {
-                    cb[kCacheAG + t * kC + s] = x;
-                    Ls[t * cp + s] = s < t ? bet[t] * x : 0.f;
-                } else {
-                    cb[kCacheP + t * kC + s] = x;
-                }
+    for (int tile = warp; tile < (2 * kC / 16) * (kC / 16); tile += n_warps) {
+        WTile<true, false> w(tile, kC);
+        w.run(DK, KQ, kq, KQ, kq);
+        w.each([&](int m, int s, float v0, float v1) {
+            const int t = m & (kC - 1);
+            const float x0 = s <= t ? v0 * expf(g[t] - g[s]) : 0.f;
+            const float x1 = s + 1 <= t ? v1 * expf(g[t] - g[s + 1]) : 0.f;
+            if (m < kC) {
+                st2(cb + kCacheAG + t * kC + s, x0, x1);
+                Ls[t * cp + s] = s < t ? bet[t] * x0 : 0.f;
+                Ls[t * cp + s + 1] = s + 1 < t ? bet[t] * x1 : 0.f;
+            } else {
+                st2(cb + kCacheP + t * kC + s, x0, x1);
             }
-        }
+        });
     }
     __syncthreads();
     // T[t][j] = -sum_{j <= s < t} L[t][s] T[s][j] for j < t, one row after the other
@@ -322,14 +330,10 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
     }
     __syncthreads();
     // W = T (diag(beta gamma) K): A = T [t][s], B = K scaled [s][a]
-    for (int gi = tid; gi < (kC / 4) * (DK / 4); gi += blockDim.x) {
-        const Tile<4, true, true> tl(gi, kC, DK);
-        float acc[4][4];
-        zero(acc);
-        tl.run(acc, kC, Ts, cp, KQ, kq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            st4(cb + kCacheW + tl.row(i) * DK + 4 * tl.tn, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
+    for (int tile = warp; tile < (kC / 16) * (DK / 16); tile += n_warps) {
+        WTile<true, true> w(tile, DK);
+        w.run(kC, Ts, cp, KQ, kq);
+        w.each([&](int t, int a, float v0, float v1) { st2(cb + kCacheW + t * DK + a, v0, v1); });
     }
 }
 
@@ -375,7 +379,7 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
     const int n_vt = DV / DVT;
     const int chain = blockIdx.x / n_vt, v0 = (blockIdx.x % n_vt) * DVT;
     const int seq = chain / H, h = chain % H;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, n_warps = blockDim.x >> 5;
     const int64_t len = (int64_t)cu_seqlens[seq + 1] - cu_seqlens[seq];
     const size_t st_off = (size_t)chain * DV * DK;
     for (int i = tid; i < DK * DVT; i += blockDim.x) {
@@ -413,32 +417,24 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
         }
         __syncthreads();
         // U~ = T diag(beta) V - W S
-        for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
-            const Tile<2, true, true> tl(gi, kC, DVT);
-            float acc[4][2];
-            zero(acc);
-            tl.run(acc, kC, Ts, cp, Vb, vq);
-            tl.run(acc, DK, Wn, kq, Ss, vq);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<float2 *>(Us + tl.row(i) * vq + 2 * tl.tn) = make_float2(acc[i][0], acc[i][1]);
+        for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
+            WTile<true, true> w(tile, DVT);
+            w.run(kC, Ts, cp, Vb, vq);
+            w.run(DK, Wn, kq, Ss, vq);
+            w.each([&](int t, int b, float v0_, float v1_) { st2(Us + t * vq + b, v0_, v1_); });
         }
         __syncthreads();
-        // S <- gamma_C S + (diag(D) K)^T U~: A(a, s) = Kd[s][a] stored [k][m]; each thread reads
+        // S <- gamma_C S + (diag(D) K)^T U~: A(a, s) = Kd[s][a] stored [k][m]; each warp reads
         // and writes only its own entries of S
         const float gamC = gam[kC - 1];
-        for (int gi = tid; gi < (DK / 4) * (DVT / 4); gi += blockDim.x) {
-            const Tile<4, false, true> tl(gi, DK, DVT);
-            float acc[4][4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 x = f4(Ss + tl.row(i) * vq + 4 * tl.tn);
-                acc[i][0] = gamC * x.x; acc[i][1] = gamC * x.y; acc[i][2] = gamC * x.z; acc[i][3] = gamC * x.w;
-            }
-            tl.run(acc, kC, Kd, kq, Us, vq);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                st4(Ss + tl.row(i) * vq + 4 * tl.tn, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
+        for (int tile = warp; tile < (DK / 16) * (DVT / 16); tile += n_warps) {
+            WTile<false, true> w(tile, DVT);
+            w.init([&](int a, int b) {
+                const float2 x = *reinterpret_cast<const float2 *>(Ss + a * vq + b);
+                return make_float2(gamC * x.x, gamC * x.y);
+            });
+            w.run(kC, Kd, kq, Us, vq);
+            w.each([&](int a, int b, float v0_, float v1_) { st2(Ss + a * vq + b, v0_, v1_); });
         }
     }
 }
@@ -488,7 +484,7 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     const int n_vt = DV / DVT;
     const int chain = blockIdx.x / n_vt, v0 = (blockIdx.x % n_vt) * DVT;
     const int seq = chain / H, h = chain % H;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, n_warps = blockDim.x >> 5;
     const int64_t len = (int64_t)cu_seqlens[seq + 1] - cu_seqlens[seq];
     const size_t st_off = (size_t)chain * DV * DK;
     for (int i = tid; i < DK * DVT; i += blockDim.x) {
@@ -528,32 +524,24 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         }
         __syncthreads();
         // dU~ = P^T dY + diag(D) K dS': A(s, t) = P[t][s] and A(s, a) = Kd^T[a][s], both [k][m]
-        for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
-            const Tile<2, false, true> tl(gi, kC, DVT);
-            float acc[4][2];
-            zero(acc);
-            tl.run(acc, kC, Ps, cp, dYs, vq);
-            tl.run(acc, DK, Kt, cp, dSs, vq);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<float2 *>(dUs + tl.row(i) * vq + 2 * tl.tn) = make_float2(acc[i][0], acc[i][1]);
+        for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
+            WTile<false, true> w(tile, DVT);
+            w.run(kC, Ps, cp, dYs, vq);
+            w.run(DK, Kt, cp, dSs, vq);
+            w.each([&](int s, int b, float v0_, float v1_) { st2(dUs + s * vq + b, v0_, v1_); });
         }
         __syncthreads();
-        // dS = gamma_C dS' + (diag(gamma) Q)^T dY - W^T dU~ (own entries of dS only)
+        // dS = gamma_C dS' + (diag(gamma) Q)^T dY - W^T dU~ (each warp: its own entries of dS)
         const float gamC = gam[kC - 1];
-        for (int gi = tid; gi < (DK / 4) * (DVT / 4); gi += blockDim.x) {
-            const Tile<4, false, true> tl(gi, DK, DVT);
-            float acc[4][4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 x = f4(dSs + tl.row(i) * vq + 4 * tl.tn);
-                acc[i][0] = gamC * x.x; acc[i][1] = gamC * x.y; acc[i][2] = gamC * x.z; acc[i][3] = gamC * x.w;
-            }
-            tl.run(acc, kC, Qg, kq, dYs, vq);
-            tl.run(acc, kC, Wn, kq, dUs, vq);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                st4(dSs + tl.row(i) * vq + 4 * tl.tn, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
+        for (int tile = warp; tile < (DK / 16) * (DVT / 16); tile += n_warps) {
+            WTile<false, true> w(tile, DVT);
+            w.init([&](int a, int b) {
+                const float2 x = *reinterpret_cast<const float2 *>(dSs + a * vq + b);
+                return make_float2(gamC * x.x, gamC * x.y);
+            });
+            w.run(kC, Qg, kq, dYs, vq);
+            w.run(kC, Wn, kq, dUs, vq);
+            w.each([&](int a, int b, float v0_, float v1_) { st2(dSs + a * vq + b, v0_, v1_); });
         }
     }
     __syncthreads();
@@ -614,7 +602,7 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
     const int c = blockIdx.y;
     const int chain = blockIdx.x / n_vt, vt = blockIdx.x % n_vt, v0 = vt * DVT;
     const int seq = chain / H, h = chain % H;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, n_warps = blockDim.x >> 5;
     int64_t c0;
     int n;
     if (!chunk_of(cu_seqlens, seq, c, c0, n)) return;
@@ -638,55 +626,40 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
     float *P = parts + (cidx * n_vt + vt) * part_floats(DK);
     float *PdP = P, *PdT = P + kC * kC, *PdW = P + 2 * kC * kC, *PdKd = PdW + kC * DK, *PdYS = PdKd + kC * DK;
     float *Pvs = PdYS + kC * DK, *PdgC = Pvs + kC;
+    const int n_tv = (kC / 16) * (DVT / 16);
     // Z = diag(beta) (V - diag(gamma) K S);  dU~ = P^T dY + diag(D) K dS'
     // (A(t, a) = K[t][a] = Kt[a][t] and A(s, t) = P[t][s], both stored [k][m])
-    for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
-        const Tile<2, false, true> tl(gi, kC, DVT);
-        float ks[4][2], kd[4][2], pd[4][2];
-        zero(ks);
-        zero(kd);
-        zero(pd);
-        tl.run(ks, DK, Kt, cp, Ss, vq);
-        tl.run(kd, DK, Kt, cp, dSs, vq);
-        tl.run(pd, kC, Ps, cp, dYs, vq);
+    for (int tile = warp; tile < n_tv; tile += n_warps) {
+        WTile<false, true> ks(tile, DVT), kd(tile, DVT), pd(tile, DVT);
+        ks.run(DK, Kt, cp, Ss, vq);
+        kd.run(DK, Kt, cp, dSs, vq);
+        pd.run(kC, Ps, cp, dYs, vq);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = tl.row(i);
+        for (int f = 0; f < 2; ++f)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int b = tl.col(j);
-                Zs[t * vq + b] = bet[t] * (Vs[t * vq + b] - gam[t] * ks[i][j]);
-                dUs[t * vq + b] = fmaf(Dd[t], kd[i][j], pd[i][j]);
+            for (int e = 0; e < 4; ++e) {
+                const int t = ks.row(e >> 1), b = ks.col(f) + (e & 1);
+                Zs[t * vq + b] = bet[t] * (Vs[t * vq + b] - gam[t] * ks.c[f][e]);
+                dUs[t * vq + b] = fmaf(Dd[t], kd.c[f][e], pd.c[f][e]);
             }
-        }
     }
     __syncthreads();
-    // U~ = T Z
-    for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
-        const Tile<2, true, true> tl(gi, kC, DVT);
-        float u[4][2];
-        zero(u);
-        tl.run(u, kC, Ts, cp, Zs, vq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float2 *>(Uts + tl.row(i) * vq + 2 * tl.tn) = make_float2(u[i][0], u[i][1]);
+    // U~ = T Z (A = T [t][s])
+    for (int tile = warp; tile < n_tv; tile += n_warps) {
+        WTile<true, true> w(tile, DVT);
+        w.run(kC, Ts, cp, Zs, vq);
+        w.each([&](int t, int b, float v0_, float v1_) { st2(Uts + t * vq + b, v0_, v1_); });
     }
     // T^T dU~ (A(t, s) = T[s][t], stored [k][m]): dV = diag(beta) T^T dU~, and V o T^T dU~
     // into Ps (P is no longer needed) for its row sums
-    for (int gi = tid; gi < (kC / 4) * (DVT / 2); gi += blockDim.x) {
-        const Tile<2, false, true> tl(gi, kC, DVT);
-        float w[4][2];
-        zero(w);
-        tl.run(w, kC, Ts, cp, dUs, vq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = tl.row(i), b = 2 * tl.tn;
-            if (t < n)
-                *reinterpret_cast<float2 *>(dv_out + ((size_t)(c0 + t) * H + h) * DV + v0 + b) =
-                    make_float2(bet[t] * w[i][0], bet[t] * w[i][1]);
-            Ps[t * cp + b] = Vs[t * vq + b] * w[i][0];
-            Ps[t * cp + b + 1] = Vs[t * vq + b + 1] * w[i][1];
-        }
+    for (int tile = warp; tile < n_tv; tile += n_warps) {
+        WTile<false, true> w(tile, DVT);
+        w.run(kC, Ts, cp, dUs, vq);
+        w.each([&](int t, int b, float w0, float w1) {
+            if (t < n) st2(dv_out + ((size_t)(c0 + t) * H + h) * DV + v0 + b, bet[t] * w0, bet[t] * w1);
+            Ps[t * cp + b] = Vs[t * vq + b] * w0;
+            Ps[t * cp + b + 1] = Vs[t * vq + b + 1] * w1;
+        });
     }
     __syncthreads();
     // row sums of V o T^T dU~: eight lanes per row
@@ -698,44 +671,22 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
         if (part == 0) Pvs[t] = acc;
     }
     // this slice's dY U~^T and dU~ Z^T [C][C] (B(b, s) = U~[s][b], Z[s][b]: stored [n][k])
-    for (int gi = tid; gi < (kC / 4) * (kC / 2); gi += blockDim.x) {
-        const Tile<2, true, false> tl(gi, kC, kC);
-        float p[4][2], tt[4][2];
-        zero(p);
-        zero(tt);
-        tl.run(p, DVT, dYs, vq, Uts, vq);
-        tl.run(tt, DVT, dUs, vq, Zs, vq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int e = tl.row(i) * kC + tl.col(j);
-                PdP[e] = p[i][j];
-                PdT[e] = tt[i][j];
-            }
+    for (int tile = warp; tile < (kC / 16) * (kC / 16); tile += n_warps) {
+        WTile<true, false> p(tile, kC), tt(tile, kC);
+        p.run(DVT, dYs, vq, Uts, vq);
+        tt.run(DVT, dUs, vq, Zs, vq);
+        p.each([&](int t, int s, float v0_, float v1_) { st2(PdP + t * kC + s, v0_, v1_); });
+        tt.each([&](int t, int s, float v0_, float v1_) { st2(PdT + t * kC + s, v0_, v1_); });
     }
     // this slice's -dU~ S^T, U~ dS'^T and dY S^T [C][DK] (B(b, a) = S[a][b]: stored [n][k])
-    for (int gi = tid; gi < (kC / 4) * (DK / 4); gi += blockDim.x) {
-        const Tile<4, true, false> tl(gi, kC, DK);
-        float acc[4][4];
-        zero(acc);
-        tl.run(acc, DVT, dUs, vq, Ss, vq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) PdW[tl.row(i) * DK + tl.col(j)] = -acc[i][j];
-        zero(acc);
-        tl.run(acc, DVT, Uts, vq, dSs, vq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) PdKd[tl.row(i) * DK + tl.col(j)] = acc[i][j];
-        zero(acc);
-        tl.run(acc, DVT, dYs, vq, Ss, vq);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) PdYS[tl.row(i) * DK + tl.col(j)] = acc[i][j];
+    for (int tile = warp; tile < (kC / 16) * (DK / 16); tile += n_warps) {
+        WTile<true, false> w(tile, DK), kd(tile, DK), ys(tile, DK);
+        w.run(DVT, dUs, vq, Ss, vq);
+        kd.run(DVT, Uts, vq, dSs, vq);
+        ys.run(DVT, dYs, vq, Ss, vq);
+        w.each([&](int t, int a, float v0_, float v1_) { st2(PdW + t * DK + a, -v0_, -v1_); });
+        kd.each([&](int t, int a, float v0_, float v1_) { st2(PdKd + t * DK + a, v0_, v1_); });
+        ys.each([&](int t, int a, float v0_, float v1_) { st2(PdYS + t * DK + a, v0_, v1_); });
     }
     // <dS', S> over this slice
     float sd = 0.f;
@@ -799,7 +750,7 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
     const int kq = ldp(DK), cp = ldp(kC);
     const int c = blockIdx.y, chain = blockIdx.x;
     const int seq = chain / H, h = chain % H;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, n_warps = blockDim.x >> 5;
     int64_t c0;
     int n;
     if (!chunk_of(cu_seqlens, seq, c, c0, n)) return;
@@ -838,33 +789,21 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         st4(G1 + t * cp + s, sum_slices4(oP + (size_t)t * kC + s));
     }
     __syncthreads();
+    const int n_cc = (kC / 16) * (kC / 16);
     // M = dT T^T into Asym (B(r, s) = T[s][r]: stored [n][k])
-    for (int gi = tid; gi < (kC / 4) * (kC / 4); gi += blockDim.x) {
-        const Tile<4, true, false> tl(gi, kC, kC);
-        float acc[4][4];
-        zero(acc);
-        tl.run(acc, kC, dGs, cp, Ts, cp);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) Asym[tl.row(i) * cp + tl.col(j)] = acc[i][j];
+    for (int tile = warp; tile < n_cc; tile += n_warps) {
+        WTile<true, false> w(tile, kC);
+        w.run(kC, dGs, cp, Ts, cp);
+        w.each([&](int t, int s, float v0, float v1) { st2(Asym + t * cp + s, v0, v1); });
     }
     __syncthreads();
     // dL = strict_tril(-T^T M) into dGs (A(t, r) = T[r][t]: stored [k][m])
-    for (int gi = tid; gi < (kC / 4) * (kC / 4); gi += blockDim.x) {
-        const Tile<4, false, true> tl(gi, kC, kC);
-        float acc[4][4];
-        zero(acc);
-        tl.run(acc, kC, Ts, cp, Asym, cp);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = tl.row(i);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int s = tl.col(j);
-                dGs[t * cp + s] = s < t ? -acc[i][j] : 0.f;
-            }
-        }
+    for (int tile = warp; tile < n_cc; tile += n_warps) {
+        WTile<false, true> w(tile, kC);
+        w.run(kC, Ts, cp, Asym, cp);
+        w.each([&](int t, int s, float v0, float v1) {
+            st2(dGs + t * cp + s, s < t ? -v0 : 0.f, s + 1 < t ? -v1 : 0.f);
+        });
     }
     __syncthreads();
     // dA + dA^T with dA = diag(beta) (dL o Gamma), into Asym (symmetric)
@@ -875,15 +814,13 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         Asym[t * cp + s] = da_ts + da_st;
     }
     // T^T dW (A(t, s) = T[s][t]), kept in registers until PdWs may be overwritten
-    constexpr int kMaxTiles = (kC / 4) * (128 / 4) / kThreadsWide;   // 1 at DK = 128
-    const int n_tiles = (kC / 4) * (DK / 4);
-    float tdw[kMaxTiles][4][4];
+    constexpr int kMaxWT = (kC / 16) * (128 / 16) / (kThreadsWide / 32);   // 2 at DK = 128
+    static_assert(kMaxWT == 2, "the tile arrays below are initialised for two tiles per warp");
+    const int n_ck = (kC / 16) * (DK / 16);
+    WTile<false, true> tdw[kMaxWT] = {WTile<false, true>(warp, DK), WTile<false, true>(warp + n_warps, DK)};
 #pragma unroll
-    for (int r = 0; r < kMaxTiles; ++r) {
-        zero(tdw[r]);
-        const int gi = tid + r * kThreadsWide;
-        if (gi < n_tiles) Tile<4, false, true>(gi, kC, DK).run(tdw[r], kC, Ts, cp, PdWs, kq);
-    }
+    for (int r = 0; r < kMaxWT; ++r)
+        if (warp + r * n_warps < n_ck) tdw[r].run(kC, Ts, cp, PdWs, kq);
     __syncthreads();
     // per entry (same thread reads and writes it): dGamma o Gamma into dGs, dL o A o Gamma into
     // Es, dP o Gamma into G1 and its transpose into G1T
@@ -909,15 +846,9 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         st4(G1 + t * cp + s0, make_float4(g1[0], g1[1], g1[2], g1[3]));
     }
 #pragma unroll
-    for (int r = 0; r < kMaxTiles; ++r) {
-        const int gi = tid + r * kThreadsWide;
-        if (gi < n_tiles) {
-            const Tile<4, false, true> tl(gi, kC, DK);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                st4(PdWs + tl.row(i) * kq + 4 * tl.tn, make_float4(tdw[r][i][0], tdw[r][i][1], tdw[r][i][2], tdw[r][i][3]));
-        }
-    }
+    for (int r = 0; r < kMaxWT; ++r)
+        if (warp + r * n_warps < n_ck)
+            tdw[r].each([&](int t, int a, float v0, float v1) { st2(PdWs + t * kq + a, v0, v1); });
     __syncthreads();
     if (tid < kC) {
         float rs = 0.f, cs = 0.f, ab = 0.f;
@@ -931,40 +862,29 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
     }
     // (dP o Gamma) K and (dP o Gamma)^T Q + (dA + dA^T) K, in registers until the region
     // Ts .. Es is free (A(t, s) = G1[t][s] = G1T[s][t], G1[s][t] and Asym[s][t]: all [k][m])
-    float aq[kMaxTiles][4][4], ak[kMaxTiles][4][4];
+    WTile<false, true> aq[kMaxWT] = {WTile<false, true>(warp, DK), WTile<false, true>(warp + n_warps, DK)};
+    WTile<false, true> ak[kMaxWT] = {WTile<false, true>(warp, DK), WTile<false, true>(warp + n_warps, DK)};
 #pragma unroll
-    for (int r = 0; r < kMaxTiles; ++r) {
-        zero(aq[r]);
-        zero(ak[r]);
-        const int gi = tid + r * kThreadsWide;
-        if (gi < n_tiles) {
-            const Tile<4, false, true> tl(gi, kC, DK);
-            tl.run(aq[r], kC, G1T, cp, Ks, kq);
-            tl.run(ak[r], kC, G1, cp, Qs, kq);
-            tl.run(ak[r], kC, Asym, cp, Ks, kq);
+    for (int r = 0; r < kMaxWT; ++r)
+        if (warp + r * n_warps < n_ck) {
+            aq[r].run(kC, G1T, cp, Ks, kq);
+            ak[r].run(kC, G1, cp, Qs, kq);
+            ak[r].run(kC, Asym, cp, Ks, kq);
         }
-    }
     __syncthreads();
     float *GQ = Ts, *GK = Ts + kC * kq;
 #pragma unroll
-    for (int r = 0; r < kMaxTiles; ++r) {
-        const int gi = tid + r * kThreadsWide;
-        if (gi < n_tiles) {
-            const Tile<4, false, true> tl(gi, kC, DK);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int o = tl.row(i) * kq + 4 * tl.tn;
-                st4(GQ + o, make_float4(aq[r][i][0], aq[r][i][1], aq[r][i][2], aq[r][i][3]));
-                st4(GK + o, make_float4(ak[r][i][0], ak[r][i][1], ak[r][i][2], ak[r][i][3]));
-            }
+    for (int r = 0; r < kMaxWT; ++r)
+        if (warp + r * n_warps < n_ck) {
+            aq[r].each([&](int t, int a, float v0, float v1) { st2(GQ + t * kq + a, v0, v1); });
+            ak[r].each([&](int t, int a, float v0, float v1) { st2(GK + t * kq + a, v0, v1); });
         }
-    }
     __syncthreads();
     // dQ = diag(gamma) dY S^T + (dP o Gamma) K;
     // dK = (dP o Gamma)^T Q + (dA + dA^T) K + diag(beta gamma) T^T dW + diag(D) dK~;
     // a warp per row t, four consecutive a per lane, with the row sums for dbeta and
     // dlog_alpha; two rows at a time so that their loads are in flight together
-    const int warp = tid >> 5, lane = tid & 31, n_warps = blockDim.x >> 5;
+    const int lane = tid & 31;
 #pragma unroll 2
     for (int t = warp; t < kC; t += n_warps) {
         float rg = 0.f, rb = 0.f, rd = 0.f;

@@ -89,11 +89,11 @@ def test_qsa_indexer_parity(lengths, Hq, r, K, dtype):
     _check(inp, r, K)
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_qsa_many_key_steps_split_over_ctas(dtype):
+@pytest.mark.parametrize("n,dtype", [(4100, "f32"), (4100, "bf16"), (9000, "bf16")])
+def test_qsa_many_key_steps_split_over_ctas(n, dtype):
     """A 4,100-token sequence at r = 1: up to 4,100 visible blocks per token, i.e. 33 key
-    steps of 128 blocks, split over several CTAs per query tile; sampled rows."""
-    n = 4100
+    steps of 128 blocks, split over several CTAs per query tile; sampled rows. 9,000 tokens:
+    72 key steps, and score rows of up to 9,000 blocks for the selection."""
     inp = W.make_qsa_inputs((n,), 2, dtype, seed=9)
     r, K = 1, 300
     I, B, T, cnt = _run(inp, r, K)
@@ -101,7 +101,7 @@ def test_qsa_many_key_steps_split_over_ctas(dtype):
     kx = inp["kx"].double().numpy()
     wq, wk = inp["wq"].double().numpy(), inp["wk"].double().numpy()
     kbv = Q.compress_keys(kx, r, wk)
-    rows = [0, 1, 127, 128, 1023, 2049, n - 1]
+    rows = [0, 1, 127, 128, 1023, 2049, n - 1] + ([8500] if n > 8500 else [])
     got, ref = [], []
     for i in rows:
         q = Q.prope(Q.rmsnorm(qx[i], wq), np.full((qx.shape[1],), i))
