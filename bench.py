@@ -650,15 +650,19 @@ def bench_backward(args, inp, device, pg):
         lens = (inp["cu_seqlens"][1:] - inp["cu_seqlens"][:-1]).tolist()
         n_cc = H * sum(-(-L // C) for L in lens)
         flops = n_cc * (28 * C * C * d + 20 * C * d * d + 4 * C ** 3)
-        # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the maximum SM clock)
-        peak = 148 * 128 * 2 * 1.965e9 / 1e12
         tf = flops / (ms * 1e-3) / 1e12
-        return {"kernel": "gdn::bwdc chunked backward (prep, fwd, state, vpart, kpart; fp32 CUDA cores)",
+        # the products run as tf32 mma.sync with a two-part operand split (three tensor-core
+        # products per product); peak: dense tf32 = measured bf16 x the nominal 1.1 / 2.25
+        peaks, kind = load_peaks()
+        peak_tf32 = peaks["bf16_tflops"] * 1.1 / 2.25
+        fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        return {"kernel": "gdn::bwdc chunked backward (prep, fwd, state, vpart, kpart; tf32x3 mma.sync)",
                 "ms_per_launch": ms, "tokens_per_s": n_tok / (ms * 1e-3), "launches": reps, "status": status,
                 "workload": "prefill shape: 4 x 4096 tokens, H=16, d=128, bf16 inputs",
-                "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                             "peak_source": "fp32 FMA rate from 148 SMs x 128 lanes at 1965 MHz",
-                             "flops_per_launch": flops}}
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf32, "unit": "TFLOP/s",
+                             "frac": tf / peak_tf32, "peak_source": f"{kind} bf16_tflops x 1.1/2.25 (tf32)",
+                             "flops_per_launch": flops, "tensor_products_per_product": 3,
+                             "fp32_fma_peak": fma_peak, "fp32_fma_frac": tf / fma_peak}}
     except Exception as exc:                      # reported, not raised
         return {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
