@@ -338,8 +338,8 @@ gdn_status gdn_featurize(const void *xq, const void *xk, const void *xv, gdn_dty
  *   blocks  [n_tok, K_B] int32 out (B_i)
  *   workspace >= gdn_qsa_workspace_bytes(...) bytes, 16-byte aligned: the normalised,
  *           rotated queries and compressed keys
- * Four launches on `stream` (vectors, scores, selection). The pages give no precision for
- * the indexer; the selection is taken on the scores this call returns.
+ * Four launches on `stream` (block and tile offsets, vectors, scores, selection). The pages
+ * give no precision for the indexer; the selection is taken on the scores this call returns.
  */
 size_t gdn_qsa_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, int Hq, int d, int r,
                                gdn_dtype dtype);
