@@ -732,7 +732,7 @@ def run_case(args):
     --case prefill:S,T,H   (bf16, d=128, chunk 64, bf16 y)
     --case prefill_gated:S,T,H (the same with the fused gate-norm, bf16 z and o)
     --case decode:N        (N sequences x 32 heads, d=128, fp32 state)
-    --case gate_norm:R     (R rows of d_v = 128: fp32 y, bf16 z and o)
+    --case gate_norm:R     (R rows of d_v = 128: bf16 y, z and o, as in the bench step)
     --case featurize:S,T,H (bf16, d=128, conv width 4)
     --case decode_tokens:N,T (N sequences x 32 heads, d=128, T tokens per call)
     --case qsa:N           (the QSA indexer on one N-token sequence, Hq=4, r=4, K=2048, bf16)
@@ -778,7 +778,7 @@ def run_case(args):
     elif kind == "gate_norm":
         (rows,) = dims
         g = torch.Generator().manual_seed(0)
-        y = torch.randn(rows, 128, generator=g).cuda()
+        y = torch.randn(rows, 128, generator=g).to(torch.bfloat16).cuda()
         z = torch.randn(rows, 128, generator=g).to(torch.bfloat16).cuda()
         wn = (torch.randn(128, generator=g) * 0.02).cuda()
         for _ in range(args.reps):
