@@ -94,7 +94,8 @@ namespace gdn {
 // n (<= kDecodeMaxTokens) consecutive tokens of every chain in one pass over S: the same
 // update as decode_step_kernel, applied token after token to each row while the row stays
 // in registers, so the state is read and written once per call instead of once per
-// token. A lane holds 16 consecutive elements of a row (LPR = d_k / 16 lanes per row), so
+// token. (d_k = d_v = 128 uses decode_tokens_pipe_kernel below; this one serves the
+// other sizes.) A lane holds 16 consecutive elements of a row (LPR = d_k / 16 lanes per row), so
 // each of the two dot products per row and token costs log2(LPR) shuffles. The tokens'
 // k, scale q, v, alpha, beta and k.(scale q) are staged in shared memory first.
 constexpr int kDecodeMaxTokens = 8;
@@ -199,6 +200,169 @@ decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
                     store4(Sc + (size_t)row[f] * DK + 16 * part + 4 * c,
                            make_float4(s[f][4 * c], s[f][4 * c + 1], s[f][4 * c + 2], s[f][4 * c + 3]));
     }
+}
+
+}  // namespace gdn
+
+namespace gdn {
+
+// ------------------------------------------------- several tokens per call, pipelined (d = 128)
+//
+// The same update as decode_tokens_kernel for d_k = d_v = 128, with the memory traffic of one
+// chain overlapped with the arithmetic of the previous one. A CTA walks the chains
+// blockIdx.x, blockIdx.x + gridDim.x, ...; each chain's state arrives in two halves of 64 rows
+// by cp.async into two shared-memory stages, its tokens (k, q, v, alpha, beta, raw) with the
+// first half into one of two token buffers. While half h of chain c is computed, half 1 - h
+// (or half 0 of the next chain) is in flight. A lane's 16 elements of a row are the float4
+// chunks at columns 32 j + 4 p (j = 0..3, p = lane % 8), so the 8 lanes of a row read 128
+// contiguous bytes; each lane copies exactly the state it later reads. The updated rows go
+// straight from registers to global memory.
+constexpr int kDecPipeThreads = 256;
+constexpr int kDecPipeHalf = 64;
+
+__device__ __forceinline__ uint32_t dec_smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dec_smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dec_smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <typename T>
+__host__ __device__ constexpr size_t decode_pipe_smem_bytes()
+{
+    return 2 * (size_t)kDecPipeHalf * 128 * sizeof(float) + 2 * 3 * (size_t)kDecodeMaxTokens * 128 * sizeof(T) +
+           2 * 2 * (size_t)kDecodeMaxTokens * sizeof(float);
+}
+
+template <typename T, typename TY>
+__global__ void __launch_bounds__(kDecPipeThreads, 2)
+decode_tokens_pipe_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                          const float *__restrict__ alpha, const float *__restrict__ beta, float *__restrict__ S,
+                          int n, int H, int n_chain, float scale, TY *__restrict__ y)
+{
+    constexpr int DK = 128, DV = 128, LPR = 8, RPW = 4, WARPS = kDecPipeThreads / 32, HALF = kDecPipeHalf;
+    constexpr int TOK = kDecodeMaxTokens, EPC = 16 / (int)sizeof(T);   // elements per 16-byte chunk
+    static_assert(2 * WARPS * RPW == HALF, "two passes of the warps cover a half");
+    extern __shared__ __align__(16) unsigned char dec_sm[];
+    float *stage = reinterpret_cast<float *>(dec_sm);                     // [2][HALF][DK]
+    T *tk = reinterpret_cast<T *>(stage + 2 * HALF * DK);                 // [2][TOK][DK]
+    T *tq = tk + 2 * TOK * DK;                                            // [2][TOK][DK]
+    T *tv = tq + 2 * TOK * DK;                                            // [2][TOK][DV]
+    float *tab = reinterpret_cast<float *>(tv + 2 * TOK * DV);            // [2][alpha, beta][TOK]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int p = lane % LPR, sub = lane / LPR;
+    auto row_of = [&](int f) { return (f * WARPS + warp) * RPW + sub; };  // row within a half
+    auto tok_row = [&](int chain, int i) -> size_t { return ((size_t)(chain / H) * n + i) * H + chain % H; };
+
+    // one commit group: half h of `chain`'s state, with h == 0 also its tokens into buffer tb
+    // (an empty group past the last chain keeps the group count uniform)
+    auto issue = [&](int chain, int h, int tb) {
+        if (chain < n_chain) {
+            const float *src = S + ((size_t)chain * DV + (size_t)h * HALF) * DK;
+            float *dst = stage + h * HALF * DK;
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+                const int r = row_of(f);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) cp_async16(dst + r * DK + 32 * j + 4 * p, src + (size_t)r * DK + 32 * j + 4 * p);
+            }
+            if (h == 0) {
+                constexpr int CK = DK / EPC, CV = DV / EPC;              // 16-byte chunks per row
+                for (int e = tid; e < n * (2 * CK + CV); e += blockDim.x) {
+                    const int i = e / (2 * CK + CV), w = e % (2 * CK + CV);
+                    const size_t tr = tok_row(chain, i);
+                    if (w < CK)
+                        cp_async16(tk + (tb * TOK + i) * DK + w * EPC, k + tr * DK + w * EPC);
+                    else if (w < 2 * CK)
+                        cp_async16(tq + (tb * TOK + i) * DK + (w - CK) * EPC, q + tr * DK + (w - CK) * EPC);
+                    else
+                        cp_async16(tv + (tb * TOK + i) * DV + (w - 2 * CK) * EPC, v + tr * DV + (w - 2 * CK) * EPC);
+                }
+                if (tid < 2 * n) {
+                    const int i = tid % n, which = tid / n;
+                    cp_async4(tab + (tb * 2 + which) * TOK + i, (which == 0 ? alpha : beta) + tok_row(chain, i));
+                }
+            }
+        }
+        cp_async_commit();
+    };
+
+    int it = 0;
+    issue(blockIdx.x, 0, 0);
+    issue(blockIdx.x, 1, 0);
+    for (int c = blockIdx.x; c < n_chain; c += gridDim.x, ++it) {
+        const int tb = it & 1;
+        float *Sc = S + (size_t)c * DV * DK;
+        for (int h = 0; h < 2; ++h) {
+            cp_async_wait1();               // this half (and its tokens) has landed, for this thread
+            __syncthreads();                // ... and for every thread
+            const float *src = stage + h * HALF * DK;
+            float s[2][16];
+#pragma unroll
+            for (int f = 0; f < 2; ++f)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 x = *reinterpret_cast<const float4 *>(src + row_of(f) * DK + 32 * j + 4 * p);
+                    s[f][4 * j] = x.x; s[f][4 * j + 1] = x.y; s[f][4 * j + 2] = x.z; s[f][4 * j + 3] = x.w;
+                }
+#pragma unroll 1
+            for (int i = 0; i < n; ++i) {
+                float kv[16], qv[16];
+                float kq = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 a4 = load4(tk + (tb * TOK + i) * DK + 32 * j + 4 * p);
+                    const float4 b4 = load4(tq + (tb * TOK + i) * DK + 32 * j + 4 * p);
+                    kv[4 * j] = a4.x; kv[4 * j + 1] = a4.y; kv[4 * j + 2] = a4.z; kv[4 * j + 3] = a4.w;
+                    qv[4 * j] = scale * b4.x; qv[4 * j + 1] = scale * b4.y;
+                    qv[4 * j + 2] = scale * b4.z; qv[4 * j + 3] = scale * b4.w;
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) kq = fmaf(kv[e], qv[e], kq);
+                kq = group_sum<LPR>(kq);
+                const float a = tab[(tb * 2) * TOK + i], b = tab[(tb * 2 + 1) * TOK + i];
+                const size_t tr = tok_row(c, i);
+#pragma unroll
+                for (int f = 0; f < 2; ++f) {
+                    float u = 0.f, r = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        u = fmaf(s[f][e], kv[e], u);
+                        r = fmaf(s[f][e], qv[e], r);
+                    }
+                    u = group_sum<LPR>(u);
+                    r = group_sum<LPR>(r);
+                    const int row = h * HALF + row_of(f);
+                    const float ev = to_f32(tv[(tb * TOK + i) * DV + row]) - a * u;
+                    const float be = b * ev;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) s[f][e] = fmaf(a, s[f][e], be * kv[e]);
+                    if (p == 0) y[tr * DV + row] = from_f32<TY>(fmaf(a, r, be * kq));
+                }
+            }
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+                const int row = h * HALF + row_of(f);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    store4(Sc + (size_t)row * DK + 32 * j + 4 * p,
+                           make_float4(s[f][4 * j], s[f][4 * j + 1], s[f][4 * j + 2], s[f][4 * j + 3]));
+            }
+            __syncthreads();                // every thread is done with this stage (and, at h = 1,
+                                            // with this chain's tokens)
+            issue(c + gridDim.x, h, tb ^ 1);
+        }
+    }
+    cp_async_wait_all();
 }
 
 }  // namespace gdn

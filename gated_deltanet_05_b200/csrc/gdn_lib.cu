@@ -602,6 +602,32 @@ gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dt
         !aligned(beta, 4) || !aligned(v, 4) || !aligned(y, 4))
         return GDN_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
+    if (d_k == 128 && d_v == 128 && aligned(v, 16)) {
+        // pipelined kernel: two persistent CTAs per SM walk the chains
+        int dev = 0, n_sm = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        const unsigned grid_p = (unsigned)(n_chain < 2LL * n_sm ? n_chain : 2LL * n_sm);
+#define GDN_DECPIPE_LAUNCH(T, TY)                                                                  \
+    {                                                                                              \
+        auto kern = gdn::decode_tokens_pipe_kernel<T, TY>;                                         \
+        constexpr int smem = (int)gdn::decode_pipe_smem_bytes<T>();                                \
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+            return GDN_ERR_CUDA;                                                                   \
+        kern<<<grid_p, gdn::kDecPipeThreads, smem, st>>>((const T *)q, (const T *)k, (const T *)v, alpha, beta, S, \
+                                                         n_tokens, H, (int)n_chain, scale, (TY *)y);  \
+    }
+        if (in_dtype == GDN_F32) {
+            if (y_dtype == GDN_F32) GDN_DECPIPE_LAUNCH(float, float)
+            else GDN_DECPIPE_LAUNCH(float, __nv_bfloat16)
+        } else {
+            if (y_dtype == GDN_F32) GDN_DECPIPE_LAUNCH(__nv_bfloat16, float)
+            else GDN_DECPIPE_LAUNCH(__nv_bfloat16, __nv_bfloat16)
+        }
+#undef GDN_DECPIPE_LAUNCH
+        return launch_status();
+    }
     const unsigned grid = (unsigned)n_chain;
 #define GDN_DECTOK_LAUNCH(DK, T, TY)                                                               \
     gdn::decode_tokens_kernel<DK, T, TY><<<grid, gdn::kDecodeTokThreads, 0, st>>>(                 \
