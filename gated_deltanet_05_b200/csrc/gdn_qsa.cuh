@@ -427,8 +427,9 @@ __device__ __forceinline__ uint32_t fkey(float x)
 // blocks, ordered by (score descending, block ascending); -1 padded. Radix selection on the
 // order-preserving keys (four 8-bit passes over the row, a 256-bin histogram per warp in
 // shared memory) finds the kb-th largest key T; the keys above T and the lowest-index keys
-// equal to T are gathered (ballots keep index order), then sorted by the warp (bitonic, in
-// its shared-memory slice). Rows with at most kb visible blocks take every block.
+// equal to T are gathered (ballots keep index order), then sorted by the warp (bitonic: in
+// registers for selections of up to kTopkRegSort entries, else in its shared-memory slice).
+// Rows with at most kb visible blocks take every block.
 constexpr int kTopkWarps = 4;
 
 __host__ __device__ inline int topk_pow2(int kb)
@@ -440,6 +441,28 @@ __host__ __device__ inline int topk_pow2(int kb)
 __host__ __device__ inline size_t topk_smem_bytes(int kb)
 {
     return (size_t)kTopkWarps * ((size_t)topk_pow2(kb) * sizeof(unsigned long long) + 256 * sizeof(int));
+}
+
+// Selections of 16..512 entries are sorted in registers: 16 keys per lane, entry i =
+// 16 lane + e. Pairs (i, i ^ jj) with jj < 16 sit in one lane; with jj >= 16 they are
+// exchanged by shuffles. kTopkRegSort entries in all (zeros pad the selection and sort last).
+constexpr int kTopkRegSort = 512;
+// where entry i of a register-sorted selection is kept in shared memory: rotated inside its
+// 16-entry group, so that the 32 lanes loading entries 16 lane + e for one e hit distinct banks
+__device__ __forceinline__ int topk_swz(int i) { return (i & ~15) | ((i + (i >> 4)) & 15); }
+
+template <int JJ>
+__device__ __forceinline__ void bitonic_in_lane(unsigned long long (&v)[16], int lane, int k)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+        if ((e & JJ) == 0) {
+            const bool desc = ((lane * 16 + e) & k) == 0;
+            const unsigned long long a = v[e], b = v[e | JJ];
+            const bool sw = desc ? (a < b) : (a > b);
+            v[e] = sw ? b : a;
+            v[e | JJ] = sw ? a : b;
+        }
 }
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
@@ -515,6 +538,8 @@ qsa_topk_kernel(const float *__restrict__ I, const int32_t *__restrict__ cu, int
     // `need` lowest-index keys equal to T
     const uint32_t T = prefix;
     const bool all = nvis <= kb;
+    const bool reg_sort = kb2 >= 16 && kb2 <= kTopkRegSort;
+    auto slot = [&](int i) { return reg_sort ? topk_swz(i) : i; };
     int n_gt = 0, n_eq = 0;
     for (int b0 = 0; b0 < nvis; b0 += 32) {
         const int b = b0 + lane;
@@ -523,15 +548,53 @@ qsa_topk_kernel(const float *__restrict__ I, const int32_t *__restrict__ cu, int
         const bool eq = b < nvis && !all && key == T;
         const unsigned mg = __ballot_sync(0xffffffffu, gt), me = __ballot_sync(0xffffffffu, eq);
         const unsigned below = (1u << lane) - 1u;
-        if (gt) sel[n_gt + __popc(mg & below)] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)b);
+        if (gt) sel[slot(n_gt + __popc(mg & below))] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)b);
         if (eq) {
             const int at = n_eq + __popc(me & below);
-            if (at < need) sel[kb - need + at] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)b);
+            if (at < need) sel[slot(kb - need + at)] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)b);
         }
         n_gt += __popc(mg);
         n_eq += __popc(me);
     }
     __syncwarp();
+    int32_t *out = B + (size_t)t * kb;
+    if (reg_sort) {
+        // bitonic sort, descending, of kTopkRegSort entries in registers
+        unsigned long long v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int i = lane * 16 + e;
+            v[e] = i < take ? sel[topk_swz(i)] : 0ull;
+        }
+        for (int k = 2; k <= kTopkRegSort; k <<= 1)
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                if (jj >= 16) {
+                    const int lm = jj >> 4;
+                    const bool upper = (lane & lm) != 0;      // this lane holds the higher index
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const bool desc = ((lane * 16 + e) & k) == 0;
+                        const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[e], lm);
+                        const bool keep_max = desc != upper;
+                        v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+                    }
+                } else if (jj == 8) {
+                    bitonic_in_lane<8>(v, lane, k);
+                } else if (jj == 4) {
+                    bitonic_in_lane<4>(v, lane, k);
+                } else if (jj == 2) {
+                    bitonic_in_lane<2>(v, lane, k);
+                } else {
+                    bitonic_in_lane<1>(v, lane, k);
+                }
+            }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int i = lane * 16 + e;
+            if (i < kb) out[i] = i < take ? (int32_t)(0xffffffffu - (uint32_t)(v[e] & 0xffffffffull)) : -1;
+        }
+        return;
+    }
     for (int i = take + lane; i < kb2; i += 32) sel[i] = 0ull;
     __syncwarp();
     // bitonic sort, descending
@@ -550,7 +613,6 @@ qsa_topk_kernel(const float *__restrict__ I, const int32_t *__restrict__ cu, int
             }
             __syncwarp();
         }
-    int32_t *out = B + (size_t)t * kb;
     for (int i = lane; i < kb; i += 32)
         out[i] = i < take ? (int32_t)(0xffffffffu - (uint32_t)(sel[i] & 0xffffffffull)) : -1;
 }
