@@ -669,7 +669,9 @@ def bench_backward(args, inp, device, pg):
 
 def bench_e2e(args, inp, device, pg, world):
     """Same step through the public API with the inputs in pinned host memory: H2D copy of
-    q, k, v, log_alpha, beta, z every step, D2H read of the output o."""
+    q, k, v, log_alpha, beta, z every step, D2H read of the output o. Steps are pipelined
+    over three streams and two device buffer sets: step i's inputs go up while step i - 1
+    computes and step i - 2's output comes down (H2D and D2H use separate copy engines)."""
     import torch
 
     import gated_deltanet_05_b200 as gdn
@@ -678,36 +680,60 @@ def bench_e2e(args, inp, device, pg, world):
     w_dev = inp["w_norm"].to(device)
     cu_host = inp["cu_seqlens"]
     cu_dev = cu_host.to(device)
-    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
-    o_host = torch.empty(inp["v"].shape, dtype=inp["v"].dtype).pin_memory()
-    stream = torch.cuda.current_stream(device)
+    dev = [{k: torch.empty_like(v, device=device) for k, v in host.items()} for _ in range(2)]
+    outs = [None, None]
+    o_host = [torch.empty(inp["v"].shape, dtype=inp["v"].dtype).pin_memory() for _ in range(2)]
+    s_in = torch.cuda.Stream(device)
+    s_cmp = torch.cuda.Stream(device)
+    s_out = torch.cuda.Stream(device)
+    done_cmp = [torch.cuda.Event(), torch.cuda.Event()]   # buffer set free again
+    done_out = [torch.cuda.Event(), torch.cuda.Event()]   # output buffer read back
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = o_host.numel() * o_host.element_size()
+    d2h = o_host[0].numel() * o_host[0].element_size()
+    first = [True, True]
 
-    def step():
-        for k in host:
-            dev[k].copy_(host[k], non_blocking=True)
-        y, _ = gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], cu_dev,
-                             chunk=C, cu_seqlens_host=cu_host, y_dtype=torch.bfloat16)
-        o = gdn.gate_norm(y, dev["z"], w_dev, out_dtype=torch.bfloat16)
-        o_host.copy_(o, non_blocking=True)
+    def step(i):
+        j = i & 1
+        with torch.cuda.stream(s_in):
+            if not first[j]:
+                s_in.wait_event(done_cmp[j])      # step i - 2 has finished reading this set
+            for k in host:
+                dev[j][k].copy_(host[k], non_blocking=True)
+            up = torch.cuda.Event()
+            up.record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(up)
+            if not first[j]:
+                s_cmp.wait_event(done_out[j])     # step i - 2's output has been read back
+            d = dev[j]
+            y, _ = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], cu_dev,
+                                 chunk=C, cu_seqlens_host=cu_host, y_dtype=torch.bfloat16)
+            outs[j] = gdn.gate_norm(y, d["z"], w_dev, out_dtype=torch.bfloat16)
+            done_cmp[j].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done_cmp[j])
+            o_host[j].copy_(outs[j], non_blocking=True)
+            done_out[j].record(s_out)
+        first[j] = False
 
-    for _ in range(2):
-        step()
+    for i in range(2):
+        step(i)
     torch.cuda.synchronize(device)
     steps = max(1, min(args.steps, 20))
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     barrier(pg, device)
-    a.record(stream)
-    for _ in range(steps):
-        step()
-    b.record(stream)
+    a.record(s_in)
+    for i in range(steps):
+        step(i)
+    s_in.wait_stream(s_out)
+    b.record(s_in)
     torch.cuda.synchronize(device)
     ms = max_over_ranks(pg, a.elapsed_time(b), device) / steps
     n_tok = inp["q"].shape[0]
     return {"value": n_tok * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "pipelined": "3 streams, 2 device buffer sets: H2D of step i, compute of i - 1, D2H of i - 2"}
 
 
 def cpu_baseline(inp, H, min_seconds=10.0, max_reps=12):
