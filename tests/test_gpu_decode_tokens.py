@@ -6,7 +6,8 @@ state. Bar: max|got - ref| / rms(ref) on every fp32 y and on the final state, fp
 <= 1e-4, bf16 inputs <= 2e-2; a bf16 y must be the round-to-nearest-even of the fp32 y
 of the same call (the two calls start from the same state). Cases: every d (16..128), d_k != d_v,
 1..8 tokens, odd head counts, more chains than SMs, a 400-token run of 100 calls of 4
-tokens, and agreement with n calls of gdn_decode_step.
+tokens, agreement with n calls of gdn_decode_step, and at d = 128 the pipelined kernel
+against the one-CTA-per-chain kernel (taken when v is not 16-byte aligned).
 """
 import numpy as np
 import pytest
@@ -110,5 +111,34 @@ def test_decode_tokens_matches_single_steps():
                                        v[:, i].contiguous().cuda(), alpha[:, i].contiguous().cuda(),
                                        beta[:, i].contiguous().cuda(), S_b) for i in range(n)], 1)
     torch.cuda.synchronize()
+    assert rel_err(f64(y_a), f64(y_b)) <= 1e-5
+    assert rel_err(f64(S_a), f64(S_b)) <= 1e-5
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_tokens_both_kernels_agree(dtype):
+    """d = 128 runs the pipelined kernel when v is 16-byte aligned and the one-CTA-per-chain
+    kernel otherwise (v only needs 4-byte alignment); both against the oracle, and against
+    each other."""
+    n_seq, n, H, d = 6, 4, 3, 128
+    q, k, v, alpha, beta = _tokens(n_seq, n, H, d, d, dtype, seed=11)
+    S0 = (torch.randn(n_seq, H, d, d, generator=torch.Generator().manual_seed(2)) * 0.05).float()
+    args = [q.cuda(), k.cuda(), v.cuda(), alpha.cuda(), beta.cuda()]
+    S_a = S0.cuda()
+    y_a = gdn.decode_tokens(*args, S_a)
+    # the same v 4 bytes into a larger buffer: 4-byte aligned (what the call requires of v),
+    # not 16-byte aligned
+    off = 4 // v.element_size()
+    big = torch.empty(v.numel() + 16, dtype=v.dtype, device="cuda")
+    v_off = big[off:off + v.numel()].view(v.shape)
+    v_off.copy_(args[2])
+    assert v_off.data_ptr() % 16 != 0 and v_off.data_ptr() % 4 == 0
+    S_b = S0.cuda()
+    y_b = gdn.decode_tokens(args[0], args[1], v_off, args[3], args[4], S_b)
+    torch.cuda.synchronize()
+    y_ref, S_ref = _oracle(q, k, v, alpha, beta, S0.numpy().astype(np.float64))
+    for y, S in ((y_a, S_a), (y_b, S_b)):
+        assert rel_err(f64(y), y_ref) <= TOL[dtype]
+        assert rel_err(f64(S), S_ref) <= TOL[dtype]
     assert rel_err(f64(y_a), f64(y_b)) <= 1e-5
     assert rel_err(f64(S_a), f64(S_b)) <= 1e-5
