@@ -246,7 +246,7 @@ __device__ __forceinline__ bool chunk_of(const int32_t *__restrict__ cu_seqlens,
 
 // --------------------------------------------------------------------------- prep
 struct PrepSmem {
-    int KQ, Ls, Ts, g, gam, bet, Dd, total;
+    int KQ, Ls, Ts, Ms, g, gam, bet, Dd, total;
 };
 __host__ __device__ inline PrepSmem prep_layout(int DK)
 {
@@ -256,6 +256,7 @@ __host__ __device__ inline PrepSmem prep_layout(int DK)
     L.KQ = o; o += 2 * kC * kq;
     L.Ls = o; o += kC * cp;
     L.Ts = o; o += kC * cp;
+    L.Ms = o; o += 3 * 16 * 16;
     L.g = o; o += kC;
     L.gam = o; o += kC;
     L.bet = o; o += kC;
@@ -265,7 +266,9 @@ __host__ __device__ inline PrepSmem prep_layout(int DK)
 }
 
 // One CTA (kThreads) per (chain, chunk): [K; Q] K^T, then A o Gamma, P and L; T = (I + L)^-1
-// row by row (four lanes per entry); W = T diag(beta gamma) K. All into the chunk's cache.
+// by 16 x 16 blocks (diagonal blocks by forward substitution, one column per thread; then
+// T_ba = -T_bb sum_{a <= k < b} L_bk T_ka, one block diagonal at a time);
+// W = T diag(beta gamma) K. All into the chunk's cache.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ log_alpha,
@@ -307,18 +310,36 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
         });
     }
     __syncthreads();
-    // T[t][j] = -sum_{j <= s < t} L[t][s] T[s][j] for j < t, one row after the other
-    {
-        const int j = tid >> 2, part = tid & 3;
-        for (int t = 1; t < kC; ++t) {
+    // diagonal blocks: column j of block b, T[t][j] = -sum_{j <= s < t} L[t][s] T[s][j] for
+    // j < t inside the block (the thread writes and reads back only its own column)
+    if (tid < kC) {
+        const int b16 = (tid >> 4) * 16, j = b16 + (tid & 15);
+        for (int t = j + 1; t < b16 + 16; ++t) {
             float x = 0.f;
-            if (j < t)
-                for (int s = j + part; s < t; s += 4) x = fmaf(Ls[t * cp + s], Ts[s * cp + j], x);
-            x += __shfl_xor_sync(0xffffffffu, x, 1);
-            x += __shfl_xor_sync(0xffffffffu, x, 2);
-            if (part == 0 && j < t) Ts[t * cp + j] = -x;
-            __syncthreads();
+            for (int sd = j; sd < t; ++sd) x = fmaf(Ls[t * cp + sd], Ts[sd * cp + j], x);
+            Ts[t * cp + j] = -x;
         }
+    }
+    __syncthreads();
+    // off-diagonal blocks, distance d = b - a = 1, 2, 3: M = sum_{a <= k < b} L_bk T_ka, then
+    // T_ba = -T_bb M (the blocks of one distance are independent)
+    float *Ms = sm + Y.Ms;
+    for (int d = 1; d < 4; ++d) {
+        const int nblk = 4 - d;
+        for (int i = tid; i < nblk * 256; i += blockDim.x) {
+            const int a = i >> 8, t = (i >> 4) & 15, j = i & 15, b = a + d;
+            float x = 0.f;
+            for (int sd = 16 * a; sd < 16 * b; ++sd) x = fmaf(Ls[(16 * b + t) * cp + sd], Ts[sd * cp + 16 * a + j], x);
+            Ms[i] = x;
+        }
+        __syncthreads();
+        for (int i = tid; i < nblk * 256; i += blockDim.x) {
+            const int a = i >> 8, t = (i >> 4) & 15, j = i & 15, b = a + d;
+            float x = 0.f;
+            for (int sd = 0; sd <= t; ++sd) x = fmaf(Ts[(16 * b + t) * cp + 16 * b + sd], Ms[(a << 8) + sd * 16 + j], x);
+            Ts[(16 * b + t) * cp + 16 * a + j] = -x;
+        }
+        __syncthreads();
     }
     for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
         const int r = i / (kC / 4), c4 = (i % (kC / 4)) * 4;
