@@ -69,10 +69,19 @@ __device__ __forceinline__ void chunk_decays(const float *__restrict__ log_alpha
                                              float *Dd)
 {
     const int lane = threadIdx.x;
+    // the four loads first, so that they are in flight together
+    float la[kC / 32], be[kC / 32];
+#pragma unroll
+    for (int j = 0; j < kC / 32; ++j) {
+        const int t = 32 * j + lane;
+        la[j] = t < n ? log_alpha[(size_t)(c0 + t) * H + h] : 0.f;
+        be[j] = t < n ? beta[(size_t)(c0 + t) * H + h] : 0.f;
+    }
     float carry = 0.f;
-    for (int base = 0; base < kC; base += 32) {
-        const int t = base + lane;
-        float x = t < n ? log_alpha[(size_t)(c0 + t) * H + h] : 0.f;
+#pragma unroll
+    for (int j = 0; j < kC / 32; ++j) {
+        const int t = 32 * j + lane;
+        float x = la[j];
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const float y_ = __shfl_up_sync(0xffffffffu, x, off);
@@ -82,7 +91,7 @@ __device__ __forceinline__ void chunk_decays(const float *__restrict__ log_alpha
         carry = __shfl_sync(0xffffffffu, x, 31);
         g[t] = x;
         gam[t] = expf(x);
-        bet[t] = t < n ? beta[(size_t)(c0 + t) * H + h] : 0.f;
+        bet[t] = be[j];
     }
     __syncwarp();
     const float gC = g[kC - 1];
@@ -128,6 +137,66 @@ __device__ __forceinline__ void load_rows_t(float *dst, int ld, const T *__restr
         dst[(a + 2) * ld + t] = x.z;
         dst[(a + 3) * ld + t] = x.w;
     }
+}
+
+// Up to R float4 row pieces of a chunk's rows per thread, loaded into registers before any is
+// stored (so all of a thread's loads are in flight together), then stored to shared memory
+// [kC][ld], or transposed ([ncol][ld]) when TRANS. Piece i = tid + r blockDim covers four
+// columns of one row: row i / nq, columns 4 (i % nq) .. (nq = ncol / 4); for TRANS a warp
+// takes 8 rows x 16 columns instead, so that its transposed stores meet at most two to a bank
+// while each row's 16 columns still fill whole sectors. Zero past n.
+template <bool TRANS>
+__device__ __forceinline__ void piece_at(int i, int nq, int &t, int &a)
+{
+    if (TRANS) {
+        const int rest = i >> 3;
+        a = (rest % nq) * 4;
+        t = (rest / nq) * 8 + (i & 7);
+    } else {
+        t = i / nq;
+        a = (i % nq) * 4;
+    }
+}
+template <bool TRANS, int R, typename T>
+__device__ __forceinline__ void fetch_rows(float4 (&x)[R], const T *__restrict__ src, int64_t c0, int n, int H,
+                                           int h, int D, int col0, int ncol)
+{
+    const int nq = ncol >> 2;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int i = threadIdx.x + r * blockDim.x;
+        int t, a;
+        piece_at<TRANS>(i, nq, t, a);
+        x[r] = (i < kC * nq && t < n) ? load4(src + ((size_t)(c0 + t) * H + h) * D + col0 + a)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+template <bool TRANS, int R>
+__device__ __forceinline__ void put_rows(float *dst, int ld, const float4 (&x)[R], int ncol)
+{
+    const int nq = ncol >> 2;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int i = threadIdx.x + r * blockDim.x;
+        if (i >= kC * nq) continue;
+        int t, a;
+        piece_at<TRANS>(i, nq, t, a);
+        if (TRANS) {
+            dst[(a + 0) * ld + t] = x[r].x;
+            dst[(a + 1) * ld + t] = x[r].y;
+            dst[(a + 2) * ld + t] = x[r].z;
+            dst[(a + 3) * ld + t] = x[r].w;
+        } else {
+            st4(dst + t * ld + a, x[r]);
+        }
+    }
+}
+// A row-major [rows][cols] fp32 block of the cache by cp.async into shared memory [rows][ld]
+// (one commit group is left to the caller)
+__device__ __forceinline__ void copy_block_async(float *dst, int ld, const float *__restrict__ src, int rows, int cols)
+{
+    const int nq = cols >> 2;
+    for (int i = threadIdx.x; i < rows * nq; i += blockDim.x) cp_async16(dst + (i / nq) * ld + (i % nq) * 4, src + 4 * (size_t)i);
 }
 
 // A row-major [rows][cols] fp32 block (global, 16-byte aligned) into shared memory [rows][ld],
@@ -360,7 +429,7 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
 
 // --------------------------------------------------------------------------- fwd
 struct FwdSmem {
-    int Kd, Wn, Ts, Vb, Us, Ss, g, gam, bet, Dd, total;
+    int Kd, Ws, Ts, Vb, Us, Ss, g, gam, bet, Dd, total;
 };
 __host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT)
 {
@@ -368,7 +437,7 @@ __host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT)
     int o = 0;
     const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
     L.Kd = o; o += kC * kq;
-    L.Wn = o; o += kC * kq;
+    L.Ws = o; o += kC * kq;
     L.Ts = o; o += kC * cp;
     L.Vb = o; o += kC * vq;
     L.Us = o; o += kC * vq;
@@ -394,7 +463,7 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
     extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
     const FwdSmem Y = fwd_layout(DK, DVT);
-    float *Kd = sm + Y.Kd, *Wn = sm + Y.Wn, *Ts = sm + Y.Ts, *Vb = sm + Y.Vb, *Us = sm + Y.Us, *Ss = sm + Y.Ss;
+    float *Kd = sm + Y.Kd, *Ws = sm + Y.Ws, *Ts = sm + Y.Ts, *Vb = sm + Y.Vb, *Us = sm + Y.Us, *Ss = sm + Y.Ss;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd;
     const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
     const int n_vt = DV / DVT;
@@ -409,11 +478,19 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
     }
     const int n_chunks = (int)((len + kC - 1) / kC);
     const int nvq = DVT / 4;
+    // T and W of a chunk are requested as soon as the buffers are free: chunk 0's here, chunk
+    // c + 1's right after chunk c's U~ product
+    auto request_tw = [&](int c) {
+        const float *cb = cache + ((size_t)chain * max_chunks + c) * cache_floats(DK);
+        copy_block_async(Ts, cp, cb + kCacheT, kC, kC);
+        copy_block_async(Ws, kq, cb + kCacheW, kC, DK);
+        cp_async_commit();
+    };
+    if (n_chunks > 0) request_tw(0);
     for (int c = 0; c < n_chunks; ++c) {
         int64_t c0;
         int n;
         chunk_of(cu_seqlens, seq, c, c0, n);
-        const float *cb = cache + ((size_t)chain * max_chunks + c) * cache_floats(DK);
         __syncthreads();
         {
             float *dst = S_chunks + ((size_t)chain * max_chunks + c) * DK * DV + v0;
@@ -422,11 +499,17 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
                 st4(dst + (size_t)a * DV + b, f4(Ss + a * vq + b));
             }
         }
-        load_rows(Kd, kq, k, c0, n, H, h, DK, 0, DK, 1.f);
-        load_rows(Vb, vq, v, c0, n, H, h, DV, v0, DVT, 1.f);
-        load_block(Ts, cp, cb + kCacheT, kC, kC, 1.f);
-        load_block(Wn, kq, cb + kCacheW, kC, DK, -1.f);
-        if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+        // the chunk's K and V rows into registers, all loads in flight together, and the
+        // decays on warp 0 (T and W are on their way)
+        {
+            float4 kr[kC * 128 / 4 / kThreadsWide], vr[kC * kDVT / 4 / kThreadsWide];
+            fetch_rows<false>(kr, k, c0, n, H, h, DK, 0, DK);
+            fetch_rows<false>(vr, v, c0, n, H, h, DV, v0, DVT);
+            if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+            put_rows<false>(Kd, kq, kr, DK);
+            put_rows<false>(Vb, vq, vr, DVT);
+        }
+        cp_async_wait_all();
         __syncthreads();
         for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
             const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
@@ -439,12 +522,17 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
         __syncthreads();
         // U~ = T diag(beta) V - W S
         for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
-            WTile<true, true> w(tile, DVT);
+            WTile<true, true> w(tile, DVT), ws(tile, DVT);
             w.run(kC, Ts, cp, Vb, vq);
-            w.run(DK, Wn, kq, Ss, vq);
+            ws.run(DK, Ws, kq, Ss, vq);
+#pragma unroll
+            for (int f = 0; f < 2; ++f)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w.c[f][e] -= ws.c[f][e];
             w.each([&](int t, int b, float v0_, float v1_) { st2(Us + t * vq + b, v0_, v1_); });
         }
         __syncthreads();
+        if (c + 1 < n_chunks) request_tw(c + 1);     // T and W are free: the next chunk's
         // S <- gamma_C S + (diag(D) K)^T U~: A(a, s) = Kd[s][a] stored [k][m]; each warp reads
         // and writes only its own entries of S
         const float gamC = gam[kC - 1];
@@ -462,7 +550,7 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
 
 // --------------------------------------------------------------------------- state
 struct StateSmem {
-    int Kt, Qg, Wn, Ps, dYs, dUs, dSs, g, gam, bet, Dd, total;
+    int Kt, Qg, Ws, Ps, dYs, dUs, dSs, g, gam, bet, Dd, total;   // Ws: two buffers
 };
 __host__ __device__ inline StateSmem state_layout(int DK, int DVT)
 {
@@ -471,7 +559,7 @@ __host__ __device__ inline StateSmem state_layout(int DK, int DVT)
     const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
     L.Kt = o; o += DK * cp;
     L.Qg = o; o += kC * kq;
-    L.Wn = o; o += kC * kq;
+    L.Ws = o; o += 2 * kC * kq;
     L.Ps = o; o += kC * cp;
     L.dYs = o; o += kC * vq;
     L.dUs = o; o += kC * vq;
@@ -498,7 +586,7 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
     const StateSmem Y = state_layout(DK, DVT);
-    float *Kt = sm + Y.Kt, *Qg = sm + Y.Qg, *Wn = sm + Y.Wn, *Ps = sm + Y.Ps;
+    float *Kt = sm + Y.Kt, *Qg = sm + Y.Qg, *Ws = sm + Y.Ws, *Ps = sm + Y.Ps;
     float *dYs = sm + Y.dYs, *dUs = sm + Y.dUs, *dSs = sm + Y.dSs;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd;
     const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
@@ -514,11 +602,19 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     }
     const int n_chunks = (int)((len + kC - 1) / kC);
     const int nvq = DVT / 4;
+    // a chunk's W goes to buffer (c & 1) at the start of the chunk after it (in this reverse
+    // order), its P right after that chunk's dU~ product; the last chunk's here
+    auto cache_of = [&](int c) { return cache + ((size_t)chain * max_chunks + c) * cache_floats(DK); };
+    if (n_chunks > 0) {
+        copy_block_async(Ws + ((n_chunks - 1) & 1) * kC * kq, kq, cache_of(n_chunks - 1) + kCacheW, kC, DK);
+        copy_block_async(Ps, cp, cache_of(n_chunks - 1) + kCacheP, kC, kC);
+        cp_async_commit();
+    }
     for (int c = n_chunks - 1; c >= 0; --c) {
         int64_t c0;
         int n;
         chunk_of(cu_seqlens, seq, c, c0, n);
-        const float *cb = cache + ((size_t)chain * max_chunks + c) * cache_floats(DK);
+        const float *Wc = Ws + (c & 1) * kC * kq;
         __syncthreads();
         {
             float *dst = dS_chunks + ((size_t)chain * max_chunks + c) * DK * DV + v0;
@@ -527,12 +623,22 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                 st4(dst + (size_t)a * DV + b, f4(dSs + a * vq + b));
             }
         }
-        load_rows_t(Kt, cp, k, c0, n, H, h, DK, DK);
-        load_rows(Qg, kq, q, c0, n, H, h, DK, 0, DK, scale);
-        load_rows(dYs, vq, dy, c0, n, H, h, DV, v0, DVT, 1.f);
-        load_block(Wn, kq, cb + kCacheW, kC, DK, -1.f);
-        load_block(Ps, cp, cb + kCacheP, kC, kC, 1.f);
-        if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+        // the chunk's K, Q and dY rows into registers, all loads in flight together, and the
+        // decays on warp 0 (W and P are on their way)
+        {
+            float4 kr[kC * 128 / 4 / kThreadsWide], qr[kC * 128 / 4 / kThreadsWide];
+            float4 yr[kC * kDVT / 4 / kThreadsWide];
+            fetch_rows<true>(kr, k, c0, n, H, h, DK, 0, DK);
+            fetch_rows<false>(qr, q, c0, n, H, h, DK, 0, DK);
+            fetch_rows<false>(yr, dy, c0, n, H, h, DV, v0, DVT);
+            if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+            put_rows<true>(Kt, cp, kr, DK);
+#pragma unroll
+            for (int r = 0; r < kC * 128 / 4 / kThreadsWide; ++r) qr[r] = scale4(qr[r], scale);
+            put_rows<false>(Qg, kq, qr, DK);
+            put_rows<false>(dYs, vq, yr, DVT);
+        }
+        cp_async_wait_all();
         __syncthreads();
         for (int i = tid; i < DK * kC / 4; i += blockDim.x) {
             const int a = i / (kC / 4), t = (i % (kC / 4)) * 4;
@@ -543,6 +649,10 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
             st4(Qg + t * kq + a, scale4(f4(Qg + t * kq + a), gam[t]));
         }
+        if (c > 0) {                                   // the other W buffer is free
+            copy_block_async(Ws + ((c - 1) & 1) * kC * kq, kq, cache_of(c - 1) + kCacheW, kC, DK);
+            cp_async_commit();
+        }
         __syncthreads();
         // dU~ = P^T dY + diag(D) K dS': A(s, t) = P[t][s] and A(s, a) = Kd^T[a][s], both [k][m]
         for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
@@ -552,6 +662,10 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             w.each([&](int s, int b, float v0_, float v1_) { st2(dUs + s * vq + b, v0_, v1_); });
         }
         __syncthreads();
+        if (c > 0) {                                   // P is free: the next chunk's
+            copy_block_async(Ps, cp, cache_of(c - 1) + kCacheP, kC, kC);
+            cp_async_commit();
+        }
         // dS = gamma_C dS' + (diag(gamma) Q)^T dY - W^T dU~ (each warp: its own entries of dS)
         const float gamC = gam[kC - 1];
         for (int tile = warp; tile < (DK / 16) * (DVT / 16); tile += n_warps) {
@@ -560,8 +674,13 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                 const float2 x = *reinterpret_cast<const float2 *>(dSs + a * vq + b);
                 return make_float2(gamC * x.x, gamC * x.y);
             });
+            WTile<false, true> wd(tile, DVT);
             w.run(kC, Qg, kq, dYs, vq);
-            w.run(kC, Wn, kq, dUs, vq);
+            wd.run(kC, Wc, kq, dUs, vq);
+#pragma unroll
+            for (int f = 0; f < 2; ++f)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w.c[f][e] -= wd.c[f][e];
             w.each([&](int a, int b, float v0_, float v1_) { st2(dSs + a * vq + b, v0_, v1_); });
         }
     }

@@ -50,6 +50,23 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v)
     *reinterpret_cast<uint2 *>(p) = raw;
 }
 
+// ---- asynchronous global -> shared copies (cp.async; completion per thread by group) ------
+__device__ __forceinline__ uint32_t cvta_shared(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(cvta_shared(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(cvta_shared(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Sum over groups of G consecutive lanes (G a power of two <= 32); every lane of the
 // group receives the total.
 template <int G> __device__ __forceinline__ float group_sum(float x)
