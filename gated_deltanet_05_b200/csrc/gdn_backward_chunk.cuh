@@ -104,6 +104,32 @@ __device__ __forceinline__ void st2(float *p, float a, float b) { *reinterpret_c
 __device__ __forceinline__ float4 scale4(float4 v, float f) { return make_float4(v.x * f, v.y * f, v.z * f, v.w * f); }
 __device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
 
+// The same from the chunk's log alpha and beta already in shared memory (la, be; n valid).
+__device__ __forceinline__ void chunk_decays_smem(const float *la_s, const float *be_s, int n, float *g, float *gam,
+                                                  float *bet, float *Dd)
+{
+    const int lane = threadIdx.x;
+    float carry = 0.f;
+#pragma unroll
+    for (int j = 0; j < kC / 32; ++j) {
+        const int t = 32 * j + lane;
+        float x = t < n ? la_s[t] : 0.f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y_ = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y_;
+        }
+        x += carry;
+        carry = __shfl_sync(0xffffffffu, x, 31);
+        g[t] = x;
+        gam[t] = expf(x);
+        bet[t] = t < n ? be_s[t] : 0.f;
+    }
+    __syncwarp();
+    const float gC = g[kC - 1];
+    for (int t = lane; t < kC; t += 32) Dd[t] = expf(gC - g[t]);
+}
+
 // Columns [col0, col0 + ncol) of a chunk's rows of a token-major [.., H, D] tensor into shared
 // memory [kC][ld] (zero past n), times f. ncol, col0 and D multiples of 4.
 template <typename T>
@@ -429,9 +455,10 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
 
 // --------------------------------------------------------------------------- fwd
 struct FwdSmem {
-    int Kd, Ws, Ts, Vb, Us, Ss, g, gam, bet, Dd, total;
+    int Kd, Ws, Ts, Vb, Us, Ss, Kraw, Vraw, las, bes, g, gam, bet, Dd, total;
 };
-__host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT)
+// esize: bytes per input element (the raw K and V rows of the next chunk wait in Kraw, Vraw)
+__host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT, int esize)
 {
     FwdSmem L;
     int o = 0;
@@ -442,6 +469,10 @@ __host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT)
     L.Vb = o; o += kC * vq;
     L.Us = o; o += kC * vq;
     L.Ss = o; o += DK * vq;
+    L.Kraw = o; o += kC * DK * esize / 4;
+    L.Vraw = o; o += kC * DVT * esize / 4;
+    L.las = o; o += kC;
+    L.bes = o; o += kC;
     L.g = o; o += kC;
     L.gam = o; o += kC;
     L.bet = o; o += kC;
@@ -452,7 +483,9 @@ __host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT)
 
 // One CTA (kThreadsWide) per (chain, d_v slice): the forward's state chain from S0
 // (value-major [DV][DK] or NULL) with the cached T and W, keeping the start state of every
-// chunk in S_chunks [chain][max_chunks][DK][DV] (the pages' orientation).
+// chunk in S_chunks [chain][max_chunks][DK][DV] (the pages' orientation). Every input of chunk
+// c + 1 is requested by cp.async while chunk c is computed: its raw K and V rows and gates
+// once chunk c's have been converted, its T and W once chunk c's U~ product is done.
 template <typename T>
 __global__ void __launch_bounds__(kThreadsWide)
 chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ log_alpha,
@@ -462,10 +495,13 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
 {
     extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
-    const FwdSmem Y = fwd_layout(DK, DVT);
+    const FwdSmem Y = fwd_layout(DK, DVT, (int)sizeof(T));
     float *Kd = sm + Y.Kd, *Ws = sm + Y.Ws, *Ts = sm + Y.Ts, *Vb = sm + Y.Vb, *Us = sm + Y.Us, *Ss = sm + Y.Ss;
+    T *Kraw = reinterpret_cast<T *>(sm + Y.Kraw), *Vraw = reinterpret_cast<T *>(sm + Y.Vraw);
+    float *las = sm + Y.las, *bes = sm + Y.bes;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd;
     const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
+    constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte piece
     const int n_vt = DV / DVT;
     const int chain = blockIdx.x / n_vt, v0 = (blockIdx.x % n_vt) * DVT;
     const int seq = chain / H, h = chain % H;
@@ -478,15 +514,35 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
     }
     const int n_chunks = (int)((len + kC - 1) / kC);
     const int nvq = DVT / 4;
-    // T and W of a chunk are requested as soon as the buffers are free: chunk 0's here, chunk
-    // c + 1's right after chunk c's U~ product
     auto request_tw = [&](int c) {
         const float *cb = cache + ((size_t)chain * max_chunks + c) * cache_floats(DK);
         copy_block_async(Ts, cp, cb + kCacheT, kC, kC);
         copy_block_async(Ws, kq, cb + kCacheW, kC, DK);
         cp_async_commit();
     };
-    if (n_chunks > 0) request_tw(0);
+    auto request_rows = [&](int c) {                  // rows past the sequence end are not copied
+        int64_t cc0;
+        int nn;
+        chunk_of(cu_seqlens, seq, c, cc0, nn);
+        const int pk = DK / EPC, pv = DVT / EPC;
+        for (int i = tid; i < nn * pk; i += blockDim.x) {
+            const int t = i / pk, w = i % pk;
+            cp_async16(Kraw + t * DK + w * EPC, k + ((size_t)(cc0 + t) * H + h) * DK + w * EPC);
+        }
+        for (int i = tid; i < nn * pv; i += blockDim.x) {
+            const int t = i / pv, w = i % pv;
+            cp_async16(Vraw + t * DVT + w * EPC, v + ((size_t)(cc0 + t) * H + h) * DV + v0 + w * EPC);
+        }
+        for (int i = tid; i < 2 * nn; i += blockDim.x) {
+            const int t = i >> 1;
+            cp_async4((i & 1) ? bes + t : las + t, ((i & 1) ? beta : log_alpha) + (size_t)(cc0 + t) * H + h);
+        }
+        cp_async_commit();
+    };
+    if (n_chunks > 0) {
+        request_tw(0);
+        request_rows(0);
+    }
     for (int c = 0; c < n_chunks; ++c) {
         int64_t c0;
         int n;
@@ -499,27 +555,21 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
                 st4(dst + (size_t)a * DV + b, f4(Ss + a * vq + b));
             }
         }
-        // the chunk's K and V rows into registers, all loads in flight together, and the
-        // decays on warp 0 (T and W are on their way)
-        {
-            float4 kr[kC * 128 / 4 / kThreadsWide], vr[kC * kDVT / 4 / kThreadsWide];
-            fetch_rows<false>(kr, k, c0, n, H, h, DK, 0, DK);
-            fetch_rows<false>(vr, v, c0, n, H, h, DV, v0, DVT);
-            if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-            put_rows<false>(Kd, kq, kr, DK);
-            put_rows<false>(Vb, vq, vr, DVT);
-        }
-        cp_async_wait_all();
+        cp_async_wait_all();                           // this chunk's inputs have landed
         __syncthreads();
+        if (tid < 32) chunk_decays_smem(las, bes, n, g, gam, bet, Dd);
+        __syncthreads();
+        // diag(D) K and diag(beta) V in fp32 (zero past n)
         for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
             const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
-            st4(Kd + t * kq + a, scale4(f4(Kd + t * kq + a), Dd[t]));
+            st4(Kd + t * kq + a, t < n ? scale4(load4(Kraw + t * DK + a), Dd[t]) : make_float4(0.f, 0.f, 0.f, 0.f));
         }
         for (int i = tid; i < kC * nvq; i += blockDim.x) {
             const int t = i / nvq, b = (i % nvq) * 4;
-            st4(Vb + t * vq + b, scale4(f4(Vb + t * vq + b), bet[t]));
+            st4(Vb + t * vq + b, t < n ? scale4(load4(Vraw + t * DVT + b), bet[t]) : make_float4(0.f, 0.f, 0.f, 0.f));
         }
         __syncthreads();
+        if (c + 1 < n_chunks) request_rows(c + 1);    // the raw rows and gates are free
         // U~ = T diag(beta) V - W S
         for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
             WTile<true, true> w(tile, DVT), ws(tile, DVT);
@@ -546,6 +596,7 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
             w.each([&](int a, int b, float v0_, float v1_) { st2(Ss + a * vq + b, v0_, v1_); });
         }
     }
+    cp_async_wait_all();
 }
 
 // --------------------------------------------------------------------------- state
