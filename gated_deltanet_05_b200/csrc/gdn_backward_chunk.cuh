@@ -801,18 +801,27 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
     const float *cb = cache + cidx * cache_floats(DK);
     const float *Sg = S_chunks + cidx * DK * DV + v0, *dSg = dS_chunks + cidx * DK * DV + v0;
     const int nvq = DVT / 4;
-#pragma unroll 4
+    // every load in flight together: the states and the cache blocks by cp.async, the K, V and
+    // dY rows into registers, the decays on warp 0
     for (int i = tid; i < DK * nvq; i += blockDim.x) {
         const int a = i / nvq, b = (i % nvq) * 4;
-        st4(Ss + a * vq + b, f4(Sg + (size_t)a * DV + b));
-        st4(dSs + a * vq + b, f4(dSg + (size_t)a * DV + b));
+        cp_async16(Ss + a * vq + b, Sg + (size_t)a * DV + b);
+        cp_async16(dSs + a * vq + b, dSg + (size_t)a * DV + b);
     }
-    load_rows_t(Kt, cp, k, c0, n, H, h, DK, DK);
-    load_rows(Vs, vq, v, c0, n, H, h, DV, v0, DVT, 1.f);
-    load_rows(dYs, vq, dy, c0, n, H, h, DV, v0, DVT, 1.f);
-    load_block(Ts, cp, cb + kCacheT, kC, kC, 1.f);
-    load_block(Ps, cp, cb + kCacheP, kC, kC, 1.f);
-    if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+    copy_block_async(Ts, cp, cb + kCacheT, kC, kC);
+    copy_block_async(Ps, cp, cb + kCacheP, kC, kC);
+    cp_async_commit();
+    {
+        float4 kr[kC * 128 / 4 / kThreadsWide], vr[kC * kDVT / 4 / kThreadsWide], yr[kC * kDVT / 4 / kThreadsWide];
+        fetch_rows<true>(kr, k, c0, n, H, h, DK, 0, DK);
+        fetch_rows<false>(vr, v, c0, n, H, h, DV, v0, DVT);
+        fetch_rows<false>(yr, dy, c0, n, H, h, DV, v0, DVT);
+        if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+        put_rows<true>(Kt, cp, kr, DK);
+        put_rows<false>(Vs, vq, vr, DVT);
+        put_rows<false>(dYs, vq, yr, DVT);
+    }
+    cp_async_wait_all();
     __syncthreads();
     float *P = parts + (cidx * n_vt + vt) * part_floats(DK);
     float *PdP = P, *PdT = P + kC * kC, *PdW = P + 2 * kC * kC, *PdKd = PdW + kC * DK, *PdYS = PdKd + kC * DK;
