@@ -382,10 +382,18 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
     int n;
     if (!chunk_of(cu_seqlens, seq, c, c0, n)) return;
     float *cb = cache + ((size_t)chain * max_chunks + c) * cache_floats(DK);
-    load_rows(KQ, kq, k, c0, n, H, h, DK, 0, DK, 1.f);
-    load_rows(KQ + kC * kq, kq, q, c0, n, H, h, DK, 0, DK, scale);
-    if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-    for (int i = tid; i < kC * kC; i += blockDim.x) Ts[(i / kC) * cp + i % kC] = (i / kC == i % kC) ? 1.f : 0.f;
+    {
+        // the K and Q rows in flight together, stored once the identity and the decays are done
+        float4 kr[kC * 128 / 4 / kThreads], qr[kC * 128 / 4 / kThreads];
+        fetch_rows<false>(kr, k, c0, n, H, h, DK, 0, DK);
+        fetch_rows<false>(qr, q, c0, n, H, h, DK, 0, DK);
+        for (int i = tid; i < kC * kC; i += blockDim.x) Ts[(i / kC) * cp + i % kC] = (i / kC == i % kC) ? 1.f : 0.f;
+        if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+#pragma unroll
+        for (int r = 0; r < kC * 128 / 4 / kThreads; ++r) qr[r] = scale4(qr[r], scale);
+        put_rows<false>(KQ, kq, kr, DK);
+        put_rows<false>(KQ + kC * kq, kq, qr, DK);
+    }
     __syncthreads();
     // [K; Q] K^T: A = KQ [m][a], B(a, s) = K[s][a] stored [n][k]
     for (int tile = warp; tile < (2 * kC / 16) * (kC / 16); tile += n_warps) {
@@ -972,22 +980,60 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         return acc;
     };
 
-    load_rows(Ks, kq, k, c0, n, H, h, DK, 0, DK, 1.f);
-    load_rows(Qs, kq, q, c0, n, H, h, DK, 0, DK, scale);
-    load_block(Ts, cp, cb + kCacheT, kC, kC, 1.f);
-    if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-#pragma unroll 4
-    for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
-        const int r = i / (DK / 4), a = (i % (DK / 4)) * 4;
-        st4(PdWs + r * kq + a, sum_slices4(oW + (size_t)r * DK + a));
+    // every load in flight together: T by cp.async; the K and Q rows and the slice sums
+    // (P dW, and dT into dGs and dP into G1) in registers; the decays on warp 0
+    copy_block_async(Ts, cp, cb + kCacheT, kC, kC);
+    cp_async_commit();
+    {
+        constexpr int RR = kC * 128 / 4 / kThreadsWide, RW = kC * 128 / 4 / kThreadsWide, RT = kC * kC / 4 / kThreadsWide;
+        float4 kr[RR], qr[RR], wr[RW], tr[RT], pr[RT];
+        fetch_rows<false>(kr, k, c0, n, H, h, DK, 0, DK);
+        fetch_rows<false>(qr, q, c0, n, H, h, DK, 0, DK);
+        const int nwq = kC * DK / 4;
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int i = tid + r * kThreadsWide;
+            const size_t off = oW + (size_t)(i / (DK / 4)) * DK + (i % (DK / 4)) * 4;
+            wr[r] = i < nwq ? f4(P0 + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int i = tid + r * kThreadsWide;
+            tr[r] = f4(P0 + oT + 4 * (size_t)i);
+            pr[r] = f4(P0 + oP + 4 * (size_t)i);
+        }
+        for (int j = 1; j < n_vt; ++j) {
+            const float *Pj = P0 + j * pf;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const int i = tid + r * kThreadsWide;
+                if (i < nwq) wr[r] = add4(wr[r], f4(Pj + oW + (size_t)(i / (DK / 4)) * DK + (i % (DK / 4)) * 4));
+            }
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+                const int i = tid + r * kThreadsWide;
+                tr[r] = add4(tr[r], f4(Pj + oT + 4 * (size_t)i));
+                pr[r] = add4(pr[r], f4(Pj + oP + 4 * (size_t)i));
+            }
+        }
+        if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+#pragma unroll
+        for (int r = 0; r < RR; ++r) qr[r] = scale4(qr[r], scale);
+        put_rows<false>(Ks, kq, kr, DK);
+        put_rows<false>(Qs, kq, qr, DK);
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int i = tid + r * kThreadsWide;
+            if (i < nwq) st4(PdWs + (i / (DK / 4)) * kq + (i % (DK / 4)) * 4, wr[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int i = tid + r * kThreadsWide, t = i / (kC / 4), s = (i % (kC / 4)) * 4;
+            st4(dGs + t * cp + s, tr[r]);
+            st4(G1 + t * cp + s, pr[r]);
+        }
     }
-    // dT into dGs and dP into G1, summed over the slices
-#pragma unroll 4
-    for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
-        const int t = i / (kC / 4), s = (i % (kC / 4)) * 4;
-        st4(dGs + t * cp + s, sum_slices4(oT + (size_t)t * kC + s));
-        st4(G1 + t * cp + s, sum_slices4(oP + (size_t)t * kC + s));
-    }
+    cp_async_wait_all();
     __syncthreads();
     const int n_cc = (kC / 16) * (kC / 16);
     // M = dT T^T into Asym (B(r, s) = T[s][r]: stored [n][k])
