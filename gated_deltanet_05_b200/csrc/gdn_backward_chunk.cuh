@@ -240,17 +240,19 @@ __device__ __forceinline__ void load_block(float *dst, int ld, const float *__re
 
 // ---- tensor-core products from shared memory --------------------------------------------
 // C[M][N] += A[M][K] B[K][N] on mma.sync m16n8k8 tiles in tf32. Each operand is split as
-// x = hi + lo with hi = tf32(x) and lo = tf32(x - hi), and A B is taken as
-// lo_A hi_B + hi_A lo_B + hi_A hi_B: the dropped lo_A lo_B and the rounding of lo leave an
-// error of order 2^-21 |A| |B|, that of an fp32 product; accumulation is fp32.
+// x = hi + lo with hi = x with its 13 low mantissa bits cleared (a tf32 value) and lo = x - hi
+// (exact in fp32; the tensor core reads only its top 19 bits), and A B is taken as
+// lo_A hi_B + hi_A lo_B + hi_A hi_B. |lo| < 2^-10 |x|, so the dropped lo_A lo_B and the bits of
+// lo the tensor core does not read leave an error below about 3 * 2^-20 |A| |B| per term:
+// fp32-level products, with fp32 accumulation.
 // A(m, k) = AMK ? A[m lda + k] : A[k lda + m];  B(k, n) = BKN ? B[k ldb + n] : B[n ldb + k].
 // A warp owns the 16 x 16 block `tile` of C (tiles numbered row-major over N / 16 columns):
 // with g = lane / 4, q = lane % 4, its elements (f, e) (fragment f = 0, 1; e = 0..3) sit at
 // row m0 + g + 8 (e / 2), column n0 + 8 f + 2 q + e % 2. M, N multiples of 16, K of 8.
 __device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
 {
-    hi = sm100::to_tf32(x);
-    lo = sm100::to_tf32(x - __uint_as_float(hi));
+    hi = __float_as_uint(x) & 0xffffe000u;
+    lo = __float_as_uint(x - __uint_as_float(hi));
 }
 
 __device__ __forceinline__ void mma8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
@@ -783,7 +785,7 @@ __host__ __device__ inline VpartSmem vpart_layout(int DK, int DVT)
 // of the sums over v, written to the slice's block of the sums buffer
 // [chain][max_chunks][n_slices][part_floats].
 template <typename T>
-__global__ void __launch_bounds__(kThreadsWide)
+__global__ void __launch_bounds__(kThreadsWide, 1)
 chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ dy,
                        const float *__restrict__ log_alpha, const float *__restrict__ beta,
                        const int32_t *__restrict__ cu_seqlens, int H, int DK, int DV, int max_chunks,
