@@ -15,7 +15,8 @@
 //     dP = dY U~^T,  dT = dU~ Z^T,  dW = -dU~ S^T,  dK~ = U~ dS'^T,  dV = diag(beta) T^T dU~
 //     dQ = diag(gamma) dY S^T + (dP o Gamma) K
 //     dK = (dP o Gamma)^T Q + diag(beta gamma) T^T dW + (dA + dA^T) K + diag(D) dK~
-//     dL = strict_tril(-T^T dT T^T),  dA = diag(beta) (dL o Gamma)
+//     dL = strict_tril(-T^T dT T^T) = strict_tril(-(T^T dU~) U~^T)  (as T Z = U~),
+//     dA = diag(beta) (dL o Gamma)
 //     dbeta = rowsum(V o T^T dU~) + gamma o rowsum(K o T^T dW) + rowsum(dL o A o Gamma)
 // and the decays gamma, Gamma, D fold into d g, then into d log alpha by a reverse
 // cumulative sum inside the chunk. (The same algebra is restated in fp64 and pinned to the
@@ -24,13 +25,14 @@
 // Five launches:
 //   chunk_bwd_prep_kernel   per (chain, chunk), all at once: T, A o Gamma, P and W of the
 //                           chunk, kept in the workspace (all that does not depend on the state)
-//   chunk_bwd_fwd_kernel    per (chain, d_v slice), chunks in order: the start state of every
-//                           chunk (the forward's state chain)
-//   chunk_bwd_state_kernel  per (chain, d_v slice), chunks in reverse: dS at every chunk end,
-//                           and dS0
+//   chunk_bwd_fwd_kernel    per (chain, d_v slice), chunks in order: the start state and U~ of
+//                           every chunk (the forward's state chain)
+//   chunk_bwd_state_kernel  per (chain, d_v slice), chunks in reverse: dS at every chunk end and
+//                           dU~ of every chunk, and dS0
 //   chunk_bwd_vpart_kernel  per (chain, chunk, d_v slice), all at once: dV, and the slice's
-//                           sums over v that the rest needs (dP, dT, dW, dK~, dY S^T, ...), each
-//                           slice into its own block (no atomics: the result is deterministic)
+//                           sums over v that the rest needs (dP, T^T dT T^T, dW, dK~, dY S^T,
+//                           ...), each slice into its own block (no atomics: the result is
+//                           deterministic)
 //   chunk_bwd_kpart_kernel  per (chain, chunk), all at once: dQ, dK, dbeta, dlog_alpha
 // Every matrix product runs from shared memory on the tensor cores (mma.sync m16n8k8, tf32)
 // with each operand split into two tf32 parts, which keeps fp32 accuracy; a warp owns a
@@ -49,10 +51,14 @@ constexpr int kThreads = 256;        // prep
 constexpr int kThreadsWide = 512;    // fwd, state, vpart and kpart
 
 __host__ __device__ inline int slice_cols(int DV) { return DV < kDVT ? DV : kDVT; }
+// bf16 inputs converted to fp32 without scaling are tf32 values (8 significant bits <= 11):
+// products with such an operand need no split of it
+template <typename T>
+__host__ __device__ constexpr bool exact_tf32() { return sizeof(T) == 2; }
 // shared-memory row stride for rows of D floats (D a multiple of 16): 16-byte aligned rows,
 // and rows g = 0..7 of a fragment load start on distinct banks
 __host__ __device__ inline int ldp(int D) { return D + 4; }
-// floats of the per-chunk sums block of one value slice: dP, dT [C][C]; dW, dK~, dY S^T
+// floats of the per-chunk sums block of one value slice: dP, T^T dT T^T [C][C]; dW, dK~, dY S^T
 // [C][DK]; the row sums of V o T^T dU~ [C]; <dS', S> [1]; rounded up to a multiple of 4
 __host__ __device__ inline size_t part_floats(int DK)
 {
@@ -303,6 +309,10 @@ struct WTile {
                 c[f][2 * h + 1] = v.y;
             }
     }
+    // EXA / EXB: every entry of A / B is a tf32 value already (its lo part is zero: bf16
+    // inputs converted to fp32 unscaled), so that operand is not split and its lo product is
+    // skipped
+    template <bool EXA = false, bool EXB = false>
     __device__ __forceinline__ void run(int K, const float *__restrict__ A, int lda, const float *__restrict__ B,
                                         int ldb)
     {
@@ -312,19 +322,27 @@ struct WTile {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int m = m0 + g + 8 * (e & 1), kk = k + q + 4 * (e >> 1);
-                split_tf32(AMK ? A[m * lda + kk] : A[kk * lda + m], ah[e], al[e]);
+                const float x = AMK ? A[m * lda + kk] : A[kk * lda + m];
+                if (EXA)
+                    ah[e] = __float_as_uint(x);
+                else
+                    split_tf32(x, ah[e], al[e]);
             }
 #pragma unroll
             for (int f = 0; f < 2; ++f)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int kk = k + q + 4 * e, nn = n0 + 8 * f + g;
-                    split_tf32(BKN ? B[kk * ldb + nn] : B[nn * ldb + kk], bh[f][e], bl[f][e]);
+                    const float x = BKN ? B[kk * ldb + nn] : B[nn * ldb + kk];
+                    if (EXB)
+                        bh[f][e] = __float_as_uint(x);
+                    else
+                        split_tf32(x, bh[f][e], bl[f][e]);
                 }
 #pragma unroll
             for (int f = 0; f < 2; ++f) {
-                mma8(c[f], al, bh[f][0], bh[f][1]);
-                mma8(c[f], ah, bl[f][0], bl[f][1]);
+                if (!EXA) mma8(c[f], al, bh[f][0], bh[f][1]);
+                if (!EXB) mma8(c[f], ah, bl[f][0], bl[f][1]);
                 mma8(c[f], ah, bh[f][0], bh[f][1]);
             }
         }
@@ -391,20 +409,20 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
         fetch_rows<false>(qr, q, c0, n, H, h, DK, 0, DK);
         for (int i = tid; i < kC * kC; i += blockDim.x) Ts[(i / kC) * cp + i % kC] = (i / kC == i % kC) ? 1.f : 0.f;
         if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-#pragma unroll
-        for (int r = 0; r < kC * 128 / 4 / kThreads; ++r) qr[r] = scale4(qr[r], scale);
         put_rows<false>(KQ, kq, kr, DK);
         put_rows<false>(KQ + kC * kq, kq, qr, DK);
     }
     __syncthreads();
-    // [K; Q] K^T: A = KQ [m][a], B(a, s) = K[s][a] stored [n][k]
+    // [K; Q] K^T: A = KQ [m][a], B(a, s) = K[s][a] stored [n][k]; Q is unscaled here (the
+    // scale goes to the Q rows of the result)
     for (int tile = warp; tile < (2 * kC / 16) * (kC / 16); tile += n_warps) {
         WTile<true, false> w(tile, kC);
-        w.run(DK, KQ, kq, KQ, kq);
+        w.template run<exact_tf32<T>(), exact_tf32<T>()>(DK, KQ, kq, KQ, kq);
         w.each([&](int m, int s, float v0, float v1) {
             const int t = m & (kC - 1);
-            const float x0 = s <= t ? v0 * expf(g[t] - g[s]) : 0.f;
-            const float x1 = s + 1 <= t ? v1 * expf(g[t] - g[s + 1]) : 0.f;
+            const float f = m < kC ? 1.f : scale;
+            const float x0 = s <= t ? f * v0 * expf(g[t] - g[s]) : 0.f;
+            const float x1 = s + 1 <= t ? f * v1 * expf(g[t] - g[s + 1]) : 0.f;
             if (m < kC) {
                 st2(cb + kCacheAG + t * kC + s, x0, x1);
                 Ls[t * cp + s] = s < t ? bet[t] * x0 : 0.f;
@@ -493,7 +511,8 @@ __host__ __device__ inline FwdSmem fwd_layout(int DK, int DVT, int esize)
 
 // One CTA (kThreadsWide) per (chain, d_v slice): the forward's state chain from S0
 // (value-major [DV][DK] or NULL) with the cached T and W, keeping the start state of every
-// chunk in S_chunks [chain][max_chunks][DK][DV] (the pages' orientation). Every input of chunk
+// chunk in S_chunks [chain][max_chunks][DK][DV] (the pages' orientation) and every chunk's
+// U~ in Ut_chunks [chain][max_chunks][C][DV]. Every input of chunk
 // c + 1 is requested by cp.async while chunk c is computed: its raw K and V rows and gates
 // once chunk c's have been converted, its T and W once chunk c's U~ product is done.
 template <typename T>
@@ -501,7 +520,7 @@ __global__ void __launch_bounds__(kThreadsWide)
 chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ log_alpha,
                      const float *__restrict__ beta, const float *__restrict__ S0,
                      const int32_t *__restrict__ cu_seqlens, int H, int DK, int DV, int max_chunks,
-                     const float *__restrict__ cache, float *__restrict__ S_chunks)
+                     const float *__restrict__ cache, float *__restrict__ S_chunks, float *__restrict__ Ut_chunks)
 {
     extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
@@ -569,31 +588,43 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
         __syncthreads();
         if (tid < 32) chunk_decays_smem(las, bes, n, g, gam, bet, Dd);
         __syncthreads();
-        // diag(D) K and diag(beta) V in fp32 (zero past n)
+        // K and V in fp32, unscaled (zero past n), so that bf16 inputs stay exact tf32
+        // operands; T diag(beta) in place (its columns scaled)
         for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
             const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
-            st4(Kd + t * kq + a, t < n ? scale4(load4(Kraw + t * DK + a), Dd[t]) : make_float4(0.f, 0.f, 0.f, 0.f));
+            st4(Kd + t * kq + a, t < n ? load4(Kraw + t * DK + a) : make_float4(0.f, 0.f, 0.f, 0.f));
         }
         for (int i = tid; i < kC * nvq; i += blockDim.x) {
             const int t = i / nvq, b = (i % nvq) * 4;
-            st4(Vb + t * vq + b, t < n ? scale4(load4(Vraw + t * DVT + b), bet[t]) : make_float4(0.f, 0.f, 0.f, 0.f));
+            st4(Vb + t * vq + b, t < n ? load4(Vraw + t * DVT + b) : make_float4(0.f, 0.f, 0.f, 0.f));
+        }
+        for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
+            const int t = i / (kC / 4), s4 = (i % (kC / 4)) * 4;
+            const float4 x = f4(Ts + t * cp + s4);
+            st4(Ts + t * cp + s4, make_float4(x.x * bet[s4], x.y * bet[s4 + 1], x.z * bet[s4 + 2], x.w * bet[s4 + 3]));
         }
         __syncthreads();
         if (c + 1 < n_chunks) request_rows(c + 1);    // the raw rows and gates are free
-        // U~ = T diag(beta) V - W S
-        for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
-            WTile<true, true> w(tile, DVT), ws(tile, DVT);
-            w.run(kC, Ts, cp, Vb, vq);
-            ws.run(DK, Ws, kq, Ss, vq);
+        // U~ = (T diag(beta)) V - W S, to Ut_chunks; diag(D) U~ into Us for the state update
+        {
+            float *dst = Ut_chunks + ((size_t)chain * max_chunks + c) * kC * DV + v0;
+            for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
+                WTile<true, true> w(tile, DVT), ws(tile, DVT);
+                w.template run<false, exact_tf32<T>()>(kC, Ts, cp, Vb, vq);
+                ws.run(DK, Ws, kq, Ss, vq);
 #pragma unroll
-            for (int f = 0; f < 2; ++f)
+                for (int f = 0; f < 2; ++f)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) w.c[f][e] -= ws.c[f][e];
-            w.each([&](int t, int b, float v0_, float v1_) { st2(Us + t * vq + b, v0_, v1_); });
+                    for (int e = 0; e < 4; ++e) w.c[f][e] -= ws.c[f][e];
+                w.each([&](int t, int b, float v0_, float v1_) {
+                    st2(dst + (size_t)t * DV + b, v0_, v1_);
+                    st2(Us + t * vq + b, Dd[t] * v0_, Dd[t] * v1_);
+                });
+            }
         }
         __syncthreads();
         if (c + 1 < n_chunks) request_tw(c + 1);     // T and W are free: the next chunk's
-        // S <- gamma_C S + (diag(D) K)^T U~: A(a, s) = Kd[s][a] stored [k][m]; each warp reads
+        // S <- gamma_C S + K^T (diag(D) U~): A(a, s) = K[s][a] stored [k][m]; each warp reads
         // and writes only its own entries of S
         const float gamC = gam[kC - 1];
         for (int tile = warp; tile < (DK / 16) * (DVT / 16); tile += n_warps) {
@@ -602,7 +633,7 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
                 const float2 x = *reinterpret_cast<const float2 *>(Ss + a * vq + b);
                 return make_float2(gamC * x.x, gamC * x.y);
             });
-            w.run(kC, Kd, kq, Us, vq);
+            w.template run<exact_tf32<T>(), false>(kC, Kd, kq, Us, vq);
             w.each([&](int a, int b, float v0_, float v1_) { st2(Ss + a * vq + b, v0_, v1_); });
         }
     }
@@ -635,14 +666,15 @@ __host__ __device__ inline StateSmem state_layout(int DK, int DVT)
 
 // One CTA (kThreadsWide) per (chain, d_v slice): dS from dS_T back through the chunks with
 // the cached W and P; dS at the end of every chunk goes to dS_chunks
-// [chain][max_chunks][DK][DV], the final one to dS0 (value-major [DV][DK]).
+// [chain][max_chunks][DK][DV] and every chunk's dU~ to dUt_chunks [chain][max_chunks][C][DV],
+// the final dS to dS0 (value-major [DV][DK]).
 template <typename T>
 __global__ void __launch_bounds__(kThreadsWide)
 chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ dy,
                        const float *__restrict__ log_alpha, const float *__restrict__ beta,
                        const int32_t *__restrict__ cu_seqlens, int H, int DK, int DV, float scale,
                        const float *__restrict__ dS_T, int max_chunks, const float *__restrict__ cache,
-                       float *__restrict__ dS_chunks, float *__restrict__ dS0)
+                       float *__restrict__ dS_chunks, float *__restrict__ dUt_chunks, float *__restrict__ dS0)
 {
     extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
@@ -701,11 +733,6 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         }
         cp_async_wait_all();
         __syncthreads();
-        for (int i = tid; i < DK * kC / 4; i += blockDim.x) {
-            const int a = i / (kC / 4), t = (i % (kC / 4)) * 4;
-            const float4 x = f4(Kt + a * cp + t);
-            st4(Kt + a * cp + t, make_float4(x.x * Dd[t], x.y * Dd[t + 1], x.z * Dd[t + 2], x.w * Dd[t + 3]));
-        }
         for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
             const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
             st4(Qg + t * kq + a, scale4(f4(Qg + t * kq + a), gam[t]));
@@ -715,12 +742,20 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             cp_async_commit();
         }
         __syncthreads();
-        // dU~ = P^T dY + diag(D) K dS': A(s, t) = P[t][s] and A(s, a) = Kd^T[a][s], both [k][m]
+        // dU~ = P^T dY + diag(D) K dS': A(s, t) = P[t][s] and A(s, a) = K^T[a][s], both [k][m]
+        // (K and dY unscaled, so that bf16 inputs stay exact tf32 operands)
         for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
-            WTile<false, true> w(tile, DVT);
-            w.run(kC, Ps, cp, dYs, vq);
-            w.run(DK, Kt, cp, dSs, vq);
-            w.each([&](int s, int b, float v0_, float v1_) { st2(dUs + s * vq + b, v0_, v1_); });
+            WTile<false, true> w(tile, DVT), kd(tile, DVT);
+            w.template run<false, exact_tf32<T>()>(kC, Ps, cp, dYs, vq);
+            kd.template run<exact_tf32<T>(), false>(DK, Kt, cp, dSs, vq);
+#pragma unroll
+            for (int f = 0; f < 2; ++f)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int s_ = w.row(hh), b = w.col(f);
+                    st2(dUs + s_ * vq + b, fmaf(Dd[s_], kd.c[f][2 * hh], w.c[f][2 * hh]),
+                        fmaf(Dd[s_], kd.c[f][2 * hh + 1], w.c[f][2 * hh + 1]));
+                }
         }
         __syncthreads();
         if (c > 0) {                                   // P is free: the next chunk's
@@ -736,13 +771,20 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                 return make_float2(gamC * x.x, gamC * x.y);
             });
             WTile<false, true> wd(tile, DVT);
-            w.run(kC, Qg, kq, dYs, vq);
+            w.template run<false, exact_tf32<T>()>(kC, Qg, kq, dYs, vq);
             wd.run(kC, Wc, kq, dUs, vq);
 #pragma unroll
             for (int f = 0; f < 2; ++f)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) w.c[f][e] -= wd.c[f][e];
             w.each([&](int a, int b, float v0_, float v1_) { st2(dSs + a * vq + b, v0_, v1_); });
+        }
+        {
+            float *dst = dUt_chunks + ((size_t)chain * max_chunks + c) * kC * DV + v0;
+            for (int i = tid; i < kC * nvq; i += blockDim.x) {
+                const int t = i / nvq, b = (i % nvq) * 4;
+                st4(dst + (size_t)t * DV + b, f4(dUs + t * vq + b));
+            }
         }
     }
     __syncthreads();
@@ -755,27 +797,22 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
 
 // --------------------------------------------------------------------------- vpart
 struct VpartSmem {
-    int Kt, Ts, Ps, Ss, dSs, Vs, dYs, Uts, dUs, Zs, g, gam, bet, Dd, red, total;
+    int Ts, Ss, dSs, Vs, dYs, Uts, dUs, Xs, bet, red, total;
 };
 __host__ __device__ inline VpartSmem vpart_layout(int DK, int DVT)
 {
     VpartSmem L;
     int o = 0;
     const int vq = ldp(DVT), cp = ldp(kC);
-    L.Kt = o; o += DK * cp;
     L.Ts = o; o += kC * cp;
-    L.Ps = o; o += kC * cp;
     L.Ss = o; o += DK * vq;
     L.dSs = o; o += DK * vq;
     L.Vs = o; o += kC * vq;
     L.dYs = o; o += kC * vq;
     L.Uts = o; o += kC * vq;
     L.dUs = o; o += kC * vq;
-    L.Zs = o; o += kC * vq;
-    L.g = o; o += kC;
-    L.gam = o; o += kC;
+    L.Xs = o; o += kC * vq;
     L.bet = o; o += kC;
-    L.Dd = o; o += kC;
     L.red = o; o += kThreadsWide / 32;
     L.total = o;
     return L;
@@ -783,21 +820,22 @@ __host__ __device__ inline VpartSmem vpart_layout(int DK, int DVT)
 
 // One CTA (kThreadsWide) per (chain, chunk, d_v slice): dV of the slice, and the slice's share
 // of the sums over v, written to the slice's block of the sums buffer
-// [chain][max_chunks][n_slices][part_floats].
+// [chain][max_chunks][n_slices][part_floats]. U~ and dU~ come from the state chains
+// (Ut_chunks, dUt_chunks [chain][max_chunks][C][DV]); with X = T^T dU~ the slice's terms are
+// dV = diag(beta) X, rowsum(V o X), dY U~^T, X U~^T, -dU~ S^T, U~ dS'^T, dY S^T and <dS', S>.
 template <typename T>
 __global__ void __launch_bounds__(kThreadsWide, 1)
-chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ dy,
-                       const float *__restrict__ log_alpha, const float *__restrict__ beta,
+chunk_bwd_vpart_kernel(const T *__restrict__ v, const T *__restrict__ dy, const float *__restrict__ beta,
                        const int32_t *__restrict__ cu_seqlens, int H, int DK, int DV, int max_chunks,
                        const float *__restrict__ cache, const float *__restrict__ S_chunks,
-                       const float *__restrict__ dS_chunks, float *__restrict__ parts, float *__restrict__ dv_out)
+                       const float *__restrict__ dS_chunks, const float *__restrict__ Ut_chunks,
+                       const float *__restrict__ dUt_chunks, float *__restrict__ parts, float *__restrict__ dv_out)
 {
     extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
     const VpartSmem Y = vpart_layout(DK, DVT);
-    float *Kt = sm + Y.Kt, *Ts = sm + Y.Ts, *Ps = sm + Y.Ps, *Ss = sm + Y.Ss, *dSs = sm + Y.dSs;
-    float *Vs = sm + Y.Vs, *dYs = sm + Y.dYs, *Uts = sm + Y.Uts, *dUs = sm + Y.dUs, *Zs = sm + Y.Zs;
-    float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd, *red = sm + Y.red;
+    float *Ts = sm + Y.Ts, *Ss = sm + Y.Ss, *dSs = sm + Y.dSs, *Vs = sm + Y.Vs, *dYs = sm + Y.dYs;
+    float *Uts = sm + Y.Uts, *dUs = sm + Y.dUs, *Xs = sm + Y.Xs, *bet = sm + Y.bet, *red = sm + Y.red;
     const int vq = ldp(DVT), cp = ldp(kC);
     const int n_vt = DV / DVT;
     const int c = blockIdx.y;
@@ -810,24 +848,27 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
     const size_t cidx = (size_t)chain * max_chunks + c;
     const float *cb = cache + cidx * cache_floats(DK);
     const float *Sg = S_chunks + cidx * DK * DV + v0, *dSg = dS_chunks + cidx * DK * DV + v0;
+    const float *Ug = Ut_chunks + cidx * kC * DV + v0, *dUg = dUt_chunks + cidx * kC * DV + v0;
     const int nvq = DVT / 4;
-    // every load in flight together: the states and the cache blocks by cp.async, the K, V and
-    // dY rows into registers, the decays on warp 0
+    // every load in flight together: the states, U~, dU~ and T by cp.async, the V and dY rows
+    // into registers
     for (int i = tid; i < DK * nvq; i += blockDim.x) {
         const int a = i / nvq, b = (i % nvq) * 4;
         cp_async16(Ss + a * vq + b, Sg + (size_t)a * DV + b);
         cp_async16(dSs + a * vq + b, dSg + (size_t)a * DV + b);
     }
+    for (int i = tid; i < kC * nvq; i += blockDim.x) {
+        const int t = i / nvq, b = (i % nvq) * 4;
+        cp_async16(Uts + t * vq + b, Ug + (size_t)t * DV + b);
+        cp_async16(dUs + t * vq + b, dUg + (size_t)t * DV + b);
+    }
     copy_block_async(Ts, cp, cb + kCacheT, kC, kC);
-    copy_block_async(Ps, cp, cb + kCacheP, kC, kC);
     cp_async_commit();
     {
-        float4 kr[kC * 128 / 4 / kThreadsWide], vr[kC * kDVT / 4 / kThreadsWide], yr[kC * kDVT / 4 / kThreadsWide];
-        fetch_rows<true>(kr, k, c0, n, H, h, DK, 0, DK);
+        float4 vr[kC * kDVT / 4 / kThreadsWide], yr[kC * kDVT / 4 / kThreadsWide];
         fetch_rows<false>(vr, v, c0, n, H, h, DV, v0, DVT);
         fetch_rows<false>(yr, dy, c0, n, H, h, DV, v0, DVT);
-        if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-        put_rows<true>(Kt, cp, kr, DK);
+        if (tid < kC) bet[tid] = tid < n ? beta[(size_t)(c0 + tid) * H + h] : 0.f;
         put_rows<false>(Vs, vq, vr, DVT);
         put_rows<false>(dYs, vq, yr, DVT);
     }
@@ -837,54 +878,29 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
     float *PdP = P, *PdT = P + kC * kC, *PdW = P + 2 * kC * kC, *PdKd = PdW + kC * DK, *PdYS = PdKd + kC * DK;
     float *Pvs = PdYS + kC * DK, *PdgC = Pvs + kC;
     const int n_tv = (kC / 16) * (DVT / 16);
-    // Z = diag(beta) (V - diag(gamma) K S);  dU~ = P^T dY + diag(D) K dS'
-    // (A(t, a) = K[t][a] = Kt[a][t] and A(s, t) = P[t][s], both stored [k][m])
-    for (int tile = warp; tile < n_tv; tile += n_warps) {
-        WTile<false, true> ks(tile, DVT), kd(tile, DVT), pd(tile, DVT);
-        ks.run(DK, Kt, cp, Ss, vq);
-        kd.run(DK, Kt, cp, dSs, vq);
-        pd.run(kC, Ps, cp, dYs, vq);
-#pragma unroll
-        for (int f = 0; f < 2; ++f)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = ks.row(e >> 1), b = ks.col(f) + (e & 1);
-                Zs[t * vq + b] = bet[t] * (Vs[t * vq + b] - gam[t] * ks.c[f][e]);
-                dUs[t * vq + b] = fmaf(Dd[t], kd.c[f][e], pd.c[f][e]);
-            }
-    }
-    __syncthreads();
-    // U~ = T Z (A = T [t][s])
-    for (int tile = warp; tile < n_tv; tile += n_warps) {
-        WTile<true, true> w(tile, DVT);
-        w.run(kC, Ts, cp, Zs, vq);
-        w.each([&](int t, int b, float v0_, float v1_) { st2(Uts + t * vq + b, v0_, v1_); });
-    }
-    // T^T dU~ (A(t, s) = T[s][t], stored [k][m]): dV = diag(beta) T^T dU~, and V o T^T dU~
-    // into Ps (P is no longer needed) for its row sums
+    // X = T^T dU~ (A(t, s) = T[s][t], stored [k][m]) into Xs; dV = diag(beta) X
     for (int tile = warp; tile < n_tv; tile += n_warps) {
         WTile<false, true> w(tile, DVT);
         w.run(kC, Ts, cp, dUs, vq);
         w.each([&](int t, int b, float w0, float w1) {
             if (t < n) st2(dv_out + ((size_t)(c0 + t) * H + h) * DV + v0 + b, bet[t] * w0, bet[t] * w1);
-            Ps[t * cp + b] = Vs[t * vq + b] * w0;
-            Ps[t * cp + b + 1] = Vs[t * vq + b + 1] * w1;
+            st2(Xs + t * vq + b, w0, w1);
         });
     }
     __syncthreads();
-    // row sums of V o T^T dU~: eight lanes per row
+    // row sums of V o X: eight lanes per row
     for (int r = tid; r < kC * 8; r += blockDim.x) {
         const int t = r >> 3, part = r & 7;
         float acc = 0.f;
-        for (int b = part; b < DVT; b += 8) acc += Ps[t * cp + b];
+        for (int b = part; b < DVT; b += 8) acc = fmaf(Vs[t * vq + b], Xs[t * vq + b], acc);
         acc = group_sum<8>(acc);
         if (part == 0) Pvs[t] = acc;
     }
-    // this slice's dY U~^T and dU~ Z^T [C][C] (B(b, s) = U~[s][b], Z[s][b]: stored [n][k])
+    // this slice's dY U~^T and X U~^T [C][C] (B(b, s) = U~[s][b]: stored [n][k])
     for (int tile = warp; tile < (kC / 16) * (kC / 16); tile += n_warps) {
         WTile<true, false> p(tile, kC), tt(tile, kC);
-        p.run(DVT, dYs, vq, Uts, vq);
-        tt.run(DVT, dUs, vq, Zs, vq);
+        p.template run<exact_tf32<T>(), false>(DVT, dYs, vq, Uts, vq);
+        tt.run(DVT, Xs, vq, Uts, vq);
         p.each([&](int t, int s, float v0_, float v1_) { st2(PdP + t * kC + s, v0_, v1_); });
         tt.each([&](int t, int s, float v0_, float v1_) { st2(PdT + t * kC + s, v0_, v1_); });
     }
@@ -893,7 +909,7 @@ chunk_bwd_vpart_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
         WTile<true, false> w(tile, DK), kd(tile, DK), ys(tile, DK);
         w.run(DVT, dUs, vq, Ss, vq);
         kd.run(DVT, Uts, vq, dSs, vq);
-        ys.run(DVT, dYs, vq, Ss, vq);
+        ys.template run<exact_tf32<T>(), false>(DVT, dYs, vq, Ss, vq);
         w.each([&](int t, int a, float v0_, float v1_) { st2(PdW + t * DK + a, -v0_, -v1_); });
         kd.each([&](int t, int a, float v0_, float v1_) { st2(PdKd + t * DK + a, v0_, v1_); });
         ys.each([&](int t, int a, float v0_, float v1_) { st2(PdYS + t * DK + a, v0_, v1_); });
@@ -983,7 +999,7 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
     };
 
     // every load in flight together: T by cp.async; the K and Q rows and the slice sums
-    // (P dW, and dT into dGs and dP into G1) in registers; the decays on warp 0
+    // (P dW, and T^T dT T^T, as dL, into dGs and dP into G1) in registers; the decays on warp 0
     copy_block_async(Ts, cp, cb + kCacheT, kC, kC);
     cp_async_commit();
     {
@@ -1030,29 +1046,14 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         }
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
+            // dL = strict_tril(-T^T dT T^T), the slices' sums of X U~^T
             const int i = tid + r * kThreadsWide, t = i / (kC / 4), s = (i % (kC / 4)) * 4;
-            st4(dGs + t * cp + s, tr[r]);
+            st4(dGs + t * cp + s, make_float4(s < t ? -tr[r].x : 0.f, s + 1 < t ? -tr[r].y : 0.f,
+                                              s + 2 < t ? -tr[r].z : 0.f, s + 3 < t ? -tr[r].w : 0.f));
             st4(G1 + t * cp + s, pr[r]);
         }
     }
     cp_async_wait_all();
-    __syncthreads();
-    const int n_cc = (kC / 16) * (kC / 16);
-    // M = dT T^T into Asym (B(r, s) = T[s][r]: stored [n][k])
-    for (int tile = warp; tile < n_cc; tile += n_warps) {
-        WTile<true, false> w(tile, kC);
-        w.run(kC, dGs, cp, Ts, cp);
-        w.each([&](int t, int s, float v0, float v1) { st2(Asym + t * cp + s, v0, v1); });
-    }
-    __syncthreads();
-    // dL = strict_tril(-T^T M) into dGs (A(t, r) = T[r][t]: stored [k][m])
-    for (int tile = warp; tile < n_cc; tile += n_warps) {
-        WTile<false, true> w(tile, kC);
-        w.run(kC, Ts, cp, Asym, cp);
-        w.each([&](int t, int s, float v0, float v1) {
-            st2(dGs + t * cp + s, s < t ? -v0 : 0.f, s + 1 < t ? -v1 : 0.f);
-        });
-    }
     __syncthreads();
     // dA + dA^T with dA = diag(beta) (dL o Gamma), into Asym (symmetric)
     for (int i = tid; i < kC * kC; i += blockDim.x) {
@@ -1115,9 +1116,9 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
 #pragma unroll
     for (int r = 0; r < kMaxWT; ++r)
         if (warp + r * n_warps < n_ck) {
-            aq[r].run(kC, G1T, cp, Ks, kq);
+            aq[r].template run<false, exact_tf32<T>()>(kC, G1T, cp, Ks, kq);
             ak[r].run(kC, G1, cp, Qs, kq);
-            ak[r].run(kC, Asym, cp, Ks, kq);
+            ak[r].template run<false, exact_tf32<T>()>(kC, Asym, cp, Ks, kq);
         }
     __syncthreads();
     float *GQ = Ts, *GK = Ts + kC * kq;

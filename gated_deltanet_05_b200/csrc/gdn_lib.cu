@@ -406,10 +406,11 @@ size_t gdn_backward_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, i
     }
     const int64_t max_chunks = (max_len + gdn::bwdc::kC - 1) / gdn::bwdc::kC;
     const int n_vt = d_v / gdn::bwdc::slice_cols(d_v);
-    // per (chain, chunk): the start state and the end-state adjoint [d_k][d_v], the chunk's
-    // cache (T, A o Gamma, P, W), and one block of sums over v per value slice
-    const size_t per_chunk = 2 * (size_t)d_k * d_v + gdn::bwdc::cache_floats(d_k) +
-                             (size_t)n_vt * gdn::bwdc::part_floats(d_k);
+    // per (chain, chunk): the start state and the end-state adjoint [d_k][d_v], U~ and dU~
+    // [C][d_v], the chunk's cache (T, A o Gamma, P, W), and one block of sums over v per
+    // value slice
+    const size_t per_chunk = 2 * (size_t)d_k * d_v + 2 * (size_t)gdn::bwdc::kC * d_v +
+                             gdn::bwdc::cache_floats(d_k) + (size_t)n_vt * gdn::bwdc::part_floats(d_k);
     return (size_t)n_seq * H * (size_t)max_chunks * per_chunk * sizeof(float);
 }
 
@@ -463,7 +464,9 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
     const size_t n_cc = (size_t)n_chain * max_chunks;
     float *S_chunks = static_cast<float *>(workspace);
     float *dS_chunks = S_chunks + n_cc * d_k * d_v;
-    float *cache = dS_chunks + n_cc * d_k * d_v;
+    float *Ut_chunks = dS_chunks + n_cc * d_k * d_v;
+    float *dUt_chunks = Ut_chunks + n_cc * kC * d_v;
+    float *cache = dUt_chunks + n_cc * kC * d_v;
     float *parts = cache + n_cc * cache_floats(d_k);
     const int smem_p = (int)(prep_layout(d_k).total * sizeof(float));
     const int smem_f = (int)(fwd_layout(d_k, dvt, in_dtype == GDN_F32 ? 4 : 2).total * sizeof(float));
@@ -492,13 +495,13 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
         kp<<<grid_c, kThreads, smem_p, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
                                              scale, (int)max_chunks, cache);                        \
         kf<<<grid_s, kThreadsWide, smem_f, st>>>((const T *)k, (const T *)v, log_alpha, beta, S0, cu_seqlens_dev, \
-                                                 H, d_k, d_v, (int)max_chunks, cache, S_chunks);    \
+                                                 H, d_k, d_v, (int)max_chunks, cache, S_chunks, Ut_chunks); \
         ks<<<grid_s, kThreadsWide, smem_s, st>>>((const T *)q, (const T *)k, (const T *)dy, log_alpha, beta,     \
                                                  cu_seqlens_dev, H, d_k, d_v, scale, dS_T, (int)max_chunks,     \
-                                                 cache, dS_chunks, dS0);                            \
-        kv<<<grid_v, kThreadsWide, smem_v, st>>>((const T *)k, (const T *)v, (const T *)dy, log_alpha, beta,     \
-                                                 cu_seqlens_dev, H, d_k, d_v, (int)max_chunks, cache, S_chunks, \
-                                                 dS_chunks, parts, dv);                             \
+                                                 cache, dS_chunks, dUt_chunks, dS0);                \
+        kv<<<grid_v, kThreadsWide, smem_v, st>>>((const T *)v, (const T *)dy, beta, cu_seqlens_dev, H, d_k, d_v, \
+                                                 (int)max_chunks, cache, S_chunks, dS_chunks, Ut_chunks,        \
+                                                 dUt_chunks, parts, dv);                            \
         kk<<<grid_c, kThreadsWide, smem_k, st>>>((const T *)q, (const T *)k, log_alpha, beta, cu_seqlens_dev, H, d_k, \
                                              n_vt, scale, (int)max_chunks, cache, parts, dq, dk, dbeta,  \
                                              dlog_alpha);                                           \

@@ -191,17 +191,18 @@ gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_
  *   dS0    [n_seq, H, d_v, d_k] fp32 out, or NULL
  *   workspace: gdn_backward_workspace_bytes(...) bytes, 16-byte aligned: per (chain, chunk
  *          of 64 tokens) the chunk's start state and the adjoint of its end state
- *          (d_k x d_v each), the chunk's cache of state-free matrices (3 x 64 x 64 + 64 x d_k
- *          floats: T, A o Gamma, P, W) and, per slice of min(d_v, 64) value columns, one
- *          block of the chunk's sums over v (2 x 64 x 64 + 3 x 64 x d_k + 64 + 1 floats,
- *          rounded up to a multiple of 4);
+ *          (d_k x d_v each), its U~ and dU~ (64 x d_v each), the chunk's cache of state-free
+ *          matrices (3 x 64 x 64 + 64 x d_k floats: T, A o Gamma, P, W) and, per slice of
+ *          min(d_v, 64) value columns, one block of the chunk's sums over v
+ *          (2 x 64 x 64 + 3 x 64 x d_k + 64 + 1 floats, rounded up to a multiple of 4);
  *          n_seq * H * ceil(max_len / 64) chunks are provided for
  *   d_k, d_v in {16, 32, 64, 128}
- * The chain rule through the chunked form, fp32 on CUDA cores, five launches: the
+ * The chain rule through the chunked form, five launches, every matrix product on the
+ * tensor cores with fp32-level accuracy (each operand split into two tf32 parts): the
  * state-free matrices of every chunk at once; a forward pass over the chunks of each
- * (chain, value slice) keeping each chunk's start state; a reverse pass for the state
- * adjoints; then, for every chunk of every chain at once, dv and the per-slice sums over v,
- * and dq, dk, dbeta, dlog_alpha. Deterministic (no atomics).
+ * (chain, value slice) keeping each chunk's start state and U~; a reverse pass for the state
+ * adjoints and dU~; then, for every chunk of every chain at once, dv and the per-slice sums
+ * over v, and dq, dk, dbeta, dlog_alpha. Deterministic (no atomics).
  */
 size_t gdn_backward_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, int H, int d_k,
                                     int d_v);

@@ -125,12 +125,12 @@ def test_decode_and_gate_norm_reject_bad_arguments(L):
 
 def test_backward_rejects_bad_arguments(L):
     cu = (ctypes.c_int32 * 3)(0, 64, 100)
-    # per (chain, 64-token chunk): two 128 x 128 states, the chunk's cache (3 x 64 x 64 +
-    # 64 x 128 floats), and two 64-column value slices' blocks of per-chunk sums
-    # (2 x 64 x 64 + 3 x 64 x 128 + 64 + 1 floats each)
+    # per (chain, 64-token chunk): two 128 x 128 states, U~ and dU~ (64 x 128 each), the
+    # chunk's cache (3 x 64 x 64 + 64 x 128 floats), and two 64-column value slices' blocks of
+    # per-chunk sums (2 x 64 x 64 + 3 x 64 x 128 + 64 + 1 floats each)
     part = (64 * (2 * 64 + 3 * 128 + 1) + 1 + 3) // 4 * 4      # rounded up to a multiple of 4
     assert L.gdn_backward_workspace_bytes(ctypes.cast(cu, ctypes.c_void_p), 2, 2, 128, 128) == \
-        2 * 2 * 1 * (2 * 128 * 128 + 64 * (3 * 64 + 128) + 2 * part) * 4
+        2 * 2 * 1 * (2 * 128 * 128 + 2 * 64 * 128 + 64 * (3 * 64 + 128) + 2 * part) * 4
     assert L.gdn_backward_workspace_bytes(None, 2, 2, 128, 128) == 0
 
     def bw(**kw):

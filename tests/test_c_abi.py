@@ -19,9 +19,11 @@ int main(void)
     int32_t cu[3] = {0, 64, 100};
     if (gdn_version() <= 0) return 1;
     if (strcmp(gdn_status_string(GDN_ERR_TIMEOUT), "GDN_ERR_TIMEOUT") != 0) return 2;
-    /* one 64-token chunk per chain: two 16 x 16 states, the chunk's cache and one block of sums */
+    /* one 64-token chunk per chain: two 16 x 16 states, U~ and dU~ (64 x 16), the chunk's
+       cache and one block of sums */
     if (gdn_backward_workspace_bytes(cu, 2, 2, 16, 16) !=
-        (size_t)2 * 2 * 1 * (2 * 16 * 16 + 64 * (3 * 64 + 16) + (64 * (2 * 64 + 3 * 16 + 1) + 1 + 3) / 4 * 4) * 4) return 3;
+        (size_t)2 * 2 * 1 * (2 * 16 * 16 + 2 * 64 * 16 + 64 * (3 * 64 + 16) + (64 * (2 * 64 + 3 * 16 + 1) + 1 + 3) / 4 * 4) * 4)
+        return 3;
     /* rejected before any launch: an unsupported head size, an unknown dtype */
     if (gdn_decode_step(0, 0, 0, GDN_F32, 0, 0, 0, 1, 1, 48, 16, 1.f, 0, GDN_F32, 0) != GDN_ERR_UNSUPPORTED) return 4;
     if (gdn_gate_norm(0, (gdn_dtype)7, 0, GDN_F32, 0, 4, 16, 1e-6f, 0, GDN_F32, 0) != GDN_ERR_INVALID_ARG) return 5;

@@ -8,6 +8,7 @@ with D_s = exp(g_C - g_s). Its reverse, given dY and dS', is the chain rule thro
 matrix products, in reverse order:
     dU~ = (Q K^T o Gamma)^T dY + diag(D) K dS';     dS = gamma_C dS' + (diag(gamma) Q)^T dY - W^T dU~
     dT = dU~ (diag(beta) V)^T - dU~ S^T (diag(beta gamma) K)^T;   dL = -T^T dT T^T (strictly lower)
+    (and T^T dT T^T = (T^T dU~) U~^T, because U~ = T (diag(beta) V - diag(beta gamma) K S))
 plus the terms of Q, K, V, beta and of gamma, Gamma and D, which become gradients of the
 in-chunk cumulative log decay g and, by a reverse cumulative sum, of log alpha. This is
 the algebra a chunked (tensor-core) backward would follow; the test pins it to the
@@ -88,8 +89,11 @@ def chunk_backward(q, k, v, la, b, cu, S0, dy, dS_T, C, scale=1.0):
                 db = np.sum(V * TdU, axis=1) + gam * np.sum(K * TdW, axis=1)
                 dK += (bb * gam)[:, None] * TdW
                 dgam += bb * np.sum(K * TdW, axis=1)
-                # T = (I + L)^-1
-                dL = np.tril(-T.T @ dT @ T.T, -1)
+                # T = (I + L)^-1; since U~ = T Z with Z = bV - bgK S and dT = dU~ Z^T, the
+                # product T^T dT T^T is (T^T dU~) U~^T, the form the kernels take
+                dL = np.tril(-TdU @ Ut.T, -1)
+                dL_full = np.tril(-T.T @ dT @ T.T, -1)
+                assert np.max(np.abs(dL - dL_full)) <= 1e-12 * max(1.0, np.max(np.abs(dL_full)))
                 # L = strict_tril(diag(b) (A o Gam))
                 db += np.sum(dL * A * Gam, axis=1)
                 dA = bb[:, None] * dL * Gam
