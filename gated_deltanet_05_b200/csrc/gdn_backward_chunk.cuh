@@ -464,19 +464,20 @@ chunk_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const fl
         }
         __syncthreads();
     }
+    // T to the cache, then T diag(beta gamma) in place (K stays unscaled: an exact operand
+    // for bf16 inputs)
     for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
         const int r = i / (kC / 4), c4 = (i % (kC / 4)) * 4;
-        st4(cb + kCacheT + r * kC + c4, f4(Ts + r * cp + c4));
-    }
-    for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
-        const int s = i / (DK / 4), a = (i % (DK / 4)) * 4;
-        st4(KQ + s * kq + a, scale4(f4(KQ + s * kq + a), bet[s] * gam[s]));
+        const float4 x = f4(Ts + r * cp + c4);
+        st4(cb + kCacheT + r * kC + c4, x);
+        st4(Ts + r * cp + c4, make_float4(x.x * bet[c4] * gam[c4], x.y * bet[c4 + 1] * gam[c4 + 1],
+                                          x.z * bet[c4 + 2] * gam[c4 + 2], x.w * bet[c4 + 3] * gam[c4 + 3]));
     }
     __syncthreads();
-    // W = T (diag(beta gamma) K): A = T [t][s], B = K scaled [s][a]
+    // W = (T diag(beta gamma)) K: A = [t][s], B = K [s][a]
     for (int tile = warp; tile < (kC / 16) * (DK / 16); tile += n_warps) {
         WTile<true, true> w(tile, DK);
-        w.run(kC, Ts, cp, KQ, kq);
+        w.template run<false, exact_tf32<T>()>(kC, Ts, cp, KQ, kq);
         w.each([&](int t, int a, float v0, float v1) { st2(cb + kCacheW + t * DK + a, v0, v1); });
     }
 }
@@ -1035,8 +1036,6 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
             }
         }
         if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-#pragma unroll
-        for (int r = 0; r < RR; ++r) qr[r] = scale4(qr[r], scale);
         put_rows<false>(Ks, kq, kr, DK);
         put_rows<false>(Qs, kq, qr, DK);
 #pragma unroll
@@ -1072,7 +1071,7 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         if (warp + r * n_warps < n_ck) tdw[r].run(kC, Ts, cp, PdWs, kq);
     __syncthreads();
     // per entry (same thread reads and writes it): dGamma o Gamma into dGs, dL o A o Gamma into
-    // Es, dP o Gamma into G1 and its transpose into G1T
+    // Es, scale (dP o Gamma) into G1 and the unscaled transpose into G1T
 #pragma unroll 2
     for (int i = tid; i < kC * kC / 4; i += blockDim.x) {
         const int t = i / (kC / 4), s0 = (i % (kC / 4)) * 4;
@@ -1092,7 +1091,8 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         }
         st4(dGs + t * cp + s0, make_float4(dgm[0], dgm[1], dgm[2], dgm[3]));
         st4(Es + t * cp + s0, make_float4(e[0], e[1], e[2], e[3]));
-        st4(G1 + t * cp + s0, make_float4(g1[0], g1[1], g1[2], g1[3]));
+        // scale (dP o Gamma) for the product with the unscaled Q
+        st4(G1 + t * cp + s0, make_float4(scale * g1[0], scale * g1[1], scale * g1[2], scale * g1[3]));
     }
 #pragma unroll
     for (int r = 0; r < kMaxWT; ++r)
@@ -1109,7 +1109,7 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         red[tid] = rs - cs;          // row sum - column sum of dGamma o Gamma
         red[kC + tid] = ab;          // row sum of dL o A o Gamma
     }
-    // (dP o Gamma) K and (dP o Gamma)^T Q + (dA + dA^T) K, in registers until the region
+    // (dP o Gamma) K and (dP o Gamma)^T (scale Q) + (dA + dA^T) K, in registers until the region
     // Ts .. Es is free (A(t, s) = G1[t][s] = G1T[s][t], G1[s][t] and Asym[s][t]: all [k][m])
     WTile<false, true> aq[kMaxWT] = {WTile<false, true>(warp, DK), WTile<false, true>(warp + n_warps, DK)};
     WTile<false, true> ak[kMaxWT] = {WTile<false, true>(warp, DK), WTile<false, true>(warp + n_warps, DK)};
@@ -1117,7 +1117,7 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
     for (int r = 0; r < kMaxWT; ++r)
         if (warp + r * n_warps < n_ck) {
             aq[r].template run<false, exact_tf32<T>()>(kC, G1T, cp, Ks, kq);
-            ak[r].run(kC, G1, cp, Qs, kq);
+            ak[r].template run<false, exact_tf32<T>()>(kC, G1, cp, Qs, kq);
             ak[r].template run<false, exact_tf32<T>()>(kC, Asym, cp, Ks, kq);
         }
     __syncthreads();
@@ -1159,7 +1159,7 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
         rb = group_sum<32>(rb);
         rd = group_sum<32>(rd);
         if (lane == 0) {
-            red[2 * kC + t] = rg + bet[t] * rb;     // dgamma_t
+            red[2 * kC + t] = scale * rg + bet[t] * rb;     // dgamma_t (Q unscaled in rg)
             red[3 * kC + t] = rb;                   // sum_a K o T^T dW
             red[4 * kC + t] = rd;                   // dD_t
         }
