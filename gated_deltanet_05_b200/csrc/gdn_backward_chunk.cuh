@@ -643,20 +643,28 @@ chunk_bwd_fwd_kernel(const T *__restrict__ k, const T *__restrict__ v, const flo
 
 // --------------------------------------------------------------------------- state
 struct StateSmem {
-    int Kt, Qg, Ws, Ps, dYs, dUs, dSs, g, gam, bet, Dd, total;   // Ws: two buffers
+    int Ks, Qg, Ws, Ps, dYs, dUs, dSs, Kraw, Qraw, Yraw, las, bes, g, gam, bet, Dd, total;
 };
-__host__ __device__ inline StateSmem state_layout(int DK, int DVT)
+// esize: bytes per input element of the raw K, Q and dY rows of the next chunk (bf16 inputs,
+// requested while the current chunk computes); 0 for fp32 inputs, whose rows are loaded at the
+// start of their own chunk (a second fp32 copy does not fit)
+__host__ __device__ inline StateSmem state_layout(int DK, int DVT, int esize)
 {
     StateSmem L;
     int o = 0;
     const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
-    L.Kt = o; o += DK * cp;
+    L.Ks = o; o += kC * kq;
     L.Qg = o; o += kC * kq;
-    L.Ws = o; o += 2 * kC * kq;
+    L.Ws = o; o += kC * kq;
     L.Ps = o; o += kC * cp;
     L.dYs = o; o += kC * vq;
     L.dUs = o; o += kC * vq;
     L.dSs = o; o += DK * vq;
+    L.Kraw = o; o += kC * DK * esize / 4;
+    L.Qraw = o; o += kC * DK * esize / 4;
+    L.Yraw = o; o += kC * DVT * esize / 4;
+    L.las = o; o += kC;
+    L.bes = o; o += kC;
     L.g = o; o += kC;
     L.gam = o; o += kC;
     L.bet = o; o += kC;
@@ -664,26 +672,35 @@ __host__ __device__ inline StateSmem state_layout(int DK, int DVT)
     L.total = o;
     return L;
 }
+template <typename T>
+__host__ __device__ constexpr bool state_prefetch() { return sizeof(T) == 2; }
 
 // One CTA (kThreadsWide) per (chain, d_v slice): dS from dS_T back through the chunks with
 // the cached W and P; dS at the end of every chunk goes to dS_chunks
 // [chain][max_chunks][DK][DV] and every chunk's dU~ to dUt_chunks [chain][max_chunks][C][DV],
-// the final dS to dS0 (value-major [DV][DK]).
+// the final dS to dS0 (value-major [DV][DK]). Three cp.async groups per chunk c, in this
+// order: W_c (at its start), the raw rows and gates of chunk c - 1 (bf16 inputs; empty
+// otherwise) once chunk c's are converted, and P_{c-1} once chunk c's dU~ product is done.
 template <typename T>
-__global__ void __launch_bounds__(kThreadsWide)
+__global__ void __launch_bounds__(kThreadsWide, 1)
 chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ dy,
                        const float *__restrict__ log_alpha, const float *__restrict__ beta,
                        const int32_t *__restrict__ cu_seqlens, int H, int DK, int DV, float scale,
                        const float *__restrict__ dS_T, int max_chunks, const float *__restrict__ cache,
                        float *__restrict__ dS_chunks, float *__restrict__ dUt_chunks, float *__restrict__ dS0)
 {
+    constexpr bool kPre = state_prefetch<T>();
     extern __shared__ __align__(16) float sm[];
     const int DVT = slice_cols(DV);
-    const StateSmem Y = state_layout(DK, DVT);
-    float *Kt = sm + Y.Kt, *Qg = sm + Y.Qg, *Ws = sm + Y.Ws, *Ps = sm + Y.Ps;
+    const StateSmem Y = state_layout(DK, DVT, kPre ? (int)sizeof(T) : 0);
+    float *Ks = sm + Y.Ks, *Qg = sm + Y.Qg, *Ws = sm + Y.Ws, *Ps = sm + Y.Ps;
     float *dYs = sm + Y.dYs, *dUs = sm + Y.dUs, *dSs = sm + Y.dSs;
+    T *Kraw = reinterpret_cast<T *>(sm + Y.Kraw), *Qraw = reinterpret_cast<T *>(sm + Y.Qraw);
+    T *Yraw = reinterpret_cast<T *>(sm + Y.Yraw);
+    float *las = sm + Y.las, *bes = sm + Y.bes;
     float *g = sm + Y.g, *gam = sm + Y.gam, *bet = sm + Y.bet, *Dd = sm + Y.Dd;
     const int kq = ldp(DK), vq = ldp(DVT), cp = ldp(kC);
+    constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte piece
     const int n_vt = DV / DVT;
     const int chain = blockIdx.x / n_vt, v0 = (blockIdx.x % n_vt) * DVT;
     const int seq = chain / H, h = chain % H;
@@ -696,11 +713,30 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     }
     const int n_chunks = (int)((len + kC - 1) / kC);
     const int nvq = DVT / 4;
-    // a chunk's W goes to buffer (c & 1) at the start of the chunk after it (in this reverse
-    // order), its P right after that chunk's dU~ product; the last chunk's here
     auto cache_of = [&](int c) { return cache + ((size_t)chain * max_chunks + c) * cache_floats(DK); };
+    auto request_rows = [&](int c) {                  // rows past the sequence end are not copied
+        int64_t cc0;
+        int nn;
+        chunk_of(cu_seqlens, seq, c, cc0, nn);
+        const int pk = DK / EPC, py = DVT / EPC;
+        for (int i = tid; i < nn * pk; i += blockDim.x) {
+            const int t = i / pk, w = i % pk;
+            const size_t off = ((size_t)(cc0 + t) * H + h) * DK + w * EPC;
+            cp_async16(Kraw + t * DK + w * EPC, k + off);
+            cp_async16(Qraw + t * DK + w * EPC, q + off);
+        }
+        for (int i = tid; i < nn * py; i += blockDim.x) {
+            const int t = i / py, w = i % py;
+            cp_async16(Yraw + t * DVT + w * EPC, dy + ((size_t)(cc0 + t) * H + h) * DV + v0 + w * EPC);
+        }
+        for (int i = tid; i < 2 * nn; i += blockDim.x) {
+            const int t = i >> 1;
+            cp_async4((i & 1) ? bes + t : las + t, ((i & 1) ? beta : log_alpha) + (size_t)(cc0 + t) * H + h);
+        }
+    };
     if (n_chunks > 0) {
-        copy_block_async(Ws + ((n_chunks - 1) & 1) * kC * kq, kq, cache_of(n_chunks - 1) + kCacheW, kC, DK);
+        if constexpr (kPre) request_rows(n_chunks - 1);
+        cp_async_commit();
         copy_block_async(Ps, cp, cache_of(n_chunks - 1) + kCacheP, kC, kC);
         cp_async_commit();
     }
@@ -708,8 +744,9 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         int64_t c0;
         int n;
         chunk_of(cu_seqlens, seq, c, c0, n);
-        const float *Wc = Ws + (c & 1) * kC * kq;
-        __syncthreads();
+        __syncthreads();                               // chunk c + 1's products are done
+        copy_block_async(Ws, kq, cache_of(c) + kCacheW, kC, DK);
+        cp_async_commit();
         {
             float *dst = dS_chunks + ((size_t)chain * max_chunks + c) * DK * DV + v0;
             for (int i = tid; i < DK * nvq; i += blockDim.x) {
@@ -717,38 +754,54 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                 st4(dst + (size_t)a * DV + b, f4(dSs + a * vq + b));
             }
         }
-        // the chunk's K, Q and dY rows into registers, all loads in flight together, and the
-        // decays on warp 0 (W and P are on their way)
-        {
-            float4 kr[kC * 128 / 4 / kThreadsWide], qr[kC * 128 / 4 / kThreadsWide];
-            float4 yr[kC * kDVT / 4 / kThreadsWide];
-            fetch_rows<true>(kr, k, c0, n, H, h, DK, 0, DK);
-            fetch_rows<false>(qr, q, c0, n, H, h, DK, 0, DK);
-            fetch_rows<false>(yr, dy, c0, n, H, h, DV, v0, DVT);
-            if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
-            put_rows<true>(Kt, cp, kr, DK);
-#pragma unroll
-            for (int r = 0; r < kC * 128 / 4 / kThreadsWide; ++r) qr[r] = scale4(qr[r], scale);
-            put_rows<false>(Qg, kq, qr, DK);
-            put_rows<false>(dYs, vq, yr, DVT);
+        if constexpr (kPre) {
+            cp_async_wait1();                          // chunk c's rows, gates and P have landed
+            __syncthreads();
+            if (tid < 32) chunk_decays_smem(las, bes, n, g, gam, bet, Dd);
+            __syncthreads();
+            // K, dY unscaled and diag(gamma) scale Q in fp32 (zero past n)
+            for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
+                const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
+                const bool in = t < n;
+                st4(Ks + t * kq + a, in ? load4(Kraw + t * DK + a) : make_float4(0.f, 0.f, 0.f, 0.f));
+                st4(Qg + t * kq + a, in ? scale4(load4(Qraw + t * DK + a), scale * gam[t]) : make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+            for (int i = tid; i < kC * nvq; i += blockDim.x) {
+                const int t = i / nvq, b = (i % nvq) * 4;
+                st4(dYs + t * vq + b, t < n ? load4(Yraw + t * DVT + b) : make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+            __syncthreads();
+            if (c > 0) request_rows(c - 1);            // the raw rows and gates are free
+        } else {
+            // the chunk's K, Q and dY rows into registers, all loads in flight together, and
+            // the decays on warp 0
+            {
+                float4 kr[kC * 128 / 4 / kThreadsWide], qr[kC * 128 / 4 / kThreadsWide];
+                float4 yr[kC * kDVT / 4 / kThreadsWide];
+                fetch_rows<false>(kr, k, c0, n, H, h, DK, 0, DK);
+                fetch_rows<false>(qr, q, c0, n, H, h, DK, 0, DK);
+                fetch_rows<false>(yr, dy, c0, n, H, h, DV, v0, DVT);
+                if (tid < 32) chunk_decays(log_alpha, beta, c0, n, H, h, g, gam, bet, Dd);
+                put_rows<false>(Ks, kq, kr, DK);
+                put_rows<false>(Qg, kq, qr, DK);
+                put_rows<false>(dYs, vq, yr, DVT);
+            }
+            cp_async_wait1();                          // P has landed
+            __syncthreads();
+            for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
+                const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
+                st4(Qg + t * kq + a, scale4(f4(Qg + t * kq + a), scale * gam[t]));
+            }
+            __syncthreads();
         }
-        cp_async_wait_all();
-        __syncthreads();
-        for (int i = tid; i < kC * DK / 4; i += blockDim.x) {
-            const int t = i / (DK / 4), a = (i % (DK / 4)) * 4;
-            st4(Qg + t * kq + a, scale4(f4(Qg + t * kq + a), gam[t]));
-        }
-        if (c > 0) {                                   // the other W buffer is free
-            copy_block_async(Ws + ((c - 1) & 1) * kC * kq, kq, cache_of(c - 1) + kCacheW, kC, DK);
-            cp_async_commit();
-        }
-        __syncthreads();
-        // dU~ = P^T dY + diag(D) K dS': A(s, t) = P[t][s] and A(s, a) = K^T[a][s], both [k][m]
+        cp_async_commit();                             // (empty without a prefetch)
+        // dU~ = P^T dY + diag(D) K dS': A(s, t) = P[t][s] stored [k][m], A(s, a) = K[s][a]
         // (K and dY unscaled, so that bf16 inputs stay exact tf32 operands)
         for (int tile = warp; tile < (kC / 16) * (DVT / 16); tile += n_warps) {
-            WTile<false, true> w(tile, DVT), kd(tile, DVT);
+            WTile<false, true> w(tile, DVT);
+            WTile<true, true> kd(tile, DVT);
             w.template run<false, exact_tf32<T>()>(kC, Ps, cp, dYs, vq);
-            kd.template run<exact_tf32<T>(), false>(DK, Kt, cp, dSs, vq);
+            kd.template run<exact_tf32<T>(), false>(DK, Ks, kq, dSs, vq);
 #pragma unroll
             for (int f = 0; f < 2; ++f)
 #pragma unroll
@@ -758,11 +811,10 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                         fmaf(Dd[s_], kd.c[f][2 * hh + 1], w.c[f][2 * hh + 1]));
                 }
         }
+        cp_async_wait1();                              // W_c has landed
         __syncthreads();
-        if (c > 0) {                                   // P is free: the next chunk's
-            copy_block_async(Ps, cp, cache_of(c - 1) + kCacheP, kC, kC);
-            cp_async_commit();
-        }
+        if (c > 0) copy_block_async(Ps, cp, cache_of(c - 1) + kCacheP, kC, kC);   // P is free
+        cp_async_commit();
         // dS = gamma_C dS' + (diag(gamma) Q)^T dY - W^T dU~ (each warp: its own entries of dS)
         const float gamC = gam[kC - 1];
         for (int tile = warp; tile < (DK / 16) * (DVT / 16); tile += n_warps) {
@@ -773,7 +825,7 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             });
             WTile<false, true> wd(tile, DVT);
             w.template run<false, exact_tf32<T>()>(kC, Qg, kq, dYs, vq);
-            wd.run(kC, Wc, kq, dUs, vq);
+            wd.run(kC, Ws, kq, dUs, vq);
 #pragma unroll
             for (int f = 0; f < 2; ++f)
 #pragma unroll
@@ -788,6 +840,7 @@ chunk_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             }
         }
     }
+    cp_async_wait_all();
     __syncthreads();
     if (dS0)
         for (int i = tid; i < DK * DVT; i += blockDim.x) {

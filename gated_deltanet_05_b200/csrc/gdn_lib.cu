@@ -470,7 +470,7 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, gdn_dtype i
     float *parts = cache + n_cc * cache_floats(d_k);
     const int smem_p = (int)(prep_layout(d_k).total * sizeof(float));
     const int smem_f = (int)(fwd_layout(d_k, dvt, in_dtype == GDN_F32 ? 4 : 2).total * sizeof(float));
-    const int smem_s = (int)(state_layout(d_k, dvt).total * sizeof(float));
+    const int smem_s = (int)(state_layout(d_k, dvt, in_dtype == GDN_BF16 ? 2 : 0).total * sizeof(float));
     const int smem_v = (int)(vpart_layout(d_k, dvt).total * sizeof(float));
     const int smem_k = (int)(kpart_layout(d_k).total * sizeof(float));
     const int optin = smem_optin();
