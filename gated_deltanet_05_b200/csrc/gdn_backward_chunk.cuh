@@ -41,6 +41,7 @@
 #pragma once
 #include "gdn_common.cuh"
 #include "sm100_ptx.cuh"
+#include <type_traits>
 
 namespace gdn {
 namespace bwdc {
@@ -348,6 +349,51 @@ struct WTile {
         }
     }
 };
+
+// Two products with one B and the same tile, C1 += A1 B and C2 += A2 B: B's fragments are
+// loaded and split once per k step for both.
+template <bool EXA1, bool EXA2, bool EXB, bool AMK, bool BKN>
+__device__ __forceinline__ void run2(WTile<AMK, BKN> &w1, WTile<AMK, BKN> &w2, int K, const float *__restrict__ A1,
+                                     const float *__restrict__ A2, int lda, const float *__restrict__ B, int ldb)
+{
+    const int m0 = w1.m0, n0 = w1.n0, g = w1.g, q = w1.q;
+#pragma unroll 2
+    for (int k = 0; k < K; k += 8) {
+        uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+        for (int f = 0; f < 2; ++f)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int kk = k + q + 4 * e, nn = n0 + 8 * f + g;
+                const float x = BKN ? B[kk * ldb + nn] : B[nn * ldb + kk];
+                if (EXB)
+                    bh[f][e] = __float_as_uint(x);
+                else
+                    split_tf32(x, bh[f][e], bl[f][e]);
+            }
+        auto one = [&](WTile<AMK, BKN> &w, const float *__restrict__ A, auto exa) {
+            constexpr bool EXA = decltype(exa)::value;
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int m = m0 + g + 8 * (e & 1), kk = k + q + 4 * (e >> 1);
+                const float x = AMK ? A[m * lda + kk] : A[kk * lda + m];
+                if (EXA)
+                    ah[e] = __float_as_uint(x);
+                else
+                    split_tf32(x, ah[e], al[e]);
+            }
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+                if (!EXA) mma8(w.c[f], al, bh[f][0], bh[f][1]);
+                if (!EXB) mma8(w.c[f], ah, bl[f][0], bl[f][1]);
+                mma8(w.c[f], ah, bh[f][0], bh[f][1]);
+            }
+        };
+        one(w1, A1, std::integral_constant<bool, EXA1>());
+        one(w2, A2, std::integral_constant<bool, EXA2>());
+    }
+}
 
 // Chunk geometry of (sequence seq, chunk c): first token and valid rows; false past the end.
 __device__ __forceinline__ bool chunk_of(const int32_t *__restrict__ cu_seqlens, int seq, int c, int64_t &c0, int &n)
@@ -953,17 +999,15 @@ chunk_bwd_vpart_kernel(const T *__restrict__ v, const T *__restrict__ dy, const 
     // this slice's dY U~^T and X U~^T [C][C] (B(b, s) = U~[s][b]: stored [n][k])
     for (int tile = warp; tile < (kC / 16) * (kC / 16); tile += n_warps) {
         WTile<true, false> p(tile, kC), tt(tile, kC);
-        p.template run<exact_tf32<T>(), false>(DVT, dYs, vq, Uts, vq);
-        tt.run(DVT, Xs, vq, Uts, vq);
+        run2<exact_tf32<T>(), false, false>(p, tt, DVT, dYs, Xs, vq, Uts, vq);
         p.each([&](int t, int s, float v0_, float v1_) { st2(PdP + t * kC + s, v0_, v1_); });
         tt.each([&](int t, int s, float v0_, float v1_) { st2(PdT + t * kC + s, v0_, v1_); });
     }
     // this slice's -dU~ S^T, U~ dS'^T and dY S^T [C][DK] (B(b, a) = S[a][b]: stored [n][k])
     for (int tile = warp; tile < (kC / 16) * (DK / 16); tile += n_warps) {
         WTile<true, false> w(tile, DK), kd(tile, DK), ys(tile, DK);
-        w.run(DVT, dUs, vq, Ss, vq);
+        run2<false, exact_tf32<T>(), false>(w, ys, DVT, dUs, dYs, vq, Ss, vq);
         kd.run(DVT, Uts, vq, dSs, vq);
-        ys.template run<exact_tf32<T>(), false>(DVT, dYs, vq, Ss, vq);
         w.each([&](int t, int a, float v0_, float v1_) { st2(PdW + t * DK + a, -v0_, -v1_); });
         kd.each([&](int t, int a, float v0_, float v1_) { st2(PdKd + t * DK + a, v0_, v1_); });
         ys.each([&](int t, int a, float v0_, float v1_) { st2(PdYS + t * DK + a, v0_, v1_); });
@@ -1169,9 +1213,8 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
 #pragma unroll
     for (int r = 0; r < kMaxWT; ++r)
         if (warp + r * n_warps < n_ck) {
-            aq[r].template run<false, exact_tf32<T>()>(kC, G1T, cp, Ks, kq);
+            run2<false, false, exact_tf32<T>()>(aq[r], ak[r], kC, G1T, Asym, cp, Ks, kq);
             ak[r].template run<false, exact_tf32<T>()>(kC, G1, cp, Qs, kq);
-            ak[r].template run<false, exact_tf32<T>()>(kC, Asym, cp, Ks, kq);
         }
     __syncthreads();
     float *GQ = Ts, *GK = Ts + kC * kq;
