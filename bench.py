@@ -644,12 +644,14 @@ def bench_backward(args, inp, device, pg):
         status = gdn.device_error(device)
         n_tok = inp["q"].shape[0]
         # products of the chunked backward per (chain, 64-token chunk), full C x C tiles:
-        # 28 C^2 d + 20 C d^2 + 4 C^3 FLOP (prep 6 C^2 d; state chain forward 2 C^2 d + 4 C d^2;
-        # state adjoints 2 C^2 d + 6 C d^2; per-slice sums 10 C^2 d + 10 C d^2; dq/dk 8 C^2 d + 4 C^3)
+        # 24 C^2 d + 16 C d^2 FLOP (prep [K; Q] K^T and W: 6 C^2 d; state chain forward
+        # T V, W S, K^T U~: 2 C^2 d + 4 C d^2; state adjoints P^T dY, K dS', Q^T dY, W^T dU~:
+        # 2 C^2 d + 6 C d^2; sums over v T^T dU~, dY U~^T, X U~^T, dU~ S^T, U~ dS'^T, dY S^T:
+        # 6 C^2 d + 6 C d^2; dq/dk T^T dW, (dP o Gamma) K, (dP o Gamma)^T Q, (dA + dA^T) K: 8 C^2 d)
         C, d, H = 64, inp["q"].shape[2], inp["q"].shape[1]
         lens = (inp["cu_seqlens"][1:] - inp["cu_seqlens"][:-1]).tolist()
         n_cc = H * sum(-(-L // C) for L in lens)
-        flops = n_cc * (28 * C * C * d + 20 * C * d * d + 4 * C ** 3)
+        flops = n_cc * (24 * C * C * d + 16 * C * d * d)
         tf = flops / (ms * 1e-3) / 1e12
         # the products run as tf32 mma.sync with a two-part operand split (three tensor-core
         # products per product); peak: dense tf32 = measured bf16 x the nominal 1.1 / 2.25
@@ -661,7 +663,7 @@ def bench_backward(args, inp, device, pg):
                 "workload": "prefill shape: 4 x 4096 tokens, H=16, d=128, bf16 inputs",
                 "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf32, "unit": "TFLOP/s",
                              "frac": tf / peak_tf32, "peak_source": f"{kind} bf16_tflops x 1.1/2.25 (tf32)",
-                             "flops_per_launch": flops, "tensor_products_per_product": 3,
+                             "flops_per_launch": flops, "tensor_products_per_product": "3, or 2 (1) with one (two) bf16 input operands",
                              "fp32_fma_peak": fma_peak, "fp32_fma_frac": tf / fma_peak}}
     except Exception as exc:                      # reported, not raised
         return {"error": f"{type(exc).__name__}: {exc}"[:300]}
