@@ -4,8 +4,8 @@
 
 One step = chunked prefill (gdn_chunk_fwd) + the sigmoid-gate zero-centred RMSNorm
 epilogue (gdn_gate_norm) over one batch of the prefill workload; the same step as one
-launch with the epilogue fused into the prefill's output stage (gdn_chunk_fwd_gated) is
-timed beside it under "fused_step". The workload: 4 sequences x 4096
+library call (gdn_chunk_fwd_gated: y into o, then the gate-norm in place) is timed beside
+it under "fused_step". The workload: 4 sequences x 4096
 tokens, H = 16, d_k = d_v = 128, chunk 64, bf16 q/k/v, fp32 state. Inputs are seeded
 synthetic draws (workloads/), resident in HBM before the timed region; q, k, v and z
 (256 MiB) exceed the 126 MB L2, so no flush is needed between steps.
@@ -313,7 +313,7 @@ def run_ours(args, rank, world, local, pg):
     elapsed_ms = max_over_ranks(pg, elapsed_ms, device)
     chunk_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     gn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    # the same step as one launch with the gate-norm fused into the prefill's output stage
+    # the same step as one gdn_chunk_fwd_gated call (y into o, then the gate-norm in place)
     fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(20)]
     for e in fevs:
         fused_step(e)
@@ -352,8 +352,8 @@ def run_ours(args, rank, world, local, pg):
                      "frac": gn_bytes / (gn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "bytes_per_launch": gn_bytes}
     fused = {"ms_per_step": fused_ms,
-             "note": "the same step as one gdn_chunk_fwd_gated launch (gate-norm in the prefill's "
-                     "output stage), 20 steps"}
+             "note": "the same step as one gdn_chunk_fwd_gated call (two launches: y into o, then "
+                     "the gate-norm in place on o), 20 steps"}
 
     shapes = {} if args.no_shapes else {
         "long": bench_prefill_shape(args, "long", device, peaks, peak_kind, pg, rank),

@@ -210,10 +210,11 @@ def chunk_fwd(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk=64, scale=1.0
 def chunk_fwd_gated(q, k, v, log_alpha, beta, cu_seqlens, z, w, eps=1e-6, S0=None, chunk=64,
                     scale=1.0, cu_seqlens_host=None, out=None, final_state=True,
                     o_dtype=torch.bfloat16, state_out=None):
-    """chunk_fwd with the output epilogue fused in: returns (o, S_T or None), where
+    """chunk_fwd and the output epilogue in one library call: returns (o, S_T or None), where
     o = sigmoid(z) * y / sqrt(mean(y^2) + eps) * (1 + w) per (token, head) and y is the
-    chunk_fwd output (never written). Tensor-core path only: bf16 q, k, v and z, d = 128,
-    chunk 64 (other shapes raise GdnError GDN_ERR_UNSUPPORTED). w [d_v] fp32."""
+    chunk_fwd output in o_dtype (written into o, then normalised in place). Tensor-core path
+    only: bf16 q, k, v and z, d = 128, chunk 64 (other shapes raise GdnError
+    GDN_ERR_UNSUPPORTED). w [d_v] fp32."""
     _cuda(z, "z")
     _cuda(w, "w")
     if z.dtype != torch.bfloat16 or z.shape != v.shape:

@@ -118,8 +118,7 @@ constexpr uint32_t OFF_WB = OFF_RECV + kRecv * TP_BYTES;     // fp16 -W^T [128 k
 constexpr uint32_t OFF_YST = OFF_WB + 16384;                 // y staging: [32 t][128 v] per epilogue warpgroup
 constexpr uint32_t YST_HALF = 16384;
 constexpr uint32_t OFF_DEC = OFF_YST + 2 * YST_HALF;         // exp(g_C - g)[64] per epilogue warp
-constexpr uint32_t OFF_RS = OFF_DEC + 8 * 64 * 4;            // gated output: 1/rms of 32 tokens per warpgroup
-constexpr uint32_t OFF_BAR = OFF_RS + 2 * 32 * 4;
+constexpr uint32_t OFF_BAR = OFF_DEC + 8 * 64 * 4;
 enum {
     B_K_FULL = 0, B_K_EMPTY = B_K_FULL + kStages, B_QV_FULL = B_K_EMPTY + kStages,
     B_QV_EMPTY = B_QV_FULL + kQVStages, B_CONV = B_QV_EMPTY + kQVStages, B_RECV = B_CONV + kQVStages,
@@ -221,18 +220,14 @@ __device__ __forceinline__ uint32_t convert_rows_bf16_f16(uint8_t *tiles, int n_
 
 // ws: kWsBytesPerSm bytes per SM id below ws_slots (the K ring of the solver CTA on
 // that SM). No other scratch.
-// GATED: the output is o = sigmoid(z) * y / sqrt(mean_v y^2 + gn_eps) * (1 + gn_w) per
-// (token, head) instead of y (the output-gate equation with the zero-centred RMSNorm),
-// written through tm_y / y; z is bf16 [n_tok][H][128], gn_w fp32 [128].
-template <typename TY, bool GATED>
+template <typename TY>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
                       const float *__restrict__ log_alpha,
                       const float *__restrict__ beta, const float *__restrict__ S0,
                       const int32_t *__restrict__ cu_seqlens, int n_seq, int H, float scale,
-                      TY *__restrict__ y, float *__restrict__ S_T, uint8_t *__restrict__ ws, int ws_slots,
-                      const __nv_bfloat16 *__restrict__ z, const float *__restrict__ gn_w, float gn_eps)
+                      TY *__restrict__ y, float *__restrict__ S_T, uint8_t *__restrict__ ws, int ws_slots)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -1051,68 +1046,7 @@ chunk_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // through the group's staging tile [t][v] and one TMA store; the partial last
                 // chunk of a sequence is written row by row with plain stores (a box store
                 // would run into the next sequence's rows).
-                if constexpr (GATED) {
-                    // o = sigmoid(z) y / rms(y) (1 + w): y goes through the staging tile in
-                    // fp32, four threads sum one token's squares, and o replaces y there for
-                    // the store (full chunk) or goes out row by row (partial chunk)
-                    const int nv = n_valid - 32 * hh;           // valid tokens of this half
-                    const size_t ostride = (size_t)H * kD;
-                    const size_t row0 = (size_t)(tok0 + 32 * hh) * H + head;
-                    // z of the 32 tokens, two per register; the loads are issued here, ahead
-                    // of the staging and the sums, and first used in the output pass
-                    uint32_t zh[16];
-                    const __nv_bfloat16 *zp = z + row0 * kD + r;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t lo = 2 * i < nv ? ld_global_u16_pinned(zp + (2 * i) * ostride) : 0u;
-                        const uint32_t hi = 2 * i + 1 < nv ? ld_global_u16_pinned(zp + (2 * i + 1) * ostride) : 0u;
-                        zh[i] = lo | (hi << 16);
-                    }
-                    uint32_t ya[32];
-                    tmem_ld_x32(tmem + lane_base + TM_Y + (c & 1) * 64 + 32 * hh, ya);
-                    tmem_wait_ld();
-                    if (r == 0) bulk_wait_read();   // the previous store has read the tile
-                    named_bar_sync(nb, 128);
-                    float *yf = reinterpret_cast<float *>(smem + OFF_YST + hh * YST_HALF);
-#pragma unroll
-                    for (int jt = 0; jt < 32; ++jt) yf[jt * kD + r] = __uint_as_float(ya[jt]);
-                    named_bar_sync(nb, 128);
-                    float *rsd = reinterpret_cast<float *>(smem + OFF_RS) + 32 * hh;
-                    {
-                        const int jt = r >> 2, qd = r & 3;      // token, quarter of its 128 values
-                        float ss = 0.f;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 f = ldsf4(yf + jt * kD + 32 * qd + 4 * ((i + 2 * qd) & 7));
-                            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, fmaf(f.z, f.z, fmaf(f.w, f.w, ss))));
-                        }
-                        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-                        if (qd == 0) rsd[jt] = rsqrtf(ss * (1.0f / kD) + gn_eps);
-                    }
-                    named_bar_sync(nb, 128);              // 1/rms ready; the fp32 tile is read
-                    const float wv = 1.0f + gn_w[r];
-                    TY *os = reinterpret_cast<TY *>(smem + OFF_YST + hh * YST_HALF);
-                    TY *op = y + row0 * kD + r;
-#pragma unroll
-                    for (int jt = 0; jt < 32; ++jt) {
-                        const float zv = __uint_as_float((jt & 1) ? (zh[jt >> 1] & 0xffff0000u) : (zh[jt >> 1] << 16));
-                        const float gate = __fdividef(1.0f, 1.0f + __expf(-zv));
-                        const TY o = from_f32<TY>(gate * (__uint_as_float(ya[jt]) * rsd[jt]) * wv);
-                        if (n_valid == kC)
-                            os[jt * kD + r] = o;
-                        else if (jt < nv)
-                            op[jt * ostride] = o;
-                    }
-                    if (n_valid == kC) {
-                        fence_proxy_async_smem();
-                        named_bar_sync(nb, 128);
-                        if (r == 0) {
-                            tma_store_3d(&tm_y, os, 0, head, (int)(tok0 + 32 * hh));
-                            bulk_commit();
-                        }
-                    }
-                } else {
+                {
                     // eight tokens at a time (off the critical path: rolled). A full chunk: the
                     // staging tile, once the previous chunk's store has read it (it had a whole
                     // chunk to do so), then one TMA store; a partial one: row by row.

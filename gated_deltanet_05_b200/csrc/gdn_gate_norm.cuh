@@ -67,10 +67,12 @@ __device__ __forceinline__ float raw_elem(const uint4 *w, int i, __nv_bfloat16)
 // sigmoid(z) with the SM's approximate exponential and division (a few ulp of fp32)
 __device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 
+// y and o may be the same buffer (TY = TO): a row is written only by the lanes that read it,
+// after all of its values are in registers (its sum of squares needs them all).
 template <typename TY, typename TZ, typename TO, int DV>
 __global__ void __launch_bounds__(kGateNormThreads)
-gate_norm_kernel(const TY *__restrict__ y, const TZ *__restrict__ z, const float *__restrict__ w,
-                 int64_t n_rows, float eps, TO *__restrict__ o)
+gate_norm_kernel(const TY *y, const TZ *__restrict__ z, const float *__restrict__ w,
+                 int64_t n_rows, float eps, TO *o)
 {
     // each lane reads 32 bytes of y per row (8 fp32 or 16 bf16 elements), kept as raw words
     // until used, so that UNROLL rows per lane are in flight at a modest register cost

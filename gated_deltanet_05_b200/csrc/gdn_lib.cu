@@ -185,12 +185,11 @@ __global__ void selftest_wait_kernel(long long limit, int mode)
 constexpr int kNoAllocMaxSms = 160;
 static __device__ __align__(256) uint8_t g_noalloc_ws[(size_t)kNoAllocMaxSms * gdn::sm100::kWsBytesPerSm];
 
-template <typename TY, bool GATED = false>
+template <typename TY>
 gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const float *la,
                               const float *beta, const float *S0, const int32_t *cu, int n_seq,
                               int64_t n_tok, int H, float scale, void *y, float *S_T, void *ws,
-                              size_t ws_bytes, cudaStream_t st, const void *z = nullptr,
-                              const float *gn_w = nullptr, float gn_eps = 0.f)
+                              size_t ws_bytes, cudaStream_t st)
 {
     const int n_ids = device_sm_ids();
     if (n_ids <= 0) return GDN_ERR_CUDA;
@@ -207,15 +206,14 @@ gdn_status launch_chunk_sm100(const void *q, const void *k, const void *v, const
         return GDN_ERR_CUDA;
     const int smem = (int)gdn::sm100::SMEM_BYTES;
     if (smem > smem_optin()) return GDN_ERR_UNSUPPORTED;
-    auto kern = gdn::sm100::chunk_fwd_bf16_kernel<TY, GATED>;
+    auto kern = gdn::sm100::chunk_fwd_bf16_kernel<TY>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return GDN_ERR_CUDA;
     // one cluster of two CTAs (solver, chain) per (sequence, head) chain
     const unsigned grid = (unsigned)(2 * (int64_t)n_seq * H);
     kern<<<grid, gdn::sm100::kThreads, smem, st>>>(mq, mk, mv, my, la, beta, S0, cu, n_seq, H, scale,
                                                    static_cast<TY *>(y), S_T,
-                                                   static_cast<uint8_t *>(ws), ws_slots,
-                                                   static_cast<const __nv_bfloat16 *>(z), gn_w, gn_eps);
+                                                   static_cast<uint8_t *>(ws), ws_slots);
     return launch_status();
 }
 
@@ -368,32 +366,22 @@ gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (o_dtype != GDN_F32 && o_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (!(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
-    // the fused epilogue lives in the tensor-core kernel only
     if (in_dtype != GDN_BF16 || d_k != 128 || d_v != 128 || chunk != 64) return GDN_ERR_UNSUPPORTED;
     if (cu_seqlens_host[0] != 0) return GDN_ERR_INVALID_ARG;
     for (int i = 0; i < n_seq; ++i)
         if (cu_seqlens_host[i + 1] < cu_seqlens_host[i]) return GDN_ERR_INVALID_ARG;
     if (n_seq == 0) return GDN_OK;
     const int64_t n_tok = cu_seqlens_host[n_seq];
-    if (n_tok == 0) {
-        if (!S_T) return GDN_OK;
-        // no tokens: S_T = S0 (or 0), which the plain call writes without the epilogue
-        return gdn_chunk_fwd(q, k, v, in_dtype, log_alpha, beta, S0, cu_seqlens_dev, cu_seqlens_host,
-                             n_seq, H, d_k, d_v, chunk, scale, o, o_dtype, S_T, workspace,
-                             workspace_bytes, stream);
-    }
-    if (!q || !k || !v || !log_alpha || !beta || !z || !w || !o) return GDN_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(z, 16) ||
-        !aligned(S0, 16) || !aligned(S_T, 16) || !aligned(log_alpha, 4) || !aligned(beta, 4) ||
-        !aligned(w, 4) || !aligned(cu_seqlens_dev, 4))
-        return GDN_ERR_INVALID_ARG;
-    cudaStream_t st = as_stream(stream);
-    if (o_dtype == GDN_F32)
-        return launch_chunk_sm100<float, true>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev, n_seq, n_tok,
-                                               H, scale, o, S_T, workspace, workspace_bytes, st, z, w, eps);
-    return launch_chunk_sm100<__nv_bfloat16, true>(q, k, v, log_alpha, beta, S0, cu_seqlens_dev, n_seq,
-                                                   n_tok, H, scale, o, S_T, workspace, workspace_bytes, st,
-                                                   z, w, eps);
+    if (n_tok > 0 && (!z || !w || !o)) return GDN_ERR_INVALID_ARG;
+    if (n_tok > 0 && (!aligned(o, 16) || !aligned(z, 16) || !aligned(w, 4))) return GDN_ERR_INVALID_ARG;
+    // y into o (in o's dtype), then the gate-norm in place on o: two launches on the stream.
+    // (A gate-norm inside the prefill kernel's output stage sat on the chain CTA's per-chunk
+    // path and measured 0.52 ms against 0.28 ms for these two launches on the prefill shape.)
+    const gdn_status rc = gdn_chunk_fwd(q, k, v, in_dtype, log_alpha, beta, S0, cu_seqlens_dev,
+                                        cu_seqlens_host, n_seq, H, d_k, d_v, chunk, scale, o, o_dtype,
+                                        S_T, workspace, workspace_bytes, stream);
+    if (rc != GDN_OK || n_tok == 0) return rc;
+    return gdn_gate_norm(o, o_dtype, z, GDN_BF16, w, n_tok * H, d_v, eps, o, o_dtype, stream);
 }
 
 size_t gdn_backward_workspace_bytes(const int32_t *cu_seqlens_host, int n_seq, int H, int d_k, int d_v)

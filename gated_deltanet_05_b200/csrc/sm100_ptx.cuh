@@ -112,15 +112,6 @@ __device__ __forceinline__ void fence_proxy_async_smem()
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// A 16-bit global load that stays where it is written (volatile asm): issued early, its
-// latency overlaps the work up to its first use instead of being moved next to it.
-__device__ __forceinline__ uint16_t ld_global_u16_pinned(const void *p)
-{
-    uint16_t v;
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-    return v;
-}
-
 __device__ __forceinline__ void named_bar_sync(int id, int n_threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n_threads) : "memory");

@@ -155,9 +155,10 @@ gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, gd
 gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *stream);
 
 /*
- * gdn_chunk_fwd_gated -- gdn_chunk_fwd with the output epilogue fused into its y stage:
- * o = sigmoid(z) * RMSNorm(y) * (1 + w) per (token, head), as gdn_gate_norm defines it,
- * written instead of y (y itself never reaches memory).
+ * gdn_chunk_fwd_gated -- gdn_chunk_fwd followed by the output epilogue in one call:
+ * o = sigmoid(z) * RMSNorm(y) * (1 + w) per (token, head), as gdn_gate_norm defines it.
+ * Two launches on the stream: the prefill writes y into o (in o_dtype), then the gate-norm
+ * rewrites o in place. No buffer besides o and the workspace is used.
  *
  * Defines: the chunked prefill of gdn_chunk_fwd followed by the output-gate equation of
  * the joezjh.github.io notes ("GDN 参数化细节") with the zero-centred RMSNorm of the pwwt.cn
@@ -167,8 +168,9 @@ gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *strea
  *   o      [n_tok, H, d_v] out, o_dtype (GDN_F32 or GDN_BF16), in place of y
  * Only the tensor-core path: in_dtype GDN_BF16, d_k = d_v = 128, chunk = 64; anything else
  * returns GDN_ERR_UNSUPPORTED (call gdn_chunk_fwd then gdn_gate_norm). The workspace is
- * that of gdn_chunk_fwd. The result equals gdn_chunk_fwd + gdn_gate_norm up to fp32
- * rounding order.
+ * that of gdn_chunk_fwd. The result is bit-identical to gdn_chunk_fwd with y_dtype = o_dtype
+ * followed by gdn_gate_norm of that y (so with GDN_BF16 o, y is rounded to bf16 first).
+ * Errors: those of gdn_chunk_fwd, then those of gdn_gate_norm.
  */
 gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_dtype in_dtype,
                                const float *log_alpha, const float *beta, const float *S0,
@@ -267,7 +269,8 @@ gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dt
  * head); the mean is over its d_v elements.
  *
  *   y      [n_rows, d_v] in y_dtype;  z [n_rows, d_v] in z_dtype;  w [d_v] fp32
- *   o      [n_rows, d_v] out in o_dtype (each dtype GDN_F32 or GDN_BF16)
+ *   o      [n_rows, d_v] out in o_dtype (each dtype GDN_F32 or GDN_BF16); o may be y itself
+ *          (in place, y_dtype = o_dtype); otherwise the two do not overlap
  *   n_rows >= 0; d_v in {16, 32, 64, 128, 256}; eps > 0 recommended (1e-6)
  */
 gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dtype z_dtype,

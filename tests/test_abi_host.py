@@ -163,7 +163,7 @@ def test_chunk_fwd_gated_rejects_bad_arguments(L):
                                      kw.get("dk", 128), kw.get("dv", 128), kw.get("chunk", 64), 1.0,
                                      kw.get("z", FAKE), kw.get("w", FAKE), kw.get("eps", 1e-6),
                                      kw.get("o", FAKE), kw.get("odt", 1), None, FAKE, 1 << 24, None)
-    assert g(dt=0) == 2            # fp32 inputs: the fused epilogue is tensor-core only
+    assert g(dt=0) == 2            # fp32 inputs: the one-call form covers the tensor-core path only
     assert g(dk=64) == 2
     assert g(chunk=32) == 2
     assert g(dt=4) == 1
