@@ -119,13 +119,26 @@ featurize_kernel(const T *__restrict__ x0, const T *__restrict__ x1, const float
 
     // taps padded to four: tap kFeatMaxWidth - W + j multiplies the row W - 1 - j back
     float w4[CPL][kFeatMaxWidth];
+    if (W == kFeatMaxWidth && (reinterpret_cast<uintptr_t>(wt) & 15) == 0) {
+        // the lane's 8 x 4 taps are 32 consecutive floats: eight 16-byte loads
+        const float4 *wp = reinterpret_cast<const float4 *>(wt + ((size_t)h * D + ch0) * kFeatMaxWidth);
 #pragma unroll
-    for (int c = 0; c < CPL; ++c)
-#pragma unroll
-        for (int j = 0; j < kFeatMaxWidth; ++j) {
-            const int jj = j - (kFeatMaxWidth - W);
-            w4[c][j] = (active && jj >= 0) ? wt[((size_t)h * D + ch0 + c) * W + jj] : 0.f;
+        for (int c = 0; c < CPL; ++c) {
+            const float4 t = active ? wp[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+            w4[c][0] = t.x;
+            w4[c][1] = t.y;
+            w4[c][2] = t.z;
+            w4[c][3] = t.w;
         }
+    } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+#pragma unroll
+            for (int j = 0; j < kFeatMaxWidth; ++j) {
+                const int jj = j - (kFeatMaxWidth - W);
+                w4[c][j] = (active && jj >= 0) ? wt[((size_t)h * D + ch0 + c) * W + jj] : 0.f;
+            }
+    }
 
     const int64_t t0 = run * kFeatRun;
     const int64_t t_end = t0 + kFeatRun < n_tok ? t0 + kFeatRun : n_tok;
