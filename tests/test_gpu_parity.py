@@ -163,6 +163,24 @@ def test_gate_norm_small(dv, ydt, zdt):
     assert rel_err(f64(o16), o_ref) <= TOL["bf16"]       # a bf16 o still meets the bf16 bar
 
 
+@pytest.mark.parametrize("dv", [64, 128, 256])
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_gate_norm_in_place(dv, dt):
+    """o may be y itself (the header's in-place form, which gdn_chunk_fwd_gated uses): the
+    result is bit-identical to the out-of-place call, including a ragged last pass of rows."""
+    g = torch.Generator().manual_seed(7 + dv)
+    rows = 4096 + 37
+    y = (torch.randn(rows, dv, generator=g) * 2).to(dt).cuda()
+    z = torch.randn(rows, dv, generator=g).to(torch.bfloat16).cuda()
+    w = (torch.randn(dv, generator=g) * 0.02).cuda()
+    want = gdn.gate_norm(y, z, w, out_dtype=dt)
+    yy = y.clone()
+    got = gdn.gate_norm(yy, z, w, out=yy)
+    torch.cuda.synchronize()
+    assert got.data_ptr() == yy.data_ptr()
+    assert torch.equal(got, want)
+
+
 def test_gate_norm_prefill_workload():
     inp = W.make_prefill_inputs(W.WORKLOADS["prefill"])
     y = inp["v"].float() * 0.7                           # an fp32 y of the workload's shape
