@@ -1,5 +1,5 @@
 // gdn_backward_chunk.cuh -- gradients of the gated delta rule through its chunked form,
-// on CUDA cores in fp32.
+// fp32-accurate, with the matrix products on the tensor cores.
 //
 // The reverse of the chunkwise forward (the four-line update of the joezjh.github.io notes
 // page "Qwen3.8-Flash-Next", section "Gated DeltaNet 核心机制", rewritten chunk by chunk,
@@ -35,9 +35,11 @@
 //                           deterministic)
 //   chunk_bwd_kpart_kernel  per (chain, chunk), all at once: dQ, dK, dbeta, dlog_alpha
 // Every matrix product runs from shared memory on the tensor cores (mma.sync m16n8k8, tf32)
-// with each operand split into two tf32 parts, which keeps fp32 accuracy; a warp owns a
-// 16 x 16 block of the result. Rows in shared memory are padded to a multiple of 4 plus 4
-// floats (16-byte aligned rows; distinct banks for the fragment loads).
+// with each operand split into two tf32 parts, which keeps fp32 accuracy; an operand that is
+// an unscaled bf16 input (K, Q, V, dY) is a tf32 value already and is not split, so the
+// kernels move the scale factors (beta, gamma, D, the q scale) onto the other operand or onto
+// the result. A warp owns a 16 x 16 block of the result. Rows in shared memory are padded to
+// a multiple of 4 plus 4 floats (16-byte aligned rows; distinct banks for the fragment loads).
 #pragma once
 #include "gdn_common.cuh"
 #include "sm100_ptx.cuh"
