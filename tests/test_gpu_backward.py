@@ -70,6 +70,31 @@ def test_backward_matches_oracle(lens, H, dk, dv, dtype, with_state):
         assert err <= 1e-4, f"{name}: {err:.3e}"
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_degenerate_gates(dtype):
+    """Degenerate gates at d = 128: beta in {0, 1} (tokens that write nothing, and full-strength
+    writes) and log alpha in {0, -30} (no decay, and a decay whose cumulative sum underflows
+    exp within a chunk), with S0 and dS_T present, against the oracle at the same bar."""
+    lens, H, d = (150, 64, 7), 2, 128
+    P = _case(lens, H, d, d, dtype, seed=77, with_state=True)
+    rng = np.random.default_rng(78)
+    N = sum(lens)
+    P["beta"] = torch.from_numpy(rng.choice([0.0, 1.0], size=(N, H)).astype(np.float32))
+    P["log_alpha"] = torch.from_numpy(rng.choice([0.0, -30.0], size=(N, H), p=[0.9, 0.1]).astype(np.float32))
+    dev = {n: (t.cuda() if t is not None else None) for n, t in P.items()}
+    got = gdn.backward(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], dev["cu"], dev["dy"],
+                       S0=dev["S0"], dS_T=dev["dS_T"], scale=0.7, cu_seqlens_host=P["cu"])
+    torch.cuda.synchronize()
+    ref = oracle.backward(P["q"], P["k"], P["v"], P["log_alpha"], P["beta"], P["cu"].numpy(), P["dy"],
+                          S0=oracle.state_from_lib(P["S0"]), dS_T=oracle.state_from_lib(P["dS_T"]), scale=0.7)
+    for name, g, r in zip(("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"), got, ref):
+        if name == "dS0":
+            r = oracle.state_to_lib(r)
+        assert torch.isfinite(g).all(), name
+        err = rel_err(f64(g), r)
+        assert err <= 1e-4, f"{name}: {err:.3e}"
+
+
 def test_backward_full_size_sampled_chains():
     """The prefill workload's shape (4 x 4096 tokens, H = 16, d = 128, bf16), as `bench.py`
     times it: every gradient finite, and the gradients of sampled (sequence, head) chains

@@ -49,6 +49,19 @@ def test_bf16_strong_decay():
     check_prefill(inp)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_degenerate_gates(dtype):
+    """beta in {0, 1} and log alpha in {0, -30} per token (no decay, and a decay whose
+    cumulative sum underflows exp within a chunk), S0 != 0: the tensor-core path (bf16) and
+    the fp32 chunk kernel against the oracle."""
+    inp = custom(dtype, (200, 64, 5), 2, 128, 64, seed=21, s0_std=0.02)
+    rng = np.random.default_rng(22)
+    shape = tuple(inp["beta"].shape)
+    inp["beta"] = torch.from_numpy(rng.choice([0.0, 1.0], size=shape).astype(np.float32))
+    inp["log_alpha"] = torch.from_numpy(rng.choice([0.0, -30.0], size=shape, p=[0.9, 0.1]).astype(np.float32))
+    check_prefill(inp)
+
+
 def test_bf16_without_final_state():
     inp = custom("bf16", (130,), 2, 128, 64, seed=13)
     y, S_T = run_prefill(inp, final_state=False)
