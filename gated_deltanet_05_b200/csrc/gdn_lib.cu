@@ -374,6 +374,10 @@ gdn_status gdn_chunk_fwd_gated(const void *q, const void *k, const void *v, gdn_
     const int64_t n_tok = cu_seqlens_host[n_seq];
     if (n_tok > 0 && (!z || !w || !o)) return GDN_ERR_INVALID_ARG;
     if (n_tok > 0 && (!aligned(o, 16) || !aligned(z, 16) || !aligned(w, 4))) return GDN_ERR_INVALID_ARG;
+    if (n_tok > 0) {                    // z is read after o is written: they must not overlap
+        const uintptr_t z0 = (uintptr_t)z, o0 = (uintptr_t)o, n = (uintptr_t)n_tok * H * d_v;
+        if (z0 < o0 + n * (o_dtype == GDN_F32 ? 4u : 2u) && o0 < z0 + n * 2u) return GDN_ERR_INVALID_ARG;
+    }
     // y into o (in o's dtype), then the gate-norm in place on o: two launches on the stream.
     // (A gate-norm inside the prefill kernel's output stage sat on the chain CTA's per-chunk
     // path and measured 0.52 ms against 0.28 ms for these two launches on the prefill shape.)
@@ -657,6 +661,17 @@ gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dt
     if (!y || !z || !w || !o) return GDN_ERR_INVALID_ARG;
     if (!aligned(y, 16) || !aligned(z, 16) || !aligned(o, 16) || !aligned(w, 4))
         return GDN_ERR_INVALID_ARG;
+    // o may be y itself with the same dtype (in place); otherwise o overlaps neither y nor z
+    {
+        auto bytes = [&](gdn_dtype dt) { return (uintptr_t)n_rows * (uintptr_t)d_v * (dt == GDN_F32 ? 4u : 2u); };
+        auto overlap = [](const void *a, uintptr_t na, const void *b, uintptr_t nb) {
+            const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+            return a0 < b0 + nb && b0 < a0 + na;
+        };
+        const uintptr_t ob = bytes(o_dtype);
+        if (y == o ? y_dtype != o_dtype : overlap(y, bytes(y_dtype), o, ob)) return GDN_ERR_INVALID_ARG;
+        if (overlap(z, bytes(z_dtype), o, ob)) return GDN_ERR_INVALID_ARG;
+    }
     cudaStream_t st = as_stream(stream);
     int dev = 0, n_sm = 148;
     cudaGetDevice(&dev);

@@ -165,7 +165,8 @@ gdn_status gdn_selftest_bounded_wait(int64_t limit_cycles, int mode, void *strea
  * translation (section 2.1.1); the same arguments as gdn_chunk_fwd, plus
  *   z      [n_tok, H, d_v] bf16 (the projected gate logits)
  *   w      [d_v] fp32 (stored zero-centred weight; the scale is 1 + w);  eps >= 0 (1e-6)
- *   o      [n_tok, H, d_v] out, o_dtype (GDN_F32 or GDN_BF16), in place of y
+ *   o      [n_tok, H, d_v] out, o_dtype (GDN_F32 or GDN_BF16), in place of y; it must not
+ *          overlap z (GDN_ERR_INVALID_ARG, checked before any launch)
  * Only the tensor-core path: in_dtype GDN_BF16, d_k = d_v = 128, chunk = 64; anything else
  * returns GDN_ERR_UNSUPPORTED (call gdn_chunk_fwd then gdn_gate_norm). The workspace is
  * that of gdn_chunk_fwd. The result is bit-identical to gdn_chunk_fwd with y_dtype = o_dtype
@@ -270,7 +271,8 @@ gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v, gdn_dt
  *
  *   y      [n_rows, d_v] in y_dtype;  z [n_rows, d_v] in z_dtype;  w [d_v] fp32
  *   o      [n_rows, d_v] out in o_dtype (each dtype GDN_F32 or GDN_BF16); o may be y itself
- *          (in place, y_dtype = o_dtype); otherwise the two do not overlap
+ *          (in place, y_dtype = o_dtype); otherwise o overlaps neither y nor z
+ *          (GDN_ERR_INVALID_ARG, checked on the host before any launch)
  *   n_rows >= 0; d_v in {16, 32, 64, 128, 256}; eps > 0 recommended (1e-6)
  */
 gdn_status gdn_gate_norm(const void *y, gdn_dtype y_dtype, const void *z, gdn_dtype z_dtype,

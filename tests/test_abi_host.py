@@ -152,6 +152,20 @@ def test_backward_rejects_bad_arguments(L):
     assert bw(n_seq=0) == 0
 
 
+def test_gate_norm_buffer_overlap(L):
+    """o may be y itself with y's dtype (in place); any other overlap of o with y or z is
+    rejected before a launch. 10 rows of d_v = 128: 2,560 bytes in bf16, 5,120 in fp32."""
+    Y, Z = 0x100000, 0x200000
+    p = ctypes.c_void_p
+    gn = lambda y, ydt, z, o, odt: L.gdn_gate_norm(p(y), ydt, p(z), 1, FAKE, 10, 128, 1e-6, p(o), odt, None)
+    assert gn(Y, 1, Z, Y, 0) == 1                 # in place needs one dtype
+    assert gn(Y, 1, Z, Y + 2544, 1) == 1          # o starts inside y
+    assert gn(Y + 2544, 1, Z, Y, 1) == 1          # y starts inside o
+    assert gn(Y, 0, Z, Y + 4096, 1) == 1          # fp32 y reaches into o
+    assert gn(Y, 1, Z, Z + 16, 1) == 1            # o overlaps z
+    assert gn(Y, 1, Y, Y, 1) == 1                 # z is o
+
+
 def test_chunk_fwd_gated_rejects_bad_arguments(L):
     cu = (ctypes.c_int32 * 3)(0, 64, 100)
     cu_bad = (ctypes.c_int32 * 3)(0, 64, 10)
@@ -175,6 +189,7 @@ def test_chunk_fwd_gated_rejects_bad_arguments(L):
     assert g(w=None) == 1
     assert g(o=None) == 1
     assert g(o=ctypes.c_void_p(0x10008)) == 1
+    assert g(z=ctypes.c_void_p(0x20000), o=ctypes.c_void_p(0x20010)) == 1   # o overlaps z
     assert g(n_seq=0) == 0
 
 
