@@ -1014,11 +1014,12 @@ chunk_bwd_vpart_kernel(const T *__restrict__ v, const T *__restrict__ dy, const 
         kd.each([&](int t, int a, float v0_, float v1_) { st2(PdKd + t * DK + a, v0_, v1_); });
         ys.each([&](int t, int a, float v0_, float v1_) { st2(PdYS + t * DK + a, v0_, v1_); });
     }
-    // <dS', S> over this slice
+    // <dS', S> over this slice (four columns per step)
     float sd = 0.f;
-    for (int i = tid; i < DK * DVT; i += blockDim.x) {
-        const int a = i / DVT, b = i % DVT;
-        sd = fmaf(dSs[a * vq + b], Ss[a * vq + b], sd);
+    for (int i = tid; i < DK * nvq; i += blockDim.x) {
+        const int a = i / nvq, b = (i % nvq) * 4;
+        const float4 x = f4(dSs + a * vq + b), y = f4(Ss + a * vq + b);
+        sd = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, sd))));
     }
     sd = group_sum<32>(sd);
     if ((tid & 31) == 0) red[tid >> 5] = sd;
@@ -1230,9 +1231,9 @@ chunk_bwd_kpart_kernel(const T *__restrict__ q, const T *__restrict__ k, const f
     // dQ = diag(gamma) dY S^T + (dP o Gamma) K;
     // dK = (dP o Gamma)^T Q + (dA + dA^T) K + diag(beta gamma) T^T dW + diag(D) dK~;
     // a warp per row t, four consecutive a per lane, with the row sums for dbeta and
-    // dlog_alpha; two rows at a time so that their loads are in flight together
+    // dlog_alpha; the warp's four rows at once so that all their loads are in flight together
     const int lane = tid & 31;
-#pragma unroll 2
+#pragma unroll 4
     for (int t = warp; t < kC; t += n_warps) {
         float rg = 0.f, rb = 0.f, rd = 0.f;
         for (int a = 4 * lane; a < DK; a += 128) {
